@@ -1,0 +1,253 @@
+/*
+ * fl.h -- C ABI of the variable-precision weight read path (libfl.so, sm_100a).
+ *
+ * A linear layer's weights are stored once as 8-bit codes split into four
+ * 2-bit planes; every 64-output-row block is read at its own depth
+ * (ZERO, D2, D4, D6, D8) straight from that one copy, a D4 pass can be
+ * escalated to D8 by adding the low planes, an entropy / top-two-margin gate
+ * over the logits decides which steps escalate, and GGUF-style Q4_K / Q6_K
+ * super-blocks are dequantized inside the product.
+ *
+ * Sources (page title, section):
+ *   [FoQLens]  "FoQLens" landing page: progress table ("a format of our own":
+ *              2, 4, 6 or 8 bits read from one copy without repacking; "the
+ *              card reads a layout inside the pass": each block of rows read
+ *              to its own depth) and the FoQZones mechanism.
+ *   [Lens]     "Precision where the question is, not everywhere", section
+ *              "The mechanism", rules 1-7, ladder ZERO < D2 < D4 < D6 < D8.
+ *   [PoD]      "Precision on Demand: Escalating Weight Bits at Uncertain
+ *              Decoding Steps in a Small Local Model", abstract.
+ *   [Ember]    "v0.3, quantized on disk, quantized in memory": GGUF K-quant
+ *              layouts, per-tensor dispatch with no silent fallback,
+ *              validated construction, dequantize only at block granularity
+ *              inside the matmul.
+ *
+ * Conventions for every call:
+ *   - Pointers named as device pointers must point to device memory of the
+ *     current CUDA device; the caller owns all buffers. The library never
+ *     allocates device or host memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Argument, shape and alignment errors are detected on
+ *     the host before anything is launched and are returned synchronously;
+ *     a failed launch returns FL_ERR_CUDA. Nothing falls back to another
+ *     path: unsupported inputs fail.
+ *   - fl_last_error() returns a message describing the most recent failure
+ *     on the calling thread.
+ *   - bf16 activations are passed as their 16-bit patterns (uint16_t).
+ *   - Batch (tokens per call) is 1..16; activations are row-major
+ *     [batch][in], outputs row-major [batch][out] fp32.
+ */
+#ifndef FL_H_
+#define FL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FL_OK = 0,
+  FL_ERR_ARG = -1,          /* null pointer, bad count, bad parameter value    */
+  FL_ERR_SHAPE = -2,        /* out/in/batch/vocab outside what the call takes  */
+  FL_ERR_UNSUPPORTED = -3,  /* a weight type the fast path does not implement  */
+  FL_ERR_ALIGN = -4,        /* a pointer is not aligned as the call requires   */
+  FL_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed            */
+  FL_ERR_WORKSPACE = -6     /* workspace missing or smaller than required      */
+} fl_status;
+
+#define FL_MAX_BATCH 16
+#define FL_MAX_STOPS 16
+#define FL_MAX_PROBLEMS 256
+
+/* GGUF tensor type ids of the two K-quant formats on the fast path ([Ember],
+ * GGUF layouts: Q2_K = 10 ... Q6_K = 14). */
+#define FL_GGML_Q4_K 12
+#define FL_GGML_Q6_K 14
+
+const char* fl_status_string(int status);
+const char* fl_last_error(void);
+int fl_version(void);
+
+/* ========================================================================= */
+/* Plane store ([FoQLens] progress table, "a format of our own": one stored   */
+/* stack, a base with refinements, any depth read from the same copy).       */
+/*                                                                           */
+/* Layout (this library's own): per block b of 64 rows, 8448 * G bytes with  */
+/* G = in / 128 column groups:                                               */
+/*   [0, 256 G)                         fp32 scale of (group g, row r) at    */
+/*                                      byte 4 (64 g + r)                    */
+/*   256 G + 2048 (G k + g) + 32 r      32 bytes of plane k (0 = top bits)   */
+/*                                      for group g, row r                   */
+/* A block read at depth d is the contiguous prefix of 256 G + 1024 G d      */
+/* bytes. Inside the 32 bytes of (k, g, r) the 128 columns are four          */
+/* little-endian 32-bit words of 16 columns; column j of word w holds        */
+/* p_k = (u >> (6 - 2k)) & 3 of u = code + 128 at bit                        */
+/* (8 (j % 4) + 6 - 2 k + 2 (j / 4)) mod 32.                                 */
+/* ========================================================================= */
+
+/* Bytes of the plane store of an out x in layer (out % 64 == 0, in % 128 == 0);
+ * 0 for an invalid shape. */
+size_t fl_plane_store_bytes(int out, int in);
+
+/* Pack int8 codes and their scales into the plane store.
+ *   codes  device, int8 [out][in] row-major, values in [-128, 127]
+ *   scales device, fp32 [out][in / 128] row-major (one scale per row per
+ *          128-column group)
+ *   store  device, fl_plane_store_bytes(out, in) bytes, 16-byte aligned;
+ *          fully overwritten.
+ * out % 64 == 0 and in % 128 == 0, else FL_ERR_SHAPE. Bit-exact. */
+fl_status fl_pack_planes(const int8_t* codes, const float* scales, int out, int in, uint8_t* store, void* stream);
+
+/* A packed layer: device pointer to its plane store and its shape. */
+typedef struct {
+  const uint8_t* store;
+  int out;
+  int in;
+} fl_plane_weight;
+
+/* ========================================================================= */
+/* Level map ([Lens] "The mechanism", rules 1-6).                            */
+/*   R_i = r_i f / (1 - f);  kappa = gamma + floor(g (m - gamma));           */
+/*   rho_i = |xy_b - c_i| / R_i;  L_i = max(0, 1 - rho_i / s_last);          */
+/*   L = min(1, sum_i L_i) (combine 0) or max_i L_i (combine 1);             */
+/*   rho* = s_last (1 - L); level = the ring rho* falls into, where ring j   */
+/*   covers [s_(j+1), s_j) with s_(kappa+1) = 0; outside every lens: gamma.  */
+/* Distance is Euclidean in the plane. R = 0 gives rho = 0 on a centre and   */
+/* +inf elsewhere. kappa == gamma (no rings) puts every block at gamma.      */
+/* Every operation is an IEEE-rounded fp32 operation in the order above      */
+/* (no fused multiply-add), so levels are reproducible bit for bit.          */
+/* ========================================================================= */
+typedef struct {
+  float f;                     /* focus area, 0 <= f < 1                     */
+  float g;                     /* focus strength, 0 <= g <= 1                */
+  int gamma;                   /* glass level, 0 <= gamma <= m               */
+  int m;                       /* top ladder index, 1 <= m <= 15             */
+  int nstops;                  /* must equal kappa - gamma                   */
+  float stops[FL_MAX_STOPS];   /* s_kappa < ... < s_(gamma+1), ascending, > 0 */
+  int combine;                 /* 0 = sum clamped to 1, 1 = max              */
+} fl_lens_params;
+
+/* xy      device, fp32 [nblocks][2] block coordinates
+ * centers device, fp32 [nlenses][2]; radii device, fp32 [nlenses] (r_i >= 0)
+ * levels  device, uint8 [nblocks] (output, level index 0..m)
+ * counts  device, uint32 [m + 1] or NULL: per-level block counts are ADDED
+ *         to it (the caller zeroes it first).
+ * nblocks >= 0, 0 <= nlenses <= 64. */
+fl_status fl_level_map(const float* xy, int nblocks, const float* centers, const float* radii, int nlenses,
+                       const fl_lens_params* params, uint8_t* levels, uint32_t* counts, void* stream);
+
+/* ========================================================================= */
+/* Depth GEMV / skinny GEMM ([FoQLens] "the card reads a layout inside the   */
+/* pass"; [PoD] top bits of 8-bit weights).                                  */
+/*   y[t][r] = sum_c w_d[r][c] x[t][c],  d = 2 * levels[r / 64],             */
+/*   w_d = s[r][c / 128] (u_d - 128 + c_d), u_d = u with its low 8 - d bits  */
+/*   cleared, c_d = (2^(8-d) - 1) / 2; a ZERO block gives y = 0.             */
+/* Arithmetic: codes enter an int8 tensor-core product exactly; x enters as  */
+/* a 15-bit fixed-point value per 128-column group (|error| <= 2^-14 of the  */
+/* group's max |x|); products accumulate in int32 per group and in fp32      */
+/* across groups.                                                            */
+/*                                                                           */
+/* levels   device, uint8 [out / 64], values 0..4 (0 ZERO .. 4 D8); values   */
+/*          above 4 are read as 4.                                           */
+/* x        device, bf16 [batch][in], 16-byte aligned; batch 1..16           */
+/* y        device, fp32 [batch][out]; overwritten                           */
+/* workspace device scratch for splitting a layer's columns across CTAs:     */
+/*          at least fl_gemv_workspace_bytes(out, in, batch) bytes, 16-byte  */
+/*          aligned, ZERO-FILLED before its first use; every successful call */
+/*          leaves it zero-filled again. Calls that share a workspace must   */
+/*          not overlap on the GPU. May be NULL when the size is 0.          */
+/* ========================================================================= */
+size_t fl_gemv_workspace_bytes(int out, int in, int batch);
+
+fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, const uint16_t* x, int batch, float* y,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Escalation residual ([PoD]: redo a step at 8 bits, written as an addition
+ * to the low pass):  y[t][r] += sum_c (w_b - w_a)[r][c] x[t][c]  with
+ * a = 2 from_levels[blk], b = 2 to_levels[blk], w_0 = 0. Reads only planes
+ * a/2 .. b/2 - 1. The levels live on the device, so the host cannot check
+ * them: a block whose to-level is not above its from-level adds nothing.
+ * Same arguments as fl_gemv_depth. */
+fl_status fl_gemv_residual(const fl_plane_weight* w, const uint8_t* from_levels, const uint8_t* to_levels,
+                           const uint16_t* x, int batch, float* y, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Several independent layers in one launch (a decode step's GEMVs).
+ * mode 0: depth GEMV (y =), levels = the depth map, to_levels unused.
+ * mode 1: residual (y +=), levels = from-levels, to_levels = to-levels.
+ * Problems are not split across CTAs, so no workspace is used. 1 <= n <=
+ * FL_MAX_PROBLEMS; all problems share `batch`. */
+typedef struct {
+  fl_plane_weight w;
+  const uint8_t* levels;
+  const uint8_t* to_levels;
+  const uint16_t* x;
+  float* y;
+} fl_gemv_problem;
+
+fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream);
+
+/* ========================================================================= */
+/* Uncertainty gate ([PoD]: redo at 8 bits when the low-precision output     */
+/* distribution looks uncertain: entropy above a threshold or a small        */
+/* top-two margin).  Per row t of logits z:                                  */
+/*   m = max z, S = sum e^(z - m), T = sum (z - m) e^(z - m),                */
+/*   entropy = ln S - T / S (nats),  i1, i2 = indices of the two largest     */
+/*   logits (ties to the lower index), margin = p1 - p2 = (1 - e^(z_i2-m))/S,*/
+/*   escalate = (entropy > tau_h) || (margin < tau_m).                       */
+/* logits device fp32 [batch][vocab], 16-byte aligned, vocab % 4 == 0,      */
+/* 4 <= vocab <= 2^24; outputs device: entropy, margin fp32 [batch], top2 int32   */
+/* [batch][2], escalate uint8 [batch]. fp32 arithmetic.                      */
+/* ========================================================================= */
+fl_status fl_logit_gate(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,
+                        float* margin, int32_t* top2, uint8_t* escalate, void* stream);
+
+/* ========================================================================= */
+/* K-quant GEMV ([Ember]: Q4_K / Q6_K native kernels, dequantize only at     */
+/* block granularity inside the product, per-tensor dispatch, unsupported    */
+/* types fail). Records of 256 weights, row-major [out][in / 256]; the value */
+/* rules are GGUF's, the byte layout is this library's own with the GGUF     */
+/* byte counts:                                                              */
+/*   Q4_K 144 B, sub-blocks j of 32: [0,2) d fp16, [2,4) dmin fp16,          */
+/*        byte 4 + j = sc_j | (mn_j & 3) << 6, nibble j of the word at 12 =   */
+/*        mn_j >> 2, byte 16 + 16 j + b = q[32 j + b] | q[32 j + 16 + b] << 4;*/
+/*        w = d sc_j q - dmin mn_j.                                          */
+/*   Q6_K 210 B, sub-blocks j of 16, q in 0..63: a record at an even place n */
+/*        in its row is [q area 192][sc_j int8 x16][d fp16], at an odd place */
+/*        [d fp16][q area 192][sc_j int8 x16]; q area: chunk t (48 B) x      */
+/*        group m (12 B = words A, B, C), W(j, L) = 16 j + 4 t + L:          */
+/*        A byte L = lo4 q[W(4m,L)] | lo4 q[W(4m+1,L)] << 4,                 */
+/*        B byte L = lo4 q[W(4m+2,L)] | lo4 q[W(4m+3,L)] << 4,               */
+/*        C byte L = hi2 q[W(4m+2,L)] | hi2 q[W(4m+3,L)] << 2                */
+/*                 | hi2 q[W(4m,L)] << 4 | hi2 q[W(4m+1,L)] << 6;            */
+/*        w = d sc_j (q - 32).                                               */
+/* blocks: device, 16-byte aligned; in % 256 == 0, and in % 2048 == 0 for    */
+/* Q6_K (rows then start 16-byte aligned and hold an even record count).     */
+/* ggml_type other than FL_GGML_Q4_K / FL_GGML_Q6_K -> FL_ERR_UNSUPPORTED.    */
+/* Same x / y / workspace rules as fl_gemv_depth.                            */
+/* ========================================================================= */
+size_t fl_kquant_bytes(int ggml_type, int out, int in);
+size_t fl_kquant_workspace_bytes(int ggml_type, int out, int in, int batch);
+
+fl_status fl_gemv_kquant(const void* blocks, int ggml_type, int out, int in, const uint16_t* x, int batch, float* y,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+typedef struct {
+  const void* blocks;
+  int ggml_type;
+  int out;
+  int in;
+  const uint16_t* x;
+  float* y;
+} fl_kquant_problem;
+
+/* Several K-quant tensors in one launch (a decode step); no workspace. */
+fl_status fl_gemv_kquant_batched(const fl_kquant_problem* problems, int n, int batch, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FL_H_ */

@@ -141,8 +141,9 @@ ORC_API double orc_dequant_depth(int8_t q, float s, int depth) {
   return (double)s * recon_code(q, depth);
 }
 
-/* Ladder: level l in {0..4} reads 2*l bits (ZERO, D2, D4, D6, D8). */
-static int level_bits(uint8_t level) { return 2 * (int)level; }
+/* Ladder: level l in {0..4} reads 2*l bits (ZERO, D2, D4, D6, D8); a level
+ * above 4 is read as 4 (library convention for out-of-range map entries). */
+static int level_bits(uint8_t level) { return 2 * (level > 4 ? 4 : (int)level); }
 
 /* y[t][r] = sum_c w_d(b(r))[r][c] * x[t][c], d = bits of levels[r / 64].    */
 ORC_API void orc_gemv_depth(const int8_t* q, const float* s, int out, int in, const uint8_t* levels,
@@ -168,7 +169,7 @@ ORC_API void orc_gemv_depth(const int8_t* q, const float* s, int out, int in, co
 /* Escalation residual: dy[t][r] = sum_c (w_b - w_a)[r][c] x[t][c] with      */
 /* a = bits(from_levels[blk]), b = bits(to_levels[blk]), w_0 = 0.            */
 /* ([Precision on Demand]: the redo at 8 bits written as an addition to the  */
-/* low pass.)                                                                */
+/* low pass.) Escalation only raises depth: a block with b <= a adds 0.      */
 ORC_API void orc_gemv_residual(const int8_t* q, const float* s, int out, int in, const uint8_t* from_levels,
                                const uint8_t* to_levels, const uint16_t* x, int batch, double* dy,
                                int nthreads) {
@@ -180,7 +181,7 @@ ORC_API void orc_gemv_residual(const int8_t* q, const float* s, int out, int in,
     int b = level_bits(to_levels[r / 64]);
     for (int t = 0; t < batch; ++t) {
       double acc = 0.0;
-      for (int c = 0; c < in; ++c) {
+      for (int c = 0; c < in && b > a; ++c) {
         int8_t qq = q[(size_t)r * in + c];
         double sc = (double)s[(size_t)r * G + c / 128];
         double dw = sc * recon_code(qq, b) - sc * recon_code(qq, a);
@@ -367,50 +368,66 @@ ORC_API void orc_logit_gate(const float* logits, int vocab, int batch, double ta
 
 /* ------------------------------------------------------------------------ */
 /* K-quant super-blocks ([Ember v0.3], GGUF layouts; dequantized per block    */
-/* inside the product). Byte layout is our own with the GGUF byte counts.    */
+/* inside the product). The value rules are GGUF's; the byte layout is our    */
+/* own with the GGUF byte counts (144 and 210 bytes per 256 weights).        */
 /*                                                                           */
-/* Q4_K, 144 bytes, 256 weights = 8 sub-blocks of 32:                        */
+/* Q4_K, 144 bytes, 8 sub-blocks j of 32 weights:                            */
 /*   [0,2) d fp16   [2,4) dmin fp16                                          */
-/*   [4,8)  sc_j low 4 bits, nibble j    [8,12) mn_j low 4 bits, nibble j     */
-/*   [12,16) high 2 bits: sc_j at bits 2j, mn_j at bits 16 + 2j              */
-/*   [16,144) q_i (4 bits), weight i in byte 16 + i/2, low nibble if i even   */
-/*   w_i = d * sc_j * q_i - dmin * mn_j,  j = i / 32                         */
-/* Q6_K, 210 bytes, 256 weights = 16 sub-blocks of 16:                       */
-/*   [0,128) low 4 bits of q_i, byte i/2, low nibble if i even                */
-/*   [128,192) high 2 bits of q_i, byte 128 + i/4, bits 2 (i % 4)             */
-/*   [192,208) sc_j int8     [208,210) d fp16                                */
-/*   w_i = d * sc_j * (q_i - 32),  j = i / 16                                */
+/*   [4,12)  byte 4 + j  = sc_j | (mn_j & 3) << 6                            */
+/*   [12,16) nibble j of the little-endian word (bits 4j..4j+3) = mn_j >> 2   */
+/*   [16,144) byte 16 + 16 j + b (b = 0..15): low nibble = q of weight        */
+/*            32 j + b, high nibble = q of weight 32 j + 16 + b              */
+/*   w = d * sc_j * q - dmin * mn_j                                          */
+/* Q6_K, 210 bytes, 16 sub-blocks j of 16 weights, 6-bit q (0..63).          */
+/*   A record's place n in its row decides where the 192-byte q area sits:    */
+/*   n even: [0,192) q, [192,208) sc_j int8, [208,210) d fp16                */
+/*   n odd:  [0,2) d fp16, [2,194) q, [194,210) sc_j int8                    */
+/*   q area: chunk t (0..3) = bytes [48 t, 48 t + 48), group m (0..3) =       */
+/*   12 bytes at 48 t + 12 m = words A, B, C; with W(j, L) = 16 j + 4 t + L:  */
+/*     A byte L = lo4 q[W(4m, L)]   | lo4 q[W(4m+1, L)] << 4                  */
+/*     B byte L = lo4 q[W(4m+2, L)] | lo4 q[W(4m+3, L)] << 4                  */
+/*     C byte L = hi2 q[W(4m+2, L)] | hi2 q[W(4m+3, L)] << 2                  */
+/*              | hi2 q[W(4m, L)] << 4 | hi2 q[W(4m+1, L)] << 6               */
+/*   w = d * sc_j * (q - 32)                                                 */
 /* ------------------------------------------------------------------------ */
 static uint16_t rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
-static uint32_t rd32(const uint8_t* p) {
-  return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
-}
 
 ORC_API void orc_dequant_q4k(const uint8_t* blk, double* w) {
   double d = fp16_to_double(rd16(blk));
   double dmin = fp16_to_double(rd16(blk + 2));
-  uint32_t lo_sc = rd32(blk + 4), lo_mn = rd32(blk + 8), hi = rd32(blk + 12);
-  for (int i = 0; i < 256; ++i) {
-    int j = i / 32;
-    int sc = (int)((lo_sc >> (4 * j)) & 15) | (int)(((hi >> (2 * j)) & 3) << 4);
-    int mn = (int)((lo_mn >> (4 * j)) & 15) | (int)(((hi >> (16 + 2 * j)) & 3) << 4);
-    uint8_t byte = blk[16 + i / 2];
-    int qv = (i % 2 == 0) ? (byte & 15) : (byte >> 4);
-    w[i] = d * (double)sc * (double)qv - dmin * (double)mn;
+  for (int j = 0; j < 8; ++j) {
+    int sc = blk[4 + j] & 63;
+    int mnlo = blk[4 + j] >> 6;
+    int nib = (j % 2 == 0) ? (blk[12 + j / 2] & 15) : (blk[12 + j / 2] >> 4);
+    int mn = mnlo | (nib << 2);
+    for (int b = 0; b < 16; ++b) {
+      uint8_t byte = blk[16 + 16 * j + b];
+      w[32 * j + b] = d * (double)sc * (double)(byte & 15) - dmin * (double)mn;
+      w[32 * j + 16 + b] = d * (double)sc * (double)(byte >> 4) - dmin * (double)mn;
+    }
   }
 }
 
-ORC_API void orc_dequant_q6k(const uint8_t* blk, double* w) {
-  double d = fp16_to_double(rd16(blk + 208));
-  for (int i = 0; i < 256; ++i) {
-    int j = i / 16;
-    int sc = (int)(int8_t)blk[192 + j];
-    uint8_t lb = blk[i / 2];
-    int lo = (i % 2 == 0) ? (lb & 15) : (lb >> 4);
-    int hi2 = (blk[128 + i / 4] >> (2 * (i % 4))) & 3;
-    int qv = lo | (hi2 << 4);
-    w[i] = d * (double)sc * (double)(qv - 32);
+ORC_API void orc_dequant_q6k(const uint8_t* blk, int odd, double* w) {
+  const uint8_t* q = blk + (odd ? 2 : 0);
+  const uint8_t* sc = blk + (odd ? 194 : 192);
+  double d = fp16_to_double(rd16(blk + (odd ? 0 : 208)));
+  int code[256];
+  for (int t = 0; t < 4; ++t) {
+    for (int m = 0; m < 4; ++m) {
+      const uint8_t* A = q + 48 * t + 12 * m;
+      const uint8_t* B = A + 4;
+      const uint8_t* C = A + 8;
+      for (int L = 0; L < 4; ++L) {
+        int j0 = 4 * m, j1 = 4 * m + 1, j2 = 4 * m + 2, j3 = 4 * m + 3;
+        code[16 * j0 + 4 * t + L] = (A[L] & 15) | (((C[L] >> 4) & 3) << 4);
+        code[16 * j1 + 4 * t + L] = (A[L] >> 4) | (((C[L] >> 6) & 3) << 4);
+        code[16 * j2 + 4 * t + L] = (B[L] & 15) | ((C[L] & 3) << 4);
+        code[16 * j3 + 4 * t + L] = (B[L] >> 4) | (((C[L] >> 2) & 3) << 4);
+      }
+    }
   }
+  for (int i = 0; i < 256; ++i) w[i] = d * (double)(int8_t)sc[i / 16] * (double)(code[i] - 32);
 }
 
 /* GGUF type ids for the two formats on the fast path. */
@@ -439,7 +456,7 @@ ORC_API int orc_gemv_kquant(const uint8_t* blocks, int type, int out, int in, co
       if (type == ORC_Q4_K)
         orc_dequant_q4k(blk, w);
       else
-        orc_dequant_q6k(blk, w);
+        orc_dequant_q6k(blk, sb & 1, w);
       for (int t = 0; t < batch; ++t)
         for (int i = 0; i < 256; ++i) acc[t] += w[i] * bf16_to_double(x[(size_t)t * in + 256 * sb + i]);
     }

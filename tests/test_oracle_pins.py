@@ -334,46 +334,53 @@ def test_gate_tie_goes_to_lower_index(orc):
 
 # ----------------------------------------------------------------------------- K-quant
 
-def _record(spec, n):
+def _record(pairs, n):
     rec = np.zeros(n, np.uint8)
-    for off, val in spec["set_bytes"]:
+    for off, val in pairs:
         rec[off] = val
     return rec
 
 
 def test_kquant_hand_built_superblocks(orc, golden):
     g = golden("kquant_superblocks.json")
-    w4 = orc.dequant_superblock(_record(g["q4k"], 144), orc.Q4_K)
+    w4 = orc.dequant_superblock(_record(g["q4k"]["set_bytes"], 144), orc.Q4_K)
     for i, v in g["q4k"]["expect"].items():
-        assert w4[int(i)] == v
-    assert np.all(w4[2:32] == -0.125) and np.all(w4[32:] == 0.0)
-    w6 = orc.dequant_superblock(_record(g["q6k"], 210), orc.Q6_K)
-    for i, v in g["q6k"]["expect"].items():
-        assert w6[int(i)] == v
-    assert np.all(w6[1:16] == 48.0) and np.all(w6[16:240] == 0.0)
+        assert w4[int(i)] == v, i
+    assert np.all(w4[2:32] == -0.125) and np.all(w4[64:] == 0.0)
+    assert np.all(np.delete(w4[32:64], 16) == -5.625)
+    for parity, key in ((0, "set_bytes_even"), (1, "set_bytes_odd")):
+        w6 = orc.dequant_superblock(_record(g["q6k"][key], 210), orc.Q6_K, parity)
+        for i, v in g["q6k"]["expect"].items():
+            assert w6[int(i)] == v, (parity, i)
+        assert np.all(w6[1:16] == 48.0) and np.all(w6[16:240] == 0.0)
 
 
 def test_kquant_saturation_and_zero_scale(orc):
     rec = np.zeros(144, np.uint8)
-    rec[0:2] = np.array([1.0], np.float16).view(np.uint8)       # d = 1
-    rec[4:8] = 0xFF                                             # sc_j low nibbles 15
-    rec[12:14] = 0xFF                                           # sc_j high bits 3 -> sc = 63
+    rec[0:2] = np.array([1.0], np.float16).view(np.uint8)       # d = 1, dmin = 0
+    rec[4:12] = 63                                              # sc_j = 63, mn_j low bits 0
     rec[16:144] = 0xFF                                          # q = 15 everywhere
     assert np.all(orc.dequant_superblock(rec, orc.Q4_K) == 63 * 15)
+    rec[2:4] = np.array([0.5], np.float16).view(np.uint8)       # dmin = 0.5
+    rec[4:12] = 63 | (3 << 6)                                   # mn_j low bits 3
+    rec[12:16] = 0xFF                                           # mn_j high nibbles 15 -> mn = 63
+    assert np.all(orc.dequant_superblock(rec, orc.Q4_K) == 63 * 15 - 0.5 * 63)
     rec6 = np.zeros(210, np.uint8)
     rec6[208:210] = np.array([0.0], np.float16).view(np.uint8)  # d = 0
     rec6[:192] = 0xFF
     rec6[192:208] = 127
-    assert np.all(orc.dequant_superblock(rec6, orc.Q6_K) == 0.0)
+    assert np.all(orc.dequant_superblock(rec6, orc.Q6_K, 0) == 0.0)
     rec6[208:210] = np.array([2.0], np.float16).view(np.uint8)
-    assert np.all(orc.dequant_superblock(rec6, orc.Q6_K) == 2.0 * 127 * 31)   # q = 63 saturated
+    assert np.all(orc.dequant_superblock(rec6, orc.Q6_K, 0) == 2.0 * 127 * 31)   # q = 63 saturated
+    odd = np.concatenate([rec6[208:210], rec6[:192], rec6[192:208]])
+    assert np.all(orc.dequant_superblock(odd, orc.Q6_K, 1) == 2.0 * 127 * 31)
 
 
 def test_kquant_roundtrip_against_source_weights(orc):
     w = synth.gaussian_weights(8, 2048, 7, 17)
     for t in (orc.Q4_K, orc.Q6_K):
         rec = synth.encode_kquant(w, t).reshape(-1, orc.RECORD_BYTES[t])
-        wr = np.concatenate([orc.dequant_superblock(r, t) for r in rec]).reshape(w.shape)
+        wr = np.concatenate([orc.dequant_superblock(r, t, i % 8) for i, r in enumerate(rec)]).reshape(w.shape)
         rel = np.sqrt(((wr - w) ** 2).mean() / (w ** 2).mean())
         assert rel < (0.12 if t == orc.Q4_K else 0.04)
         sub = 32 if t == orc.Q4_K else 16
@@ -382,14 +389,15 @@ def test_kquant_roundtrip_against_source_weights(orc):
 
 
 def test_kquant_gemv_is_dequant_then_matmul(orc):
-    out, inn = 96, 1024
+    out, inn = 96, 2048
     w = synth.gaussian_weights(out, inn, 7, 18)
     x = synth.bf16_normal((3, inn), 7, 19)
     xf = synth.bf16_bits_to_f32(x).astype(np.float64)
     for t in (orc.Q4_K, orc.Q6_K):
         blocks = synth.encode_kquant(w, t)
         rec = blocks.reshape(-1, orc.RECORD_BYTES[t])
-        W = np.concatenate([orc.dequant_superblock(r, t) for r in rec]).reshape(out, inn)
+        W = np.concatenate([orc.dequant_superblock(r, t, i % (inn // 256))
+                            for i, r in enumerate(rec)]).reshape(out, inn)
         y = orc.gemv_kquant(blocks, t, out, inn, x)
         assert np.allclose(y, xf @ W.T, rtol=1e-12, atol=1e-12)
     with pytest.raises(ValueError):

@@ -86,7 +86,11 @@ def _fp16(a):
 
 
 def encode_q4k(w: np.ndarray) -> np.ndarray:
-    """Encode rows of weights (in % 256 == 0) as 144-byte Q4_K records, row-major."""
+    """Encode rows of weights (in % 256 == 0) as 144-byte Q4_K records, row-major.
+
+    Layout: [0,2) d fp16, [2,4) dmin fp16, byte 4 + j = sc_j | (mn_j & 3) << 6,
+    nibble j of the word at 12 = mn_j >> 2, byte 16 + 16 j + b = q[32 j + b] | q[32 j + 16 + b] << 4.
+    """
     out, inn = w.shape
     assert inn % 256 == 0
     sb = w.reshape(-1, 8, 32).astype(np.float32)
@@ -106,25 +110,29 @@ def encode_q4k(w: np.ndarray) -> np.ndarray:
     step = (d * sc.astype(np.float32)).astype(np.float32)[:, :, None]
     off = (dm * mn.astype(np.float32)).astype(np.float32)[:, :, None]
     q = np.where(step > 0, np.rint((sb + off) / np.where(step > 0, step, 1)), 0)
-    q = np.clip(q, 0, 15).astype(np.uint8).reshape(n, 256)
+    q = np.clip(q, 0, 15).astype(np.uint8)                       # [n, 8, 32]
     rec = np.zeros((n, 144), np.uint8)
     rec[:, 0:2] = d16.view(np.uint8).reshape(n, 2)
     rec[:, 2:4] = m16.view(np.uint8).reshape(n, 2)
-    j = np.arange(8)
-    lo_sc = ((sc & 15) << (4 * j)).sum(axis=1).astype(np.uint32)
-    lo_mn = ((mn & 15) << (4 * j)).sum(axis=1).astype(np.uint32)
-    hib = (((sc >> 4) & 3) << (2 * j)).sum(axis=1) + (((mn >> 4) & 3) << (16 + 2 * j)).sum(axis=1)
-    rec[:, 4:8] = lo_sc.astype("<u4").view(np.uint8).reshape(n, 4)
-    rec[:, 8:12] = lo_mn.astype("<u4").view(np.uint8).reshape(n, 4)
-    rec[:, 12:16] = hib.astype("<u4").view(np.uint8).reshape(n, 4)
-    rec[:, 16:144] = q[:, 0::2] | (q[:, 1::2] << 4)
+    rec[:, 4:12] = (sc | ((mn & 3) << 6)).astype(np.uint8)
+    nib = (mn >> 2).astype(np.uint8)
+    rec[:, 12:16] = nib[:, 0::2] | (nib[:, 1::2] << 4)
+    rec[:, 16:144] = (q[:, :, :16] | (q[:, :, 16:] << 4)).reshape(n, 128)
     return rec.reshape(-1)
 
 
 def encode_q6k(w: np.ndarray) -> np.ndarray:
-    """Encode rows of weights (in % 256 == 0) as 210-byte Q6_K records, row-major."""
+    """Encode rows of weights (in % 2048 == 0) as 210-byte Q6_K records, row-major.
+
+    A record's layout depends on its index n in its row: n even -> [0,192) q, [192,208)
+    int8 scales, [208,210) d; n odd -> [0,2) d, [2,194) q, [194,210) scales. The q area
+    holds, for chunk t (48 bytes) and group m (12 bytes: words A, B, C), with
+    W(j, L) = 16 j + 4 t + L: A byte L = lo4 q[W(4m,L)] | lo4 q[W(4m+1,L)] << 4,
+    B byte L = lo4 q[W(4m+2,L)] | lo4 q[W(4m+3,L)] << 4, C byte L = hi2 q[W(4m+2,L)]
+    | hi2 q[W(4m+3,L)] << 2 | hi2 q[W(4m,L)] << 4 | hi2 q[W(4m+1,L)] << 6.
+    """
     out, inn = w.shape
-    assert inn % 256 == 0
+    assert inn % 2048 == 0, "Q6_K rows must hold a multiple of 8 records"
     sb = w.reshape(-1, 16, 16).astype(np.float32)
     n = sb.shape[0]
     a = (np.abs(sb).max(axis=2) / np.float32(31.0)).astype(np.float32)
@@ -134,14 +142,26 @@ def encode_q6k(w: np.ndarray) -> np.ndarray:
     sc = np.clip(sc, -128, 127).astype(np.int64)
     step = (d * sc.astype(np.float32)).astype(np.float32)[:, :, None]
     q = np.where(step > 0, np.rint(sb / np.where(step > 0, step, 1)), 0)
-    q = (np.clip(q, -32, 31) + 32).astype(np.uint8).reshape(n, 256)
+    q = (np.clip(q, -32, 31) + 32).astype(np.uint8)               # [n, 16 j, 16 = 4 t + L]
+    qj = q.reshape(n, 4, 4, 4, 4)                                  # [n, m, s, t, L], j = 4 m + s
+    lo4 = qj & 15
+    hi2 = qj >> 4
+    A = lo4[:, :, 0] | (lo4[:, :, 1] << 4)                         # [n, m, t, L]
+    B = lo4[:, :, 2] | (lo4[:, :, 3] << 4)
+    Cw = hi2[:, :, 2] | (hi2[:, :, 3] << 2) | (hi2[:, :, 0] << 4) | (hi2[:, :, 1] << 6)
+    area = np.stack([A, B, Cw], axis=3)                           # [n, m, t, word, L]
+    area = area.transpose(0, 2, 1, 3, 4).reshape(n, 192)          # chunk t, group m, word, lane
     rec = np.zeros((n, 210), np.uint8)
-    lo = q & 15
-    hi2 = q >> 4
-    rec[:, 0:128] = lo[:, 0::2] | (lo[:, 1::2] << 4)
-    rec[:, 128:192] = hi2[:, 0::4] | (hi2[:, 1::4] << 2) | (hi2[:, 2::4] << 4) | (hi2[:, 3::4] << 6)
-    rec[:, 192:208] = sc.astype(np.int8).view(np.uint8)
-    rec[:, 208:210] = d16.view(np.uint8).reshape(n, 2)
+    scb = sc.astype(np.int8).view(np.uint8)
+    db = d16.view(np.uint8).reshape(n, 2)
+    even = (np.arange(n) % 2) == 0                                 # rows hold an even count of records
+    rec[even, 0:192] = area[even]
+    rec[even, 192:208] = scb[even]
+    rec[even, 208:210] = db[even]
+    odd = ~even
+    rec[odd, 0:2] = db[odd]
+    rec[odd, 2:194] = area[odd]
+    rec[odd, 194:210] = scb[odd]
     return rec.reshape(-1)
 
 

@@ -43,6 +43,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define FL_API __attribute__((visibility("default")))
+#else
+#define FL_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -66,9 +72,9 @@ typedef enum {
 #define FL_GGML_Q4_K 12
 #define FL_GGML_Q6_K 14
 
-const char* fl_status_string(int status);
-const char* fl_last_error(void);
-int fl_version(void);
+FL_API const char* fl_status_string(int status);
+FL_API const char* fl_last_error(void);
+FL_API int fl_version(void);
 
 /* ========================================================================= */
 /* Plane store ([FoQLens] progress table, "a format of our own": one stored   */
@@ -89,7 +95,7 @@ int fl_version(void);
 
 /* Bytes of the plane store of an out x in layer (out % 64 == 0, in % 128 == 0);
  * 0 for an invalid shape. */
-size_t fl_plane_store_bytes(int out, int in);
+FL_API size_t fl_plane_store_bytes(int out, int in);
 
 /* Pack int8 codes and their scales into the plane store.
  *   codes  device, int8 [out][in] row-major, values in [-128, 127]
@@ -98,7 +104,7 @@ size_t fl_plane_store_bytes(int out, int in);
  *   store  device, fl_plane_store_bytes(out, in) bytes, 16-byte aligned;
  *          fully overwritten.
  * out % 64 == 0 and in % 128 == 0, else FL_ERR_SHAPE. Bit-exact. */
-fl_status fl_pack_planes(const int8_t* codes, const float* scales, int out, int in, uint8_t* store, void* stream);
+FL_API fl_status fl_pack_planes(const int8_t* codes, const float* scales, int out, int in, uint8_t* store, void* stream);
 
 /* A packed layer: device pointer to its plane store and its shape. */
 typedef struct {
@@ -135,7 +141,7 @@ typedef struct {
  * counts  device, uint32 [m + 1] or NULL: per-level block counts are ADDED
  *         to it (the caller zeroes it first).
  * nblocks >= 0, 0 <= nlenses <= 64. */
-fl_status fl_level_map(const float* xy, int nblocks, const float* centers, const float* radii, int nlenses,
+FL_API fl_status fl_level_map(const float* xy, int nblocks, const float* centers, const float* radii, int nlenses,
                        const fl_lens_params* params, uint8_t* levels, uint32_t* counts, void* stream);
 
 /* ========================================================================= */
@@ -159,9 +165,9 @@ fl_status fl_level_map(const float* xy, int nblocks, const float* centers, const
 /*          leaves it zero-filled again. Calls that share a workspace must   */
 /*          not overlap on the GPU. May be NULL when the size is 0.          */
 /* ========================================================================= */
-size_t fl_gemv_workspace_bytes(int out, int in, int batch);
+FL_API size_t fl_gemv_workspace_bytes(int out, int in, int batch);
 
-fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, const uint16_t* x, int batch, float* y,
+FL_API fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, const uint16_t* x, int batch, float* y,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* Escalation residual ([PoD]: redo a step at 8 bits, written as an addition
@@ -170,7 +176,7 @@ fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, const u
  * a/2 .. b/2 - 1. The levels live on the device, so the host cannot check
  * them: a block whose to-level is not above its from-level adds nothing.
  * Same arguments as fl_gemv_depth. */
-fl_status fl_gemv_residual(const fl_plane_weight* w, const uint8_t* from_levels, const uint8_t* to_levels,
+FL_API fl_status fl_gemv_residual(const fl_plane_weight* w, const uint8_t* from_levels, const uint8_t* to_levels,
                            const uint16_t* x, int batch, float* y, void* workspace, size_t workspace_bytes,
                            void* stream);
 
@@ -187,7 +193,7 @@ typedef struct {
   float* y;
 } fl_gemv_problem;
 
-fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream);
+FL_API fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream);
 
 /* ========================================================================= */
 /* Uncertainty gate ([PoD]: redo at 8 bits when the low-precision output     */
@@ -201,7 +207,7 @@ fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int
 /* 4 <= vocab <= 2^24; outputs device: entropy, margin fp32 [batch], top2 int32   */
 /* [batch][2], escalate uint8 [batch]. fp32 arithmetic.                      */
 /* ========================================================================= */
-fl_status fl_logit_gate(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,
+FL_API fl_status fl_logit_gate(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,
                         float* margin, int32_t* top2, uint8_t* escalate, void* stream);
 
 /* ========================================================================= */
@@ -228,10 +234,10 @@ fl_status fl_logit_gate(const float* logits, int vocab, int batch, float tau_h, 
 /* ggml_type other than FL_GGML_Q4_K / FL_GGML_Q6_K -> FL_ERR_UNSUPPORTED.    */
 /* Same x / y / workspace rules as fl_gemv_depth.                            */
 /* ========================================================================= */
-size_t fl_kquant_bytes(int ggml_type, int out, int in);
-size_t fl_kquant_workspace_bytes(int ggml_type, int out, int in, int batch);
+FL_API size_t fl_kquant_bytes(int ggml_type, int out, int in);
+FL_API size_t fl_kquant_workspace_bytes(int ggml_type, int out, int in, int batch);
 
-fl_status fl_gemv_kquant(const void* blocks, int ggml_type, int out, int in, const uint16_t* x, int batch, float* y,
+FL_API fl_status fl_gemv_kquant(const void* blocks, int ggml_type, int out, int in, const uint16_t* x, int batch, float* y,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 typedef struct {
@@ -244,7 +250,7 @@ typedef struct {
 } fl_kquant_problem;
 
 /* Several K-quant tensors in one launch (a decode step); no workspace. */
-fl_status fl_gemv_kquant_batched(const fl_kquant_problem* problems, int n, int batch, void* stream);
+FL_API fl_status fl_gemv_kquant_batched(const fl_kquant_problem* problems, int n, int batch, void* stream);
 
 #ifdef __cplusplus
 }

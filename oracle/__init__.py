@@ -50,8 +50,8 @@ def _load():
                 "orc_max_threads": (i, []),
                 "orc_quantize_int8": (None, [P, i, i, P, P]),
                 "orc_dequant_depth": (d, [C.c_int8, f, i]),
-                "orc_gemv_depth": (None, [P, P, i, i, P, P, i, P, i]),
-                "orc_gemv_residual": (None, [P, P, i, i, P, P, P, i, P, i]),
+                "orc_gemv_depth": (None, [P, P, i, i, P, P, i, P, P, i]),
+                "orc_gemv_residual": (None, [P, P, i, i, P, P, P, i, P, P, i]),
                 "orc_store_bytes": (C.c_size_t, [i, i]),
                 "orc_pack_planes": (None, [P, P, i, i, P]),
                 "orc_unpack_planes": (None, [P, i, i, P, P]),
@@ -61,7 +61,7 @@ def _load():
                 "orc_logit_gate": (None, [P, i, i, d, d, P, P, P, P]),
                 "orc_dequant_q4k": (None, [P, P]),
                 "orc_dequant_q6k": (None, [P, i, P]),
-                "orc_gemv_kquant": (i, [P, i, i, i, P, i, P, i]),
+                "orc_gemv_kquant": (i, [P, i, i, i, P, i, P, P, i]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -99,7 +99,8 @@ def dequant_depth(q: int, s: float, depth: int) -> float:
     return float(_load().orc_dequant_depth(int(q), float(s), int(depth)))
 
 
-def gemv_depth(q, s, levels, x_bf16, nthreads: int = 0) -> np.ndarray:
+def gemv_depth(q, s, levels, x_bf16, nthreads: int = 0, with_mass: bool = False):
+    """y [batch, out] in float64; with_mass also returns sum_c |w_d| |x| per output."""
     q = np.ascontiguousarray(q, np.int8)
     s = np.ascontiguousarray(s, np.float32)
     levels = np.ascontiguousarray(levels, np.uint8)
@@ -107,11 +108,13 @@ def gemv_depth(q, s, levels, x_bf16, nthreads: int = 0) -> np.ndarray:
     out, inn = q.shape
     batch = x.shape[0]
     y = np.empty((batch, out), np.float64)
-    _load().orc_gemv_depth(_p(q), _p(s), out, inn, _p(levels), _p(x), batch, _p(y), nthreads)
-    return y
+    m = np.empty((batch, out), np.float64) if with_mass else None
+    _load().orc_gemv_depth(_p(q), _p(s), out, inn, _p(levels), _p(x), batch, _p(y), _p(m) if with_mass else None,
+                           nthreads)
+    return (y, m) if with_mass else y
 
 
-def gemv_residual(q, s, from_levels, to_levels, x_bf16, nthreads: int = 0) -> np.ndarray:
+def gemv_residual(q, s, from_levels, to_levels, x_bf16, nthreads: int = 0, with_mass: bool = False):
     q = np.ascontiguousarray(q, np.int8)
     s = np.ascontiguousarray(s, np.float32)
     a = np.ascontiguousarray(from_levels, np.uint8)
@@ -120,8 +123,10 @@ def gemv_residual(q, s, from_levels, to_levels, x_bf16, nthreads: int = 0) -> np
     out, inn = q.shape
     batch = x.shape[0]
     y = np.empty((batch, out), np.float64)
-    _load().orc_gemv_residual(_p(q), _p(s), out, inn, _p(a), _p(b), _p(x), batch, _p(y), nthreads)
-    return y
+    m = np.empty((batch, out), np.float64) if with_mass else None
+    _load().orc_gemv_residual(_p(q), _p(s), out, inn, _p(a), _p(b), _p(x), batch, _p(y),
+                              _p(m) if with_mass else None, nthreads)
+    return (y, m) if with_mass else y
 
 
 def store_bytes(out: int, inn: int) -> int:
@@ -200,13 +205,15 @@ def dequant_superblock(rec: np.ndarray, ggml_type: int, index_in_row: int = 0) -
     return w
 
 
-def gemv_kquant(blocks, ggml_type: int, out: int, inn: int, x_bf16, nthreads: int = 0) -> np.ndarray:
+def gemv_kquant(blocks, ggml_type: int, out: int, inn: int, x_bf16, nthreads: int = 0, with_mass: bool = False):
     blocks = np.ascontiguousarray(blocks, np.uint8)
     x = _bf16_bits(x_bf16)
     batch = x.shape[0]
     assert batch <= 16
     y = np.empty((batch, out), np.float64)
-    rc = _load().orc_gemv_kquant(_p(blocks), int(ggml_type), out, inn, _p(x), batch, _p(y), nthreads)
+    m = np.empty((batch, out), np.float64) if with_mass else None
+    rc = _load().orc_gemv_kquant(_p(blocks), int(ggml_type), out, inn, _p(x), batch, _p(y),
+                                 _p(m) if with_mass else None, nthreads)
     if rc != 0:
         raise ValueError("unsupported K-quant type")
-    return y
+    return (y, m) if with_mass else y

@@ -146,22 +146,27 @@ ORC_API double orc_dequant_depth(int8_t q, float s, int depth) {
 static int level_bits(uint8_t level) { return 2 * (level > 4 ? 4 : (int)level); }
 
 /* y[t][r] = sum_c w_d(b(r))[r][c] * x[t][c], d = bits of levels[r / 64].    */
+/* mass (optional) receives sum_c |w_d[r][c]| |x[t][c]|, the scale of the    */
+/* tolerance the GPU result is held to.                                      */
 ORC_API void orc_gemv_depth(const int8_t* q, const float* s, int out, int in, const uint8_t* levels,
-                            const uint16_t* x, int batch, double* y, int nthreads) {
+                            const uint16_t* x, int batch, double* y, double* mass, int nthreads) {
   const int G = in / 128;
   set_threads(nthreads);
 #pragma omp parallel for schedule(static)
   for (int r = 0; r < out; ++r) {
     int d = level_bits(levels[r / 64]);
     for (int t = 0; t < batch; ++t) {
-      double acc = 0.0;
+      double acc = 0.0, am = 0.0;
       if (d > 0) {
         for (int c = 0; c < in; ++c) {
           double w = (double)s[(size_t)r * G + c / 128] * recon_code(q[(size_t)r * in + c], d);
-          acc += w * bf16_to_double(x[(size_t)t * in + c]);
+          double xv = bf16_to_double(x[(size_t)t * in + c]);
+          acc += w * xv;
+          am += fabs(w) * fabs(xv);
         }
       }
       y[(size_t)t * out + r] = acc;
+      if (mass) mass[(size_t)t * out + r] = am;
     }
   }
 }
@@ -171,7 +176,7 @@ ORC_API void orc_gemv_depth(const int8_t* q, const float* s, int out, int in, co
 /* ([Precision on Demand]: the redo at 8 bits written as an addition to the  */
 /* low pass.) Escalation only raises depth: a block with b <= a adds 0.      */
 ORC_API void orc_gemv_residual(const int8_t* q, const float* s, int out, int in, const uint8_t* from_levels,
-                               const uint8_t* to_levels, const uint16_t* x, int batch, double* dy,
+                               const uint8_t* to_levels, const uint16_t* x, int batch, double* dy, double* mass,
                                int nthreads) {
   const int G = in / 128;
   set_threads(nthreads);
@@ -180,14 +185,17 @@ ORC_API void orc_gemv_residual(const int8_t* q, const float* s, int out, int in,
     int a = level_bits(from_levels[r / 64]);
     int b = level_bits(to_levels[r / 64]);
     for (int t = 0; t < batch; ++t) {
-      double acc = 0.0;
+      double acc = 0.0, am = 0.0;
       for (int c = 0; c < in && b > a; ++c) {
         int8_t qq = q[(size_t)r * in + c];
         double sc = (double)s[(size_t)r * G + c / 128];
         double dw = sc * recon_code(qq, b) - sc * recon_code(qq, a);
-        acc += dw * bf16_to_double(x[(size_t)t * in + c]);
+        double xv = bf16_to_double(x[(size_t)t * in + c]);
+        acc += dw * xv;
+        am += fabs(dw) * fabs(xv);
       }
       dy[(size_t)t * out + r] = acc;
+      if (mass) mass[(size_t)t * out + r] = am;
     }
   }
 }
@@ -436,7 +444,7 @@ ORC_API void orc_dequant_q6k(const uint8_t* blk, int odd, double* w) {
 
 /* y[t][r] = sum_c w[r][c] x[t][c], each super-block dequantized then dotted.*/
 ORC_API int orc_gemv_kquant(const uint8_t* blocks, int type, int out, int in, const uint16_t* x, int batch,
-                            double* y, int nthreads) {
+                            double* y, double* mass, int nthreads) {
   int rec;
   if (type == ORC_Q4_K)
     rec = 144;
@@ -449,8 +457,8 @@ ORC_API int orc_gemv_kquant(const uint8_t* blocks, int type, int out, int in, co
 #pragma omp parallel for schedule(static)
   for (int r = 0; r < out; ++r) {
     double w[256];
-    double acc[16];
-    for (int t = 0; t < batch; ++t) acc[t] = 0.0;
+    double acc[16], am[16];
+    for (int t = 0; t < batch; ++t) acc[t] = am[t] = 0.0;
     for (int sb = 0; sb < nsb; ++sb) {
       const uint8_t* blk = blocks + ((size_t)r * nsb + sb) * rec;
       if (type == ORC_Q4_K)
@@ -458,9 +466,16 @@ ORC_API int orc_gemv_kquant(const uint8_t* blocks, int type, int out, int in, co
       else
         orc_dequant_q6k(blk, sb & 1, w);
       for (int t = 0; t < batch; ++t)
-        for (int i = 0; i < 256; ++i) acc[t] += w[i] * bf16_to_double(x[(size_t)t * in + 256 * sb + i]);
+        for (int i = 0; i < 256; ++i) {
+          double xv = bf16_to_double(x[(size_t)t * in + 256 * sb + i]);
+          acc[t] += w[i] * xv;
+          am[t] += fabs(w[i]) * fabs(xv);
+        }
     }
-    for (int t = 0; t < batch; ++t) y[(size_t)t * out + r] = acc[t];
+    for (int t = 0; t < batch; ++t) {
+      y[(size_t)t * out + r] = acc[t];
+      if (mass) mass[(size_t)t * out + r] = am[t];
+    }
   }
   return 0;
 }

@@ -1,0 +1,374 @@
+"""CUDA path vs the CPU oracle, element by element, through the C-ABI.
+
+Bars: bit-exact for the plane store, level maps, top-2 indices and gate
+decisions (outside a band where fp32 rounding could flip them); for
+outputs |y_gpu - y_ref| <= 2e-3 * sum_c |w||x| + 1e-5 (fp32 accumulation).
+"""
+import numpy as np
+import pytest
+
+from variable_precision_weight_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2e-3, 1e-5
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from variable_precision_weight_b200 import build
+    build.build()
+    from variable_precision_weight_b200 import fl
+    return torch, fl
+
+
+def dev(torch, a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def check_close(y_gpu, y_ref, mass, what=""):
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bound = REL * mass + ABS
+    bad = err > bound
+    assert not bad.any(), f"{what}: {bad.sum()} outputs outside tolerance, worst ratio {(err / bound).max():.3g}"
+    return float((err / bound).max())
+
+
+def pack_gpu(torch, fl, q, s):
+    out, inn = q.shape
+    store = torch.empty(fl.fl_plane_store_bytes(out, inn), dtype=torch.uint8, device="cuda")
+    fl.fl_pack_planes(dev(torch, q), dev(torch, s), out, inn, store)
+    return store
+
+
+def gemv_gpu(torch, fl, store, out, inn, levels, x, mode=0, to_levels=None, y0=None):
+    batch = x.shape[0]
+    y = torch.zeros((batch, out), dtype=torch.float32, device="cuda") if y0 is None else dev(torch, y0.astype(np.float32))
+    wsb = fl.fl_gemv_workspace_bytes(out, inn, batch)
+    ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    w = fl.plane_weight(store, out, inn)
+    if mode == 0:
+        fl.fl_gemv_depth(w, dev(torch, levels), dev(torch, x), batch, y, ws, wsb)
+    else:
+        fl.fl_gemv_residual(w, dev(torch, levels), dev(torch, to_levels), dev(torch, x), batch, y, ws, wsb)
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), ws
+
+
+# ----------------------------------------------------------------------------- plane store
+
+@pytest.mark.parametrize("out,inn", [(64, 128), (192, 1664), (1024, 1024), (128, 14336)])
+def test_pack_bit_exact(env, orc, out, inn):
+    torch, fl = env
+    rng = synth.rng(11, out, inn)
+    q = rng.integers(-128, 128, size=(out, inn)).astype(np.int8)
+    s = rng.random((out, inn // 128), dtype=np.float32)
+    st = pack_gpu(torch, fl, q, s).cpu().numpy()
+    assert np.array_equal(st, orc.pack_planes(q, s))
+
+
+def test_pack_all_codes(env, orc):
+    torch, fl = env
+    q = (np.arange(64 * 256) % 256 - 128).astype(np.int8).reshape(64, 256)
+    s = np.linspace(0, 1, 128, dtype=np.float32).reshape(64, 2)
+    assert np.array_equal(pack_gpu(torch, fl, q, s).cpu().numpy(), orc.pack_planes(q, s))
+
+
+# ----------------------------------------------------------------------------- depth GEMV
+
+CASES = [
+    # out, in, batch, level spec
+    (1024, 1024, 1, "uniform"),       # config-0 shape, seeded mixed depths
+    (448, 1664, 1, "uniform"),        # 13 groups: ragged tiles at every depth
+    (448, 1664, 3, "uniform"),
+    (448, 1664, 4, "uniform"),
+    (448, 1664, 5, "uniform"),        # second N-tile
+    (320, 2048, 8, "uniform"),
+    (320, 2048, 16, "uniform"),
+    (256, 14336, 1, "uniform"),       # few blocks, wide rows: column slices + tickets
+    (256, 14336, 16, "uniform"),
+    (2048, 1024, 1, "d4"),
+    (640, 3072, 2, "zero_heavy"),
+]
+
+
+def levels_for(spec, nblocks, key):
+    if spec == "uniform":
+        return synth.seeded_levels(nblocks, *key)
+    if spec == "d4":
+        return np.full(nblocks, 2, np.uint8)
+    lv = synth.seeded_levels(nblocks, *key)
+    lv[::2] = 0
+    return lv
+
+
+@pytest.mark.parametrize("out,inn,batch,spec", CASES)
+def test_gemv_depth_vs_oracle(env, orc, out, inn, batch, spec):
+    torch, fl = env
+    q, s = synth.int8_layer(out, inn, 21, out, inn)
+    lv = levels_for(spec, out // 64, (22, out, inn))
+    x = synth.bf16_normal((batch, inn), 23, out, inn, batch)
+    store = pack_gpu(torch, fl, q, s)
+    y, ws = gemv_gpu(torch, fl, store, out, inn, lv, x)
+    yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+    check_close(y, yref, mass, f"depth {out}x{inn} b{batch}")
+    zero_rows = np.repeat(lv == 0, 64)
+    assert np.all(y[:, zero_rows] == 0.0)
+
+
+def test_gemv_workspace_left_zero(env, orc):
+    torch, fl = env
+    out, inn, batch = 256, 14336, 4
+    q, s = synth.int8_layer(out, inn, 24)
+    lv = synth.seeded_levels(out // 64, 25)
+    x = synth.bf16_normal((batch, inn), 26)
+    store = pack_gpu(torch, fl, q, s)
+    wsb = fl.fl_gemv_workspace_bytes(out, inn, batch)
+    assert wsb > 0
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    y = torch.empty((batch, out), dtype=torch.float32, device="cuda")
+    w = fl.plane_weight(store, out, inn)
+    yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+    for _ in range(3):  # tickets return to zero, so repeated calls stay correct
+        fl.fl_gemv_depth(w, dev(torch, lv), dev(torch, x), batch, y, ws, wsb)
+        torch.cuda.synchronize()
+        check_close(y.cpu().numpy(), yref, mass, "repeat")
+    nt = (out // 64) * 4
+    assert int(ws[:nt].count_nonzero().item()) == 0
+    with pytest.raises(fl.FlError) as e:
+        fl.fl_gemv_depth(w, dev(torch, lv), dev(torch, x), batch, y, ws, wsb - 16)
+    assert e.value.status == -6
+
+
+def test_gemv_high_dynamic_range_x(env, orc):
+    """One large element per 128-column group: x enters as a 15-bit fixed point per group,
+    so the error stays within sum_g 2^-14 max_g|x| sum_{c in g} |w| (|w| <= 128 s)."""
+    torch, fl = env
+    out, inn = 128, 1024
+    q, s = synth.int8_layer(out, inn, 27)
+    lv = np.array([4, 2], np.uint8)
+    xf = synth.rng(28).standard_normal((1, inn), dtype=np.float32)
+    xf[0, ::128] = 300.0
+    x = synth.f32_to_bf16_bits(xf)
+    store = pack_gpu(torch, fl, q, s)
+    y, _ = gemv_gpu(torch, fl, store, out, inn, lv, x)
+    yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+    gmax = np.abs(synth.bf16_bits_to_f32(x).reshape(-1, 128)).max(axis=1)          # [G]
+    fixed = (2.0 ** -14) * 128 * 128 * (s.astype(np.float64) * gmax[None, :]).sum(1)  # [out]
+    assert np.all(np.abs(y[0] - yref[0]) <= fixed + REL * mass[0] + ABS)
+
+
+def test_residual_vs_oracle_and_identity(env, orc):
+    torch, fl = env
+    out, inn, batch = 512, 2048, 2
+    q, s = synth.int8_layer(out, inn, 31)
+    a = synth.seeded_levels(out // 64, 32)
+    b = np.maximum(a, synth.seeded_levels(out // 64, 33))
+    b[0], a[0] = 2, 3                                  # a non-raising block adds nothing
+    x = synth.bf16_normal((batch, inn), 34)
+    store = pack_gpu(torch, fl, q, s)
+    y0 = synth.rng(35).standard_normal((batch, out)).astype(np.float32)
+    y, _ = gemv_gpu(torch, fl, store, out, inn, a, x, mode=1, to_levels=b, y0=y0)
+    dref, mass = orc.gemv_residual(q, s, a, b, x, with_mass=True)
+    check_close(y, y0.astype(np.float64) + dref, mass, "residual")
+    assert np.array_equal(y[:, :64], y0[:, :64])
+    # D4 pass + residual(D4 -> D8) == D8 pass
+    d4 = np.full(out // 64, 2, np.uint8)
+    d8 = np.full(out // 64, 4, np.uint8)
+    y4, _ = gemv_gpu(torch, fl, store, out, inn, d4, x)
+    y48, _ = gemv_gpu(torch, fl, store, out, inn, d4, x, mode=1, to_levels=d8, y0=y4)
+    y8ref, mass8 = orc.gemv_depth(q, s, d8, x, with_mass=True)
+    check_close(y48, y8ref, mass8, "D4+res")
+
+
+def test_residual_split_columns(env, orc):
+    torch, fl = env
+    out, inn, batch = 128, 8192, 4
+    q, s = synth.int8_layer(out, inn, 36)
+    a = np.array([1, 2], np.uint8)
+    b = np.array([4, 3], np.uint8)
+    x = synth.bf16_normal((batch, inn), 37)
+    store = pack_gpu(torch, fl, q, s)
+    assert fl.fl_gemv_workspace_bytes(out, inn, batch) > 0
+    y, _ = gemv_gpu(torch, fl, store, out, inn, a, x, mode=1, to_levels=b)
+    dref, mass = orc.gemv_residual(q, s, a, b, x, with_mass=True)
+    check_close(y, dref, mass, "residual split")
+
+
+def test_batched_problems(env, orc):
+    torch, fl = env
+    shapes = [(2048, 1024), (1024, 1024), (1024, 2048), (3072, 1024), (1024, 3072), (640, 128)]
+    batch = 2
+    items, refs, keep = [], [], []
+    for i, (o, n) in enumerate(shapes):
+        q, s = synth.int8_layer(o, n, 41, i)
+        lv = synth.seeded_levels(o // 64, 42, i)
+        x = synth.bf16_normal((batch, n), 43, i)
+        st = pack_gpu(torch, fl, q, s)
+        y = torch.zeros((batch, o), dtype=torch.float32, device="cuda")
+        lvd, xd = dev(torch, lv), dev(torch, x)
+        keep += [st, lvd, xd, y]
+        items.append((st, o, n, lvd, None, xd, y))
+        refs.append(orc.gemv_depth(q, s, lv, x, with_mass=True))
+    arr = fl.gemv_problems(items)
+    fl.fl_gemv_batched(arr, len(items), batch, 0)
+    torch.cuda.synchronize()
+    for (st, o, n, lvd, _, xd, y), (yref, mass) in zip(items, refs):
+        check_close(y.cpu().numpy(), yref, mass, f"batched {o}x{n}")
+
+
+# ----------------------------------------------------------------------------- level map
+
+def test_level_map_bit_exact(env, orc, golden):
+    torch, fl = env
+    nb = 14708
+    xy, cxy, r = synth.lens_inputs(nb, 8, 51)
+    for (f, g, gamma, combine) in ((0.3, 0.75, 1, 0), (0.3, 0.75, 1, 1), (0.5, 1.0, 0, 0), (0.3, 0.75, 3, 0),
+                                   (0.3, 1.0, 3, 0), (0.9, 0.5, 2, 1), (0.0, 0.75, 1, 0)):
+        kappa = orc.lens_kappa(g, gamma, 4)
+        stops = synth.even_stops(kappa, gamma)
+        ref = orc.level_map(xy, cxy, r * (4 if f < 0.5 else 1), f, g, gamma, 4, stops, combine)
+        lev = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        cnt = torch.zeros(5, dtype=torch.int32, device="cuda")
+        p = fl.lens_params(f, g, gamma, 4, stops, combine)
+        fl.fl_level_map(dev(torch, xy), nb, dev(torch, cxy), dev(torch, r * (4 if f < 0.5 else 1)), 8, p, lev, cnt)
+        torch.cuda.synchronize()
+        got = lev.cpu().numpy()
+        assert np.array_equal(got, ref), (f, g, gamma, combine, (got != ref).sum())
+        assert np.array_equal(cnt.cpu().numpy(), np.bincount(ref, minlength=5))
+    gd = golden("lens_hand_maps.json")
+    P = gd["params"]
+    one = gd["single_lens"]
+    blocks = np.array(one["blocks"], np.float32)
+    lev = torch.empty(len(blocks), dtype=torch.uint8, device="cuda")
+    p = fl.lens_params(P["f"], P["g"], P["gamma"], P["m"], P["stops"], 0)
+    fl.fl_level_map(dev(torch, blocks), len(blocks), dev(torch, np.array([one["center"]], np.float32)),
+                    dev(torch, np.array([one["r"]], np.float32)), 1, p, lev, None)
+    torch.cuda.synchronize()
+    assert lev.cpu().numpy().tolist() == one["levels_sum"]
+
+
+# ----------------------------------------------------------------------------- gate
+
+@pytest.mark.parametrize("vocab,batch", [(151936, 1), (151936, 3), (128256, 16), (1000, 2), (4, 1)])
+def test_logit_gate_vs_oracle(env, orc, vocab, batch):
+    torch, fl = env
+    z = synth.rng(61, vocab, batch).standard_normal((batch, vocab), dtype=np.float32) * np.float32(0.7)
+    if batch > 1:
+        z[1, 17] = 9.0
+        z[1, 5000 % vocab] = 9.0       # a tie for the top
+    H, M, top2, _ = orc.logit_gate(z, 0.0, 0.0)
+    tau_h, tau_m = float(np.median(H)), float(np.median(M))
+    _, _, _, esc_ref = orc.logit_gate(z, tau_h, tau_m)
+    zd = dev(torch, z)
+    e = torch.empty(batch, dtype=torch.float32, device="cuda")
+    m = torch.empty(batch, dtype=torch.float32, device="cuda")
+    t2 = torch.empty((batch, 2), dtype=torch.int32, device="cuda")
+    es = torch.empty(batch, dtype=torch.uint8, device="cuda")
+    fl.fl_logit_gate(zd, vocab, batch, tau_h, tau_m, e, m, t2, es)
+    torch.cuda.synchronize()
+    e, m, t2, es = e.cpu().numpy(), m.cpu().numpy(), t2.cpu().numpy(), es.cpu().numpy()
+    assert np.array_equal(t2, top2)
+    assert np.allclose(e, H, rtol=1e-5, atol=1e-6)
+    assert np.allclose(m, M, rtol=1e-5, atol=1e-7)
+    band = (np.abs(H - tau_h) <= 1e-4 * abs(tau_h) + 1e-6) | (np.abs(M - tau_m) <= 1e-6)
+    assert np.array_equal(es[~band], esc_ref[~band])
+    assert np.array_equal(es, ((e > np.float32(tau_h)) | (m < np.float32(tau_m))).astype(np.uint8))
+
+
+def test_logit_gate_closed_forms(env):
+    torch, fl = env
+    V = 151936
+    z = np.full((2, V), 0.5, np.float32)
+    z[1, 1234] = 300.0
+    e = torch.empty(2, dtype=torch.float32, device="cuda")
+    m = torch.empty(2, dtype=torch.float32, device="cuda")
+    t2 = torch.empty((2, 2), dtype=torch.int32, device="cuda")
+    es = torch.empty(2, dtype=torch.uint8, device="cuda")
+    fl.fl_logit_gate(dev(torch, z), V, 2, 5.0, 0.5, e, m, t2, es)
+    torch.cuda.synchronize()
+    e, m, t2, es = e.cpu().numpy(), m.cpu().numpy(), t2.cpu().numpy(), es.cpu().numpy()
+    assert abs(e[0] - np.log(V)) <= 1e-5 * np.log(V) and m[0] == 0.0 and t2[0].tolist() == [0, 1] and es[0] == 1
+    assert e[1] < 1e-6 and m[1] == 1.0 and t2[1].tolist() == [1234, 0] and es[1] == 0
+
+
+# ----------------------------------------------------------------------------- K-quant
+
+@pytest.mark.parametrize("ggml_type,out,inn,batch", [
+    (12, 512, 2048, 1), (12, 192, 8192, 3), (12, 64, 256, 1), (12, 128, 1280, 5), (12, 256, 2048, 16),
+    (14, 512, 2048, 1), (14, 192, 8192, 4), (14, 128, 4096, 8), (14, 64, 2048, 16),
+])
+def test_kquant_vs_oracle(env, orc, ggml_type, out, inn, batch):
+    torch, fl = env
+    w = synth.gaussian_weights(out, inn, 71, ggml_type, out, inn)
+    blocks = synth.encode_kquant(w, ggml_type)
+    x = synth.bf16_normal((batch, inn), 72, out, inn, batch)
+    y = torch.zeros((batch, out), dtype=torch.float32, device="cuda")
+    wsb = fl.fl_kquant_workspace_bytes(ggml_type, out, inn, batch)
+    ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+    fl.fl_gemv_kquant(dev(torch, blocks), ggml_type, out, inn, dev(torch, x), batch, y, ws, wsb)
+    torch.cuda.synchronize()
+    yref, mass = orc.gemv_kquant(blocks, ggml_type, out, inn, x, with_mass=True)
+    check_close(y.cpu().numpy(), yref, mass, f"kquant {ggml_type} {out}x{inn} b{batch}")
+
+
+def test_kquant_negative_and_saturated_scales(env, orc):
+    """Q6_K int8 scales of both signs (and -128), Q4_K scales/mins at 0 and 63."""
+    torch, fl = env
+    out, inn = 128, 4096
+    w = synth.gaussian_weights(out, inn, 75)
+    b6 = synth.encode_kquant(w, fl.FL_GGML_Q6_K).reshape(-1, 210).copy()
+    rng = synth.rng(76)
+    for i in range(b6.shape[0]):
+        base = 192 if i % 2 == 0 else 194
+        sc = b6[i, base:base + 16].view(np.int8)
+        sc[:] = rng.integers(-128, 128, 16).astype(np.int8)
+    b4 = synth.encode_kquant(w, fl.FL_GGML_Q4_K).reshape(-1, 144).copy()
+    b4[::3, 4:12] = 63 | (3 << 6)                      # sc = 63, mn low bits 3
+    b4[::3, 12:16] = 0xFF                              # mn = 63
+    b4[1::3, 4:12] = 0                                 # sc = mn = 0 -> only -dmin*0
+    x = synth.bf16_normal((2, inn), 77)
+    for t, blk in ((fl.FL_GGML_Q6_K, b6.reshape(-1)), (fl.FL_GGML_Q4_K, b4.reshape(-1))):
+        y = torch.zeros((2, out), dtype=torch.float32, device="cuda")
+        wsb = fl.fl_kquant_workspace_bytes(t, out, inn, 2)
+        ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        fl.fl_gemv_kquant(dev(torch, blk), t, out, inn, dev(torch, x), 2, y, ws, wsb)
+        torch.cuda.synchronize()
+        yref, mass = orc.gemv_kquant(blk, t, out, inn, x, with_mass=True)
+        check_close(y.cpu().numpy(), yref, mass, f"kquant edge {t}")
+
+
+def test_kquant_batched_mixed_types(env, orc):
+    torch, fl = env
+    mix = [(12, 2048, 2048), (14, 512, 2048), (12, 512, 2048), (14, 2048, 8192), (12, 1024, 4096)]
+    batch = 1
+    items, refs, keep = [], [], []
+    for i, (t, o, n) in enumerate(mix):
+        w = synth.gaussian_weights(o, n, 73, i)
+        blk = synth.encode_kquant(w, t)
+        x = synth.bf16_normal((batch, n), 74, i)
+        bd, xd = dev(torch, blk), dev(torch, x)
+        y = torch.zeros((batch, o), dtype=torch.float32, device="cuda")
+        keep += [bd, xd, y]
+        items.append((bd, t, o, n, xd, y))
+        refs.append(orc.gemv_kquant(blk, t, o, n, x, with_mass=True))
+    fl.fl_gemv_kquant_batched(fl.kquant_problems(items), len(items), batch)
+    torch.cuda.synchronize()
+    for (bd, t, o, n, xd, y), (yref, mass) in zip(items, refs):
+        check_close(y.cpu().numpy(), yref, mass, f"kq batched {t} {o}x{n}")
+
+
+def test_kquant_unsupported_type_fails_on_device_box(env):
+    torch, fl = env
+    x = torch.zeros((1, 256), dtype=torch.int16, device="cuda")
+    y = torch.zeros((1, 64), dtype=torch.float32, device="cuda")
+    blk = torch.zeros(64 * 176, dtype=torch.uint8, device="cuda")
+    with pytest.raises(fl.FlError) as e:
+        fl.fl_gemv_kquant(blk, 13, 64, 256, x, 1, y)
+    assert e.value.status == -3

@@ -1,0 +1,183 @@
+// Shared device helpers for libfl (sm_100a): status plumbing, mbarrier and
+// bulk-copy PTX, the int8 tensor-core instruction, and the per-group
+// fixed-point form of the activation vector used by the int8 products.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "../../include/fl.h"
+
+namespace fl {
+
+// ---------------------------------------------------------------- host status
+
+void set_error(const char* fmt, ...);
+fl_status fail(fl_status st, const char* fmt, ...);
+fl_status cuda_fail(cudaError_t e, const char* what);
+int device_sm_count();
+
+#define FL_CHECK_CUDA(call, what)                   \
+  do {                                              \
+    cudaError_t e__ = (call);                       \
+    if (e__ != cudaSuccess) return fl::cuda_fail(e__, what); \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- device PTX
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait on an mbarrier phase. Returns false (and leaves the caller to
+// record the failure) if the phase has not completed after `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 26)) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t k = 0; k < limit; ++k) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
+// 1-D bulk copy global -> shared (own CTA), completion counted on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t rotr32(uint32_t v, uint32_t n) {
+  return __funnelshift_r(v, v, n);
+}
+
+// D (s32 16x8) += A (u8 16x32, row) * B (s8 32x8, col).
+__device__ __forceinline__ void mma_u8s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D (s32 16x8) += A (u8 16x16, row) * B (s8 16x8, col).
+__device__ __forceinline__ void mma_u8s8_k16(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// ---------------------------------------------------------------- activations as int8 digits
+//
+// For the int8 tensor-core products each 128-column group of each activation
+// row is written as a 15-bit fixed-point integer  v_c = rint(x_c 2^sigma)
+// with sigma = 14 - E, where max_c |x_c| < 2^E, so |v_c| <= 2^14; v_c is then
+// split into two balanced signed bytes  v_c = 256 hi_c + lo_c,
+// hi_c in [-64, 64], lo_c in [-128, 127].  The group keeps 2^-sigma (to undo
+// the scaling) and sum_c v_c (for the constant part of the reconstruction).
+// Absolute error per element <= 2^(E - 15) <= 2^-14 max |x_c|.
+
+struct XDigitView {
+  int8_t* digits;      // [2 * batch_pad][stride]: row 2b = hi digits of batch b, 2b + 1 = lo digits
+  float* inv_scale;    // [batch_pad][ngroups] 2^-sigma
+  int32_t* gsum;       // [batch_pad][ngroups * sub] sums of v over each sub-group
+  int stride;          // bytes per digit row
+  int ngroups;
+};
+
+// Compute the digits of columns [col0, col0 + 128 * ngroups) of x (batch rows)
+// into smem. Called by `nthreads` threads starting at thread index `tid`.
+// `sub` = number of equal sub-groups per 128 columns whose sums are kept
+// (1 for the plane store, 4 for Q4_K, 8 for Q6_K). Digit rows exist for
+// b < batch only; for batch <= b < batch_pad the sums and scales are zeroed.
+//
+// `perm` = 1 stores the digits of each 32-column chunk in the order
+// (0-3, 16-19, 4-7, 20-23, 8-11, 24-27, 12-15, 28-31), so that the two k32
+// operand halves of one lane (columns 4t..4t+3 and 16+4t..16+4t+3 of the
+// chunk) are adjacent; `perm` = 0 keeps column order.
+__device__ __forceinline__ void build_x_digits(const uint16_t* __restrict__ x, int in, int batch, int batch_pad,
+                                               int col0, XDigitView v, int sub, int tid, int nthreads,
+                                               int perm = 0) {
+  // one warp per (batch row, group): 32 lanes x 4 columns
+  const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
+  const int per_sub = 128 / sub;
+  for (int item = wid; item < batch_pad * v.ngroups; item += nw) {
+    const int b = item / v.ngroups, g = item % v.ngroups;
+    if (b >= batch) {  // padding rows: no digits are stored, their sums and scales read as zero
+      if (lane == 0) v.inv_scale[b * v.ngroups + g] = 0.f;
+      if (lane < sub) v.gsum[(b * v.ngroups + g) * sub + lane] = 0;
+      continue;
+    }
+    int8_t* hi = v.digits + (size_t)(2 * b) * v.stride + 128 * g;
+    int8_t* lo = v.digits + (size_t)(2 * b + 1) * v.stride + 128 * g;
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)b * in + col0 + 128 * g + 4 * lane);
+    float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                  __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+    float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    int E = 0;
+    if (m > 0.f) {
+      frexpf(m, &E);  // m = mant * 2^E, mant in [0.5, 1)  ->  m < 2^E
+    }
+    const int sigma = (m > 0.f) ? (14 - E) : 0;
+    uint32_t hw = 0, lw = 0;
+    int part = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int vv = __float2int_rn(ldexpf(f[i], sigma));
+      const int h = (vv + 128) >> 8;
+      const int l = vv - 256 * h;
+      hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
+      lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
+      part += vv;
+    }
+    const int wpos = perm ? (8 * (lane >> 3) + 2 * (lane & 3) + ((lane >> 2) & 1)) : lane;
+    reinterpret_cast<uint32_t*>(hi)[wpos] = hw;
+    reinterpret_cast<uint32_t*>(lo)[wpos] = lw;
+    // sums over sub-groups of per_sub columns (per_sub / 4 lanes each)
+    const int lanes_per_sub = per_sub / 4;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+      if (o < lanes_per_sub) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane % lanes_per_sub == 0) v.gsum[(b * v.ngroups + g) * sub + lane / lanes_per_sub] = part;
+    if (lane == 0) v.inv_scale[b * v.ngroups + g] = ldexpf(1.0f, -sigma);
+  }
+}
+
+}  // namespace fl

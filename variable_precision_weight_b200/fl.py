@@ -1,0 +1,204 @@
+"""Thin Python binding over libfl.so: the C-ABI entry points under the same names.
+
+Argument marshalling only: tensors become raw pointers, ``stream=None`` means
+torch's current CUDA stream, and a non-zero status raises :class:`FlError`
+with the library's message. Every step of the read path runs in the CUDA
+library; importing this module fails loudly when libfl.so is missing (build it
+with ``python -m variable_precision_weight_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfl.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libfl.so not found at {LIB_PATH}; run `python -m variable_precision_weight_b200.build`")
+
+_lib = C.CDLL(LIB_PATH)
+
+FL_OK = 0
+FL_MAX_BATCH = 16
+FL_MAX_STOPS = 16
+FL_MAX_PROBLEMS = 256
+FL_GGML_Q4_K = 12
+FL_GGML_Q6_K = 14
+STATUS = {0: "FL_OK", -1: "FL_ERR_ARG", -2: "FL_ERR_SHAPE", -3: "FL_ERR_UNSUPPORTED", -4: "FL_ERR_ALIGN",
+          -5: "FL_ERR_CUDA", -6: "FL_ERR_WORKSPACE"}
+
+
+class FlError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class fl_plane_weight(C.Structure):
+    _fields_ = [("store", C.c_void_p), ("out", C.c_int), ("in_", C.c_int)]
+
+
+class fl_lens_params(C.Structure):
+    _fields_ = [("f", C.c_float), ("g", C.c_float), ("gamma", C.c_int), ("m", C.c_int), ("nstops", C.c_int),
+                ("stops", C.c_float * FL_MAX_STOPS), ("combine", C.c_int)]
+
+
+class fl_gemv_problem(C.Structure):
+    _fields_ = [("w", fl_plane_weight), ("levels", C.c_void_p), ("to_levels", C.c_void_p), ("x", C.c_void_p),
+                ("y", C.c_void_p)]
+
+
+class fl_kquant_problem(C.Structure):
+    _fields_ = [("blocks", C.c_void_p), ("ggml_type", C.c_int), ("out", C.c_int), ("in_", C.c_int),
+                ("x", C.c_void_p), ("y", C.c_void_p)]
+
+
+_P, _I, _F, _S = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+_sigs = {
+    "fl_status_string": (C.c_char_p, [_I]),
+    "fl_last_error": (C.c_char_p, []),
+    "fl_version": (_I, []),
+    "fl_plane_store_bytes": (_S, [_I, _I]),
+    "fl_pack_planes": (_I, [_P, _P, _I, _I, _P, _P]),
+    "fl_level_map": (_I, [_P, _I, _P, _P, _I, C.POINTER(fl_lens_params), _P, _P, _P]),
+    "fl_gemv_workspace_bytes": (_S, [_I, _I, _I]),
+    "fl_gemv_depth": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P, _S, _P]),
+    "fl_gemv_residual": (_I, [C.POINTER(fl_plane_weight), _P, _P, _P, _I, _P, _P, _S, _P]),
+    "fl_gemv_batched": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, _P]),
+    "fl_logit_gate": (_I, [_P, _I, _I, _F, _F, _P, _P, _P, _P, _P]),
+    "fl_kquant_bytes": (_S, [_I, _I, _I]),
+    "fl_kquant_workspace_bytes": (_S, [_I, _I, _I, _I]),
+    "fl_gemv_kquant": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _S, _P]),
+    "fl_gemv_kquant_batched": (_I, [C.POINTER(fl_kquant_problem), _I, _I, _P]),
+}
+for _name, (_res, _args) in _sigs.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_sigs)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _check(status: int) -> None:
+    if status != FL_OK:
+        raise FlError(status, (_lib.fl_last_error() or b"").decode())
+
+
+def fl_status_string(status: int) -> str:
+    return _lib.fl_status_string(status).decode()
+
+
+def fl_last_error() -> str:
+    return (_lib.fl_last_error() or b"").decode()
+
+
+def fl_version() -> int:
+    return int(_lib.fl_version())
+
+
+def fl_plane_store_bytes(out: int, inn: int) -> int:
+    return int(_lib.fl_plane_store_bytes(out, inn))
+
+
+def fl_pack_planes(codes, scales, out: int, inn: int, store, stream=None) -> None:
+    _check(_lib.fl_pack_planes(_ptr(codes), _ptr(scales), out, inn, _ptr(store), _stream(stream)))
+
+
+def plane_weight(store, out: int, inn: int) -> fl_plane_weight:
+    return fl_plane_weight(_ptr(store), out, inn)
+
+
+def lens_params(f: float, g: float, gamma: int, m: int, stops, combine: int) -> fl_lens_params:
+    p = fl_lens_params()
+    p.f, p.g, p.gamma, p.m, p.combine = float(f), float(g), int(gamma), int(m), int(combine)
+    stops = [float(s) for s in stops]
+    p.nstops = len(stops)
+    for i, s in enumerate(stops):
+        p.stops[i] = s
+    return p
+
+
+def fl_level_map(xy, nblocks: int, centers, radii, nlenses: int, params: fl_lens_params, levels, counts=None,
+                 stream=None) -> None:
+    _check(_lib.fl_level_map(_ptr(xy), nblocks, _ptr(centers), _ptr(radii), nlenses, C.byref(params), _ptr(levels),
+                             _ptr(counts), _stream(stream)))
+
+
+def fl_gemv_workspace_bytes(out: int, inn: int, batch: int) -> int:
+    return int(_lib.fl_gemv_workspace_bytes(out, inn, batch))
+
+
+def fl_gemv_depth(w: fl_plane_weight, levels, x, batch: int, y, workspace=None, workspace_bytes: int = 0,
+                  stream=None) -> None:
+    _check(_lib.fl_gemv_depth(C.byref(w), _ptr(levels), _ptr(x), batch, _ptr(y), _ptr(workspace), workspace_bytes,
+                              _stream(stream)))
+
+
+def fl_gemv_residual(w: fl_plane_weight, from_levels, to_levels, x, batch: int, y, workspace=None,
+                     workspace_bytes: int = 0, stream=None) -> None:
+    _check(_lib.fl_gemv_residual(C.byref(w), _ptr(from_levels), _ptr(to_levels), _ptr(x), batch, _ptr(y),
+                                 _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def gemv_problems(items) -> "C.Array":
+    """items: iterable of (store, out, in, levels, to_levels, x, y) -> fl_gemv_problem array."""
+    items = list(items)
+    arr = (fl_gemv_problem * len(items))()
+    for i, (store, out, inn, lv, lt, x, y) in enumerate(items):
+        arr[i] = fl_gemv_problem(fl_plane_weight(_ptr(store), out, inn), _ptr(lv), _ptr(lt), _ptr(x), _ptr(y))
+    return arr
+
+
+def fl_gemv_batched(problems, n: int, batch: int, mode: int, stream=None) -> None:
+    _check(_lib.fl_gemv_batched(problems, n, batch, mode, _stream(stream)))
+
+
+def fl_logit_gate(logits, vocab: int, batch: int, tau_h: float, tau_m: float, entropy, margin, top2, escalate,
+                  stream=None) -> None:
+    _check(_lib.fl_logit_gate(_ptr(logits), vocab, batch, float(tau_h), float(tau_m), _ptr(entropy), _ptr(margin),
+                              _ptr(top2), _ptr(escalate), _stream(stream)))
+
+
+def fl_kquant_bytes(ggml_type: int, out: int, inn: int) -> int:
+    return int(_lib.fl_kquant_bytes(ggml_type, out, inn))
+
+
+def fl_kquant_workspace_bytes(ggml_type: int, out: int, inn: int, batch: int) -> int:
+    return int(_lib.fl_kquant_workspace_bytes(ggml_type, out, inn, batch))
+
+
+def fl_gemv_kquant(blocks, ggml_type: int, out: int, inn: int, x, batch: int, y, workspace=None,
+                   workspace_bytes: int = 0, stream=None) -> None:
+    _check(_lib.fl_gemv_kquant(_ptr(blocks), ggml_type, out, inn, _ptr(x), batch, _ptr(y), _ptr(workspace),
+                               workspace_bytes, _stream(stream)))
+
+
+def kquant_problems(items) -> "C.Array":
+    """items: iterable of (blocks, ggml_type, out, in, x, y) -> fl_kquant_problem array."""
+    items = list(items)
+    arr = (fl_kquant_problem * len(items))()
+    for i, (blk, t, out, inn, x, y) in enumerate(items):
+        arr[i] = fl_kquant_problem(_ptr(blk), t, out, inn, _ptr(x), _ptr(y))
+    return arr
+
+
+def fl_gemv_kquant_batched(problems, n: int, batch: int, stream=None) -> None:
+    _check(_lib.fl_gemv_kquant_batched(problems, n, batch, _stream(stream)))

@@ -24,7 +24,8 @@ namespace cg = cooperative_groups;
 namespace fl {
 
 constexpr int kClusterCtas = 8;
-constexpr int kGateThreads = 256;
+constexpr int kGateThreads = 1024;
+constexpr int kGateUnroll = 8;  // float4 loads in flight per thread
 
 struct GateAcc {
   float m, S, T;   // running max, sum e^(z-m), sum (z-m) e^(z-m)
@@ -92,7 +93,7 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kGateThre
   // this CTA's slice, in float4 units
   const int n4 = vocab / 4;
   const int per = (n4 + kClusterCtas - 1) / kClusterCtas;
-  const int q0 = rank * per, q1 = min(n4, q0 + per);
+  const int q0s = rank * per, q1 = min(n4, q0s + per);
 
   GateAcc a;
   a.m = -INFINITY;
@@ -100,10 +101,18 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kGateThre
   a.T = 0.f;
   a.v1 = a.v2 = -INFINITY;
   a.i1 = a.i2 = 0x7fffffff;
-  for (int q = q0 + (int)threadIdx.x; q < q1; q += kGateThreads) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(z) + q);
-    const float e[4] = {v.x, v.y, v.z, v.w};
-    float mx = fmaxf(fmaxf(e[0], e[1]), fmaxf(e[2], e[3]));
+  // All of a thread's 16-byte loads are issued before any is used (a row slice is at most
+  // kGateUnroll float4 per thread for the vocabularies in use; longer rows loop).
+  for (int q0 = q0s + (int)threadIdx.x; q0 < q1; q0 += kGateThreads * kGateUnroll) {
+    float4 v[kGateUnroll];
+#pragma unroll
+    for (int k = 0; k < kGateUnroll; ++k) {
+      const int q = q0 + k * kGateThreads;
+      v[k] = (q < q1) ? __ldg(reinterpret_cast<const float4*>(z) + q) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+    float mx = a.m;
+#pragma unroll
+    for (int k = 0; k < kGateUnroll; ++k) mx = fmaxf(mx, fmaxf(fmaxf(v[k].x, v[k].y), fmaxf(v[k].z, v[k].w)));
     if (mx > a.m) {
       if (a.S > 0.f) {
         const float r = expf(a.m - mx);
@@ -113,12 +122,19 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kGateThre
       a.m = mx;
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float dz = e[k] - a.m;
-      const float ex = expf(dz);
-      a.S += ex;
-      a.T += dz * ex;
-      push_top2(a, e[k], 4 * q + k);
+    for (int k = 0; k < kGateUnroll; ++k) {
+      const int q = q0 + k * kGateThreads;
+      if (q < q1) {
+        const float e[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float dz = e[c] - a.m;
+          const float ex = expf(dz);
+          a.S += ex;
+          a.T += dz * ex;
+          push_top2(a, e[c], 4 * q + c);
+        }
+      }
     }
   }
   // warp, then CTA
@@ -130,10 +146,14 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kGateThre
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) s_warp[warp] = a;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    GateAcc c = s_warp[0];
-    for (int w = 1; w < kGateThreads / 32; ++w) merge(c, s_warp[w]);
-    s_cta = c;
+  if (warp == 0) {  // the 32 warp partials, merged by warp 0 with shuffles
+    GateAcc c = s_warp[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      GateAcc b = shfl_acc(c, o);
+      merge(c, b);
+    }
+    if (lane == 0) s_cta = c;
   }
   cluster.sync();
   if (rank == 0 && threadIdx.x == 0) {

@@ -9,24 +9,29 @@
 // and c_0 := 128, u_0 := 0 (the ZERO level contributes nothing).
 //
 // How (B200): one persistent CTA per SM, warp-specialised.
-//  * A producer warp walks the CTA's contiguous range of work units
-//    (problem, column slice, 64-row block) and, per tile of whole 128-column
-//    groups, issues 1-D bulk copies of the block's scales and of the planes
-//    the block's depth needs (a contiguous span per plane in the store) into
-//    a 4-stage shared-memory ring guarded by mbarriers. Planes the depth does
-//    not need are never fetched.
-//  * Eight consumer warps (4 m-tiles of 16 rows x 2 group parities) assemble,
-//    per 16 columns, the code bytes u_d from the plane words with one AND/OR
-//    per plane and one rotate (the store layout places each plane's field so
-//    that this yields u_d in byte lanes), and feed them as the u8 operand of
-//    mma.sync m16n8k32 against the activations written as two signed int8
-//    digits of a 15-bit per-group fixed point. Integer sums per 128-column
-//    group are turned into fp32 with the group scale and the constant part
-//    (c_d - 128) sum_c x_c, then accumulated in fp32.
-//  * When a layer has too few blocks to fill the GPU its columns are split
-//    into slices; each slice writes a partial to the caller's workspace and
-//    the last CTA to finish a block (an atomic ticket) adds the partials in
-//    slice order, so results are deterministic. No CTA ever waits on another.
+//  * Work unit = (problem, column slice, 64-row block); each CTA owns a
+//    contiguous, cost-balanced range of units.
+//  * Four consumer teams of four warps. A team owns whole units (its four
+//    warps are the block's four 16-row m-tiles, so a warp's row sums are
+//    final when the unit ends) and two private stages of the shared-memory
+//    ring. Units go to the teams round-robin.
+//  * A producer warp caches the levels of the CTA's units in shared memory,
+//    then walks the four teams' unit streams, claims a team's next free
+//    stage, writes a tile header and issues 1-D bulk copies of the scales and
+//    of the planes the block's depth needs (one copy when the tile spans the
+//    whole row). Planes the depth does not need are never fetched.
+//  * Per 128-column group a warp assembles the code bytes u_d of its rows
+//    from the plane words with one AND/OR per plane and one rotate per four
+//    columns (the store layout places each plane's field so that this yields
+//    u_d in byte lanes), feeds them as the u8 operand of mma.sync m16n8k32
+//    against the activations written as two signed int8 digits of a 15-bit
+//    per-group fixed point (built once per CTA for every slice it touches),
+//    and turns the int32 group sum into fp32 with the group scale and the
+//    constant part (c_b - c_a) sum_c x_c.
+//  * Layers with too few blocks to fill the GPU are split into column slices;
+//    a slice writes a partial to the caller's workspace and the last team to
+//    finish a block (atomic ticket) adds the slices in order. No CTA ever
+//    waits on another; every mbarrier wait is bounded.
 #include <algorithm>
 #include <vector>
 
@@ -35,18 +40,24 @@
 namespace fl {
 namespace gemv {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStages = 4;
-constexpr int kStageBytes = 36864;
-constexpr int kMaxCtas = 512;
-constexpr int kSmemLimit = 232448 - 6144;  // opt-in shared memory per block on B200, less static use
+constexpr int kTeams = 4;
+constexpr int kTeamWarps = 4;
+constexpr int kTeamThreads = 32 * kTeamWarps;
+constexpr int kConsumerWarps = kTeams * kTeamWarps;
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kProducerWarps = kTeams;  // producer warp t feeds team t
+constexpr int kThreads = kConsumers + 32 * kProducerWarps;
+constexpr int kTeamStages = 2;
+constexpr int kStages = kTeams * kTeamStages;
+constexpr int kStageBytes = 18432;
+constexpr int kMaxCtas = 1024;
+constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
+constexpr int kLevelCache = 4096;     // units per CTA whose plane ranges are cached in smem
+constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
+constexpr int kDigitBudget = kSmemLimit - kStages * kStageBytes;
 
-// Groups per tile for a given number of planes: largest tg with
-// tg * (256 + 2048 np) <= kStageBytes.
-__host__ __device__ constexpr int tile_groups(int np) {
-  return np == 1 ? 16 : np == 2 ? 8 : np == 3 ? 5 : 4;
-}
+// Groups per tile for np planes: largest tg with tg * (256 + 2048 np) <= kStageBytes.
+__host__ __device__ constexpr int tile_groups(int np) { return np == 1 ? 8 : np == 2 ? 4 : 2; }
 
 struct Problem {
   const uint8_t* store;
@@ -68,17 +79,49 @@ struct Args {
   int nproblems;
   int batch;
   int mode;            // 0 depth (y =), 1 residual (y +=)
-  int digit_stride;    // bytes per digit row in smem
-  int max_slice_groups;
   int ncta;
   int cta_begin[kMaxCtas + 1];
   Problem p[MAXP];
 };
 
-__device__ int g_error;  // set on a bounded wait that ran out (never expected)
+__device__ int g_error;  // set when a bounded wait runs out (never expected)
+
+enum : int { kTileData = 0, kTileZero = 1, kTileEnd = 2 };
+enum : int { kFirst = 1, kLast = 2 };
+
+struct __align__(16) TileHdr {
+  int kind, flags;
+  int p, j, b;       // problem, slice, block
+  int k0, np;        // plane range read
+  int g0, tg;        // first group of the tile within the slice, groups in the tile
+  int slot;          // activation-digit slot of (p, j)
+  int slices;        // column slices of the problem
+  int ystride;       // 64 * nblocks = out
+  float* y;          // output of the problem
+};
+
+// One (problem, column slice) touched by a CTA: the units [u0, u1) of the CTA's range (relative
+// to its first unit) are its blocks b0, b0 + 1, ...; everything the producer and consumers need
+// is copied here once, so the hot loops never index the kernel-parameter problem table.
+// Activation digits: rows 2b / 2b+1 hold the hi / lo digits of batch row b (stride bytes per
+// row); gconst[(padded batch row) * ngroups + group] = (2^-sigma, 2^-sigma sum_c v_c).
+struct __align__(16) Slot {
+  int p, j, u0, u1, b0;
+  int nblocks, G, ngroups, slices, gfirst;  // gfirst = first group of the slice in the row
+  int stride;
+  uint32_t digits;   // smem address
+  uint32_t gconst;   // smem address
+  const uint8_t* store;
+  const uint8_t* lv_from;
+  const uint8_t* lv_to;
+  const uint16_t* x;
+  float* y;
+  float* partial;
+  uint32_t* tickets;
+};
 
 struct UnitCursor {
-  int p, j, b, u;  // problem, slice, block, global unit
+  int p, j, b, u;
 };
 
 template <int MAXP>
@@ -106,21 +149,6 @@ __device__ __forceinline__ void cursor_next(const Args<MAXP>& a, UnitCursor& c) 
   }
 }
 
-// Plane range [k0, k0 + np) read for a block.
-template <int MAXP>
-__device__ __forceinline__ void plane_range(const Args<MAXP>& a, const Problem& P, int b, int& k0, int& np) {
-  int lf = min((int)P.lv_from[b], 4);
-  if (a.mode == 0) {
-    k0 = 0;
-    np = lf;
-  } else {
-    int lt = min((int)P.lv_to[b], 4);
-    k0 = lf;
-    np = max(0, lt - lf);
-  }
-}
-
-__device__ __forceinline__ int slice_g0(const Problem& P, int j) { return j * P.slice_groups; }
 __device__ __forceinline__ int slice_ng(const Problem& P, int j) {
   return min(P.slice_groups, P.G - j * P.slice_groups);
 }
@@ -132,95 +160,167 @@ __host__ __device__ constexpr uint32_t plane_mask(int k, int i) {
              : ((0x03030303u << ((6 - 2 * k + 2 * i) & 7)) | (0x03030303u >> (32 - ((6 - 2 * k + 2 * i) & 7))));
 }
 
-// One 128-column group for one m-tile: 4 k32 MMAs per N-tile.
-// W[kk][r][w]: word w (0,1) of row r (0: g, 1: g + 8) of plane k0 + kk.
-template <int K0, int NP, int NT>
-__device__ __forceinline__ void group_mma(const uint2 (&W)[4][2], const uint4 (&B)[NT][2], int32_t (&C)[NT][4]) {
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int w = s >> 1;
-    const int i0 = 2 * (s & 1), i1 = i0 + 1;
-    uint32_t u[2][2];  // [row][i0/i1]
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int i = h ? i1 : i0;
-        uint32_t acc = 0;
-#pragma unroll
-        for (int kk = 0; kk < NP; ++kk) {
-          const uint32_t word = w ? W[kk][r].y : W[kk][r].x;
-          acc |= word & plane_mask(K0 + kk, i);
-        }
-        u[r][h] = (i == 0) ? acc : rotr32(acc, 2 * i);
-      }
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// c_b - c_a with c_0 = 128: the constant part of the read of planes [k0, k0 + np).
+__device__ __forceinline__ float cfac_of(int k0, int np) {
+  const int b = 2 * (k0 + np), a = 2 * k0;
+  const int cb2 = (1 << (8 - b)) - 1;
+  const int ca2 = (a == 0) ? 256 : (1 << (8 - a)) - 1;
+  return 0.5f * (float)(cb2 - ca2);
+}
+
+// Digits of columns [col0, col0 + 128 ngroups) of x into one slot (see fl_common.cuh for the
+// number format). Called by nthreads consumer threads, tid in [0, nthreads).
+__device__ __forceinline__ void build_slot(const uint16_t* __restrict__ x, int in, int batch, int batch_pad, int col0,
+                                           const Slot& sl, int tid, int nthreads) {
+  const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
+  for (int item = wid; item < batch_pad * sl.ngroups; item += nw) {
+    const int b = item / sl.ngroups, g = item % sl.ngroups;
+    const uint32_t gc = sl.gconst + 8u * (uint32_t)item;
+    if (b >= batch) {
+      if (lane == 0) asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(0.f), "f"(0.f) : "memory");
+      continue;
     }
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)b * in + col0 + 128 * g + 4 * lane);
+    const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+    float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t b0 = (s == 0) ? B[nt][0].x : (s == 1) ? B[nt][0].z : (s == 2) ? B[nt][1].x : B[nt][1].z;
-      const uint32_t b1 = (s == 0) ? B[nt][0].y : (s == 1) ? B[nt][0].w : (s == 2) ? B[nt][1].y : B[nt][1].w;
-      mma_u8s8(C[nt], u[0][0], u[1][0], u[0][1], u[1][1], b0, b1);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    int E = 0;
+    if (m > 0.f) frexpf(m, &E);
+    const int sigma = (m > 0.f) ? (14 - E) : 0;
+    uint32_t hw = 0, lw = 0;
+    int part = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int vv = __float2int_rn(ldexpf(f[i], sigma));
+      const int h = (vv + 128) >> 8;
+      const int l = vv - 256 * h;
+      hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
+      lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
+      part += vv;
     }
+    const uint32_t dh = sl.digits + (uint32_t)((2 * b) * sl.stride + 128 * g + 4 * lane);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh), "r"(hw) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)sl.stride), "r"(lw) : "memory");
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0)
+      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(ldexpf(1.0f, -sigma)),
+                   "f"(ldexpf((float)part, -sigma))
+                   : "memory");
   }
 }
 
+// One tile for one warp: all tg groups of the tile for rows r0 = 16 mt + g and r0 + 8.
+// Per group: plane words, activation digits, code bytes by mask/or/rotate, 4 k32 MMAs per
+// N-tile in two independent chains, then the group's scale and constant part in fp32.
 template <int K0, int NP, int NT>
-__device__ __forceinline__ void tile_compute(const uint8_t* stage, int tg, int gl_begin, int slice_goff,
-                                             const int8_t* digits, int digit_stride, int ndrows,
-                                             const float* inv_scale, const int32_t* gsum, int ngroups_slice,
-                                             int two_c, int mt, int lane, float (&acc)[NT][2]) {
-  const int g = lane >> 2, t = lane & 3;
-  const int r0 = 16 * mt + g;
-  const uint8_t* planes = stage + 256 * tg;
-  for (int gl = gl_begin; gl < tg; gl += 2) {
-    const int gs = slice_goff + gl;  // group index within the slice
-    uint4 B[NT][2];
+__device__ __forceinline__ void tile_compute(uint32_t stage, int tg, const uint32_t (&dlane)[NT],
+                                             const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
+                                             int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
+  constexpr int TG = tile_groups(NP);
+  const uint32_t planes = stage + 256u * tg;
+  const uint32_t wrow = planes + 32u * r0 + 8u * t;
+  const uint32_t srow = stage + 4u * r0;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int row = 8 * nt + g;
-      if (row < ndrows) {
-        const uint4* src = reinterpret_cast<const uint4*>(digits + (size_t)row * digit_stride + 128 * gs + 32 * t);
-        B[nt][0] = src[0];
-        B[nt][1] = src[1];
-      } else {
-        B[nt][0] = make_uint4(0, 0, 0, 0);
-        B[nt][1] = make_uint4(0, 0, 0, 0);
+  for (int gl = 0; gl < TG; ++gl) {
+    if (gl < tg) {
+      const int gs = slice_goff + gl;
+      uint2 W[NP][2];
+#pragma unroll
+      for (int kk = 0; kk < NP; ++kk) {
+        const uint32_t pk = wrow + 2048u * (kk * tg + gl);
+        W[kk][0] = lds_v2(pk);
+        W[kk][1] = lds_v2(pk + 256u);
       }
-    }
-    uint2 W[4][2];
+      uint4 B[NT][2];
 #pragma unroll
-    for (int kk = 0; kk < NP; ++kk) {
-      const uint8_t* pk = planes + 2048 * (kk * tg + gl);
-      W[kk][0] = *reinterpret_cast<const uint2*>(pk + 32 * r0 + 8 * t);
-      W[kk][1] = *reinterpret_cast<const uint2*>(pk + 32 * (r0 + 8) + 8 * t);
-    }
-    int32_t C[NT][4];
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t src = dlane[nt] + dstep[nt] * (uint32_t)gs;
+        B[nt][0] = lds_v4(src);
+        B[nt][1] = lds_v4(src + 16u);
+      }
+      const float s0 = lds_f32(srow + 256u * gl), s1 = lds_f32(srow + 256u * gl + 32u);
+      int32_t C[NT][4], D[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) C[nt][0] = C[nt][1] = C[nt][2] = C[nt][3] = 0;
-    group_mma<K0, NP, NT>(W, B, C);
-    const float* sc = reinterpret_cast<const float*>(stage + 256 * gl);
-    const float s0 = sc[r0], s1 = sc[r0 + 8];
+      for (int nt = 0; nt < NT; ++nt) {
+        C[nt][0] = C[nt][1] = C[nt][2] = C[nt][3] = 0;
+        D[nt][0] = D[nt][1] = D[nt][2] = D[nt][3] = 0;
+      }
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int bb = 4 * nt + t;  // batch row held by this lane
-      const int32_t X = gsum[bb * ngroups_slice + gs];
-      const float h = 0.5f * inv_scale[bb * ngroups_slice + gs];
-      const int32_t v0 = C[nt][0] * 512 + C[nt][1] * 2 + two_c * X;
-      const int32_t v1 = C[nt][2] * 512 + C[nt][3] * 2 + two_c * X;
-      acc[nt][0] = fmaf(static_cast<float>(v0), s0 * h, acc[nt][0]);
-      acc[nt][1] = fmaf(static_cast<float>(v1), s1 * h, acc[nt][1]);
+      for (int st = 0; st < 4; ++st) {
+        const int w = st >> 1;
+        const int i0 = 2 * (st & 1), i1 = i0 + 1;
+        uint32_t u[2][2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int i = h ? i1 : i0;
+            uint32_t v = 0;
+#pragma unroll
+            for (int kk = 0; kk < NP; ++kk) v |= (w ? W[kk][r].y : W[kk][r].x) & plane_mask(K0 + kk, i);
+            u[r][h] = (i == 0) ? v : rotr32(v, 2 * i);
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint32_t b0 = (st == 0) ? B[nt][0].x : (st == 1) ? B[nt][0].z : (st == 2) ? B[nt][1].x : B[nt][1].z;
+          const uint32_t b1 = (st == 0) ? B[nt][0].y : (st == 1) ? B[nt][0].w : (st == 2) ? B[nt][1].y : B[nt][1].w;
+          if (st < 2)
+            mma_u8s8(C[nt], u[0][0], u[1][0], u[0][1], u[1][1], b0, b1);
+          else
+            mma_u8s8(D[nt], u[0][0], u[1][0], u[0][1], u[1][1], b0, b1);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float2 hc = lds_f2(gc_lane + 8u * (uint32_t)(nt * 4 * gstride + gs));
+        const float off = cfac * hc.y;
+        const float v0 = fmaf((float)((C[nt][0] + D[nt][0]) * 256 + (C[nt][1] + D[nt][1])), hc.x, off);
+        const float v1 = fmaf((float)((C[nt][2] + D[nt][2]) * 256 + (C[nt][3] + D[nt][3])), hc.x, off);
+        acc[nt][0] = fmaf(v0, s0, acc[nt][0]);
+        acc[nt][1] = fmaf(v1, s1, acc[nt][1]);
+      }
     }
   }
 }
 
 template <int NT>
-__device__ __forceinline__ void dispatch_tile(int k0, int np, const uint8_t* stage, int tg, int gl_begin,
-                                              int slice_goff, const int8_t* digits, int digit_stride, int ndrows,
-                                              const float* inv_scale, const int32_t* gsum, int ngs, int two_c,
-                                              int mt, int lane, float (&acc)[NT][2]) {
-#define FL_TILE(K0_, NP_)                                                                                        \
-  tile_compute<K0_, NP_, NT>(stage, tg, gl_begin, slice_goff, digits, digit_stride, ndrows, inv_scale, gsum, ngs, \
-                             two_c, mt, lane, acc)
+__device__ __forceinline__ void dispatch_tile(int k0, int np, uint32_t stage, int tg, const uint32_t (&dlane)[NT],
+                                              const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
+                                              int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
+#define FL_TILE(K0_, NP_) \
+  tile_compute<K0_, NP_, NT>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc)
   switch (k0 * 8 + np) {
     case 0 * 8 + 1: FL_TILE(0, 1); break;
     case 0 * 8 + 2: FL_TILE(0, 2); break;
@@ -237,212 +337,299 @@ __device__ __forceinline__ void dispatch_tile(int k0, int np, const uint8_t* sta
 #undef FL_TILE
 }
 
-// 2 (c_b - c_a) with c_0 = 128: the constant part of the read, doubled so it is an integer.
-__device__ __forceinline__ int two_c_of(int k0, int np) {
-  const int b = 2 * (k0 + np), a = 2 * k0;
-  const int cb2 = (1 << (8 - b)) - 1;
-  const int ca2 = (a == 0) ? 256 : (1 << (8 - a)) - 1;
-  return cb2 - ca2;
-}
-
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+// Plane range [k0, k0 + np) read for block b, packed as k0 << 4 | np.
+__device__ __forceinline__ int plane_range(int mode, const uint8_t* lv_from, const uint8_t* lv_to, int b) {
+  const int lf = min((int)__ldg(lv_from + b), 4);
+  if (mode == 0) return lf;
+  const int lt = min((int)__ldg(lv_to + b), 4);
+  return (lf << 4) | max(0, lt - lf);
 }
 
 template <int MAXP, int NT>
 __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ float xfer[4][NT][2][32];  // gp = 1 warps hand their sums to gp = 0
-  __shared__ int s_ticket;
+  __shared__ TileHdr hdr[kStages];
+  __shared__ Slot slots[kMaxSlots];
+  __shared__ uint8_t lvc[kLevelCache];
+  __shared__ __align__(16) uint8_t zeros[160];
+  __shared__ int s_ticket[kTeams];
+  __shared__ int s_nslots;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u_begin = a.cta_begin[blockIdx.x], u_end = a.cta_begin[blockIdx.x + 1];
   if (u_begin >= u_end) return;
+  const int nunits = u_end - u_begin;
 
-  uint8_t* stages = smem;
-  int8_t* digits = reinterpret_cast<int8_t*>(smem + kStages * kStageBytes);
-  const int ndrows = 2 * a.batch;
-  float* inv_scale = reinterpret_cast<float*>(smem + kStages * kStageBytes + (size_t)ndrows * a.digit_stride);
-  int32_t* gsum = reinterpret_cast<int32_t*>(inv_scale + 4 * NT * a.max_slice_groups);
-
+  if (threadIdx.x < 40) reinterpret_cast<uint32_t*>(zeros)[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kConsumerWarps);
+      mbar_init(&empty_bar[s], kTeamWarps);
     }
     fence_mbar_init();
+    // one slot per distinct (problem, slice) of the range, digits laid out back to back
+    uint32_t off = 0;
+    int n = 0;
+    const uint32_t base = smem_u32(smem + kStages * kStageBytes);
+    UnitCursor c = cursor_at(a, u_begin);
+    int u = u_begin;
+    while (u < u_end && n < kMaxSlots) {
+      const Problem& P = a.p[c.p];
+      const int slice_end = P.unit_begin + (c.j + 1) * P.nblocks;  // first unit after this slice
+      Slot sl;
+      sl.p = c.p;
+      sl.j = c.j;
+      sl.u0 = u - u_begin;
+      sl.u1 = min(u_end, slice_end) - u_begin;
+      sl.b0 = c.b;
+      sl.nblocks = P.nblocks;
+      sl.G = P.G;
+      sl.ngroups = slice_ng(P, c.j);
+      sl.slices = P.slices;
+      sl.gfirst = c.j * P.slice_groups;
+      sl.stride = 128 * sl.ngroups + 16;
+      sl.digits = base + off;
+      off += 2 * a.batch * sl.stride;
+      sl.gconst = base + off;
+      off += 8 * 4 * NT * sl.ngroups;
+      sl.store = P.store;
+      sl.lv_from = P.lv_from;
+      sl.lv_to = P.lv_to;
+      sl.x = P.x;
+      sl.y = P.y;
+      sl.partial = P.partial;
+      sl.tickets = P.tickets;
+      slots[n++] = sl;
+      u = min(u_end, slice_end);
+      if (u < u_end) {
+        c.b = 0;
+        if (++c.j == P.slices) {
+          c.j = 0;
+          ++c.p;
+        }
+      }
+    }
+    s_nslots = n;
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0;
-      UnitCursor c = cursor_at(a, u_begin);
-      for (; c.u < u_end; cursor_next(a, c)) {
-        const Problem& P = a.p[c.p];
-        int k0, np;
-        plane_range(a, P, c.b, k0, np);
-        if (np == 0) continue;
-        const int tgm = tile_groups(np);
-        const int g0s = slice_g0(P, c.j), ngs = slice_ng(P, c.j);
-        const uint8_t* blk = P.store + (size_t)c.b * 8448u * P.G;
-        for (int g0 = 0; g0 < ngs; g0 += tgm) {
-          const int tg = min(tgm, ngs - g0);
-          if (issued >= (uint32_t)kStages) {
-            if (!mbar_wait(&empty_bar[s], phase ^ 1u)) {
-              atomicExch(&g_error, 1);
-              return;
-            }
-          }
-          uint8_t* st = stages + s * kStageBytes;
-          const uint32_t bytes = 256u * tg + 2048u * tg * np;
-          mbar_expect_tx(&full_bar[s], bytes);
-          const int gg = g0s + g0;
-          bulk_g2s(st, blk + 256u * gg, 256u * tg, &full_bar[s]);
-          for (int kk = 0; kk < np; ++kk)
-            bulk_g2s(st + 256 * tg + 2048 * tg * kk, blk + 256u * P.G + 2048u * ((size_t)P.G * (k0 + kk) + gg),
-                     2048u * tg, &full_bar[s]);
-          ++issued;
-          if (++s == kStages) {
-            s = 0;
-            phase ^= 1u;
-          }
+  if (warp >= kConsumerWarps) {
+    // ---------------------------------------------------------------- producer warps
+    const int nsl = s_nslots;
+    // 1. plane ranges of the CTA's units into the level cache (all producer threads)
+    {
+      int si = 0;
+      for (int k = threadIdx.x - kConsumers; k < nunits && k < kLevelCache; k += 32 * kProducerWarps) {
+        while (si + 1 < nsl && k >= slots[si].u1) ++si;
+        const Slot& sl = slots[si];
+        lvc[k] = (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, sl.b0 + (k - sl.u0));
+      }
+    }
+    named_bar(6, 32 * kProducerWarps);
+    if (lane != 0) return;
+    // 2. producer warp t walks team t's units t, t + kTeams, ... of the range
+    const int team = warp - kConsumerWarps;
+    int issued = 0;
+    auto claim = [&](int& s) -> bool {
+      s = kTeamStages * team + (issued % kTeamStages);
+      if (issued >= kTeamStages) {
+        const uint32_t ph = (uint32_t)((issued / kTeamStages - 1) & 1);
+        if (!mbar_wait(&empty_bar[s], ph)) {
+          atomicExch(&g_error, 1);
+          return false;
         }
       }
+      return true;
+    };
+    bool ok = true;
+    int si = 0;
+    for (int k = team; k < nunits && ok; k += kTeams) {
+      while (si + 1 < nsl && k >= slots[si].u1) ++si;
+      const Slot& sl = slots[si];
+      const int b = sl.b0 + (k - sl.u0);
+      const int pr = (k < kLevelCache) ? (int)lvc[k] : plane_range(a.mode, sl.lv_from, sl.lv_to, b);
+      const int k0 = pr >> 4, np = pr & 15;
+      int s;
+      if (np == 0) {
+        if (a.mode == 0 && sl.j == 0 && (ok = claim(s))) {
+          TileHdr& h = hdr[s];
+          h.kind = kTileZero;
+          h.flags = kFirst | kLast;
+          h.p = sl.p;
+          h.j = sl.j;
+          h.b = b;
+          h.slot = si;
+          h.ystride = 64 * sl.nblocks;
+          h.y = sl.y;
+          mbar_arrive(&full_bar[s]);
+          ++issued;
+        }
+        continue;
+      }
+      const int tgm = tile_groups(np);
+      const int ngs = sl.ngroups;
+      const uint8_t* blk = sl.store + (size_t)b * 8448u * sl.G;
+      for (int g0 = 0; g0 < ngs && ok; g0 += tgm) {
+        const int tg = min(tgm, ngs - g0);
+        if (!(ok = claim(s))) break;
+        TileHdr& h = hdr[s];
+        h.kind = kTileData;
+        h.flags = (g0 == 0 ? kFirst : 0) | (g0 + tg >= ngs ? kLast : 0);
+        h.p = sl.p;
+        h.j = sl.j;
+        h.b = b;
+        h.k0 = k0;
+        h.np = np;
+        h.g0 = g0;
+        h.tg = tg;
+        h.slot = si;
+        h.slices = sl.slices;
+        h.ystride = 64 * sl.nblocks;
+        h.y = sl.y;
+        uint8_t* st = smem + s * kStageBytes;
+        const int gg = sl.gfirst + g0;
+        const uint32_t bytes = 256u * tg + 2048u * tg * np;
+        mbar_expect_tx(&full_bar[s], bytes);
+        if (tg == sl.G && k0 == 0) {
+          bulk_g2s(st, blk, bytes, &full_bar[s]);  // the whole depth-d prefix of the block
+        } else {
+          bulk_g2s(st, blk + 256u * gg, 256u * tg, &full_bar[s]);
+          for (int kk = 0; kk < np; ++kk)
+            bulk_g2s(st + 256 * tg + 2048 * tg * kk, blk + 256u * sl.G + 2048u * ((size_t)sl.G * (k0 + kk) + gg),
+                     2048u * tg, &full_bar[s]);
+        }
+        ++issued;
+      }
+    }
+    int s;
+    if (ok && claim(s)) {
+      hdr[s].kind = kTileEnd;
+      mbar_arrive(&full_bar[s]);
     }
     return;
   }
 
-  // -------------------------------------------------------------- consumers
-  const int mt = warp & 3, gp = warp >> 2;
-  int s = 0;
-  uint32_t phase = 0;
-  int cur_p = -1, cur_j = -1;
-  UnitCursor c = cursor_at(a, u_begin);
-  for (; c.u < u_end; cursor_next(a, c)) {
-    const Problem& P = a.p[c.p];
-    const int ngs = slice_ng(P, c.j);
-    if (c.p != cur_p || c.j != cur_j) {
-      named_bar(1, 32 * kConsumerWarps);
-      XDigitView v;
-      v.digits = digits;
-      v.inv_scale = inv_scale;
-      v.gsum = gsum;
-      v.stride = a.digit_stride;
-      v.ngroups = ngs;
-      build_x_digits(P.x, P.G * 128, a.batch, 4 * NT, 128 * slice_g0(P, c.j), v, 1, threadIdx.x,
-                     32 * kConsumerWarps);
-      named_bar(1, 32 * kConsumerWarps);
-      cur_p = c.p;
-      cur_j = c.j;
+  // ------------------------------------------------------------------ consumer warps
+  // 1. activation digits of every (problem, slice) the range touches
+  for (int i = 0; i < s_nslots; ++i) {
+    const Slot& sl = slots[i];
+    build_slot(sl.x, sl.G * 128, a.batch, 4 * NT, 128 * sl.gfirst, sl, threadIdx.x, kConsumers);
+  }
+  named_bar(1, kConsumers);
+
+  // 2. team loop
+  const int team = warp / kTeamWarps, mt = warp % kTeamWarps;
+  const int tt = threadIdx.x % kTeamThreads;
+  const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * mt + g;
+  const uint32_t smem_base = smem_u32(smem);
+  float acc[NT][2];
+  float cfac = 0.f;
+  int cur_slot = -1;
+  uint32_t dlane[NT], dstep[NT], gc_lane = 0;
+  int gstride = 1;
+  for (int k = 0;; ++k) {
+    const int s = kTeamStages * team + (k % kTeamStages);
+    if (!mbar_wait(&full_bar[s], (uint32_t)((k / kTeamStages) & 1))) {
+      if (lane == 0) atomicExch(&g_error, 2);
+      return;
     }
-    int k0, np;
-    plane_range(a, P, c.b, k0, np);
-    const int row_base = 64 * c.b + 16 * mt;
-    const int g = lane >> 2, t = lane & 3;
-    if (np == 0) {
-      if (a.mode == 0 && c.j == 0 && gp == 0) {
-        for (int nt = 0; nt < NT; ++nt) {
-          const int bb = 4 * nt + t;
-          if (bb < a.batch) {
-            P.y[(size_t)bb * 64 * P.nblocks + row_base + g] = 0.f;
-            P.y[(size_t)bb * 64 * P.nblocks + row_base + g + 8] = 0.f;
-          }
+    TileHdr h;
+    {
+      const uint4* hv = reinterpret_cast<const uint4*>(&hdr[s]);
+      uint4* dv = reinterpret_cast<uint4*>(&h);
+#pragma unroll
+      for (int q = 0; q < (int)(sizeof(TileHdr) / 16); ++q) dv[q] = hv[q];
+    }
+    if (h.kind == kTileEnd) break;
+    const size_t ystride = (size_t)h.ystride;
+    const int row_base = 64 * h.b + 16 * mt;
+    if (h.kind == kTileZero) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int bb = 4 * nt + t;
+        if (bb < a.batch) {
+          h.y[(size_t)bb * ystride + row_base + g] = 0.f;
+          h.y[(size_t)bb * ystride + row_base + g + 8] = 0.f;
         }
       }
       continue;
     }
-    float acc[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-    const int tgm = tile_groups(np);
-    const int two_c = two_c_of(k0, np);
-    for (int g0 = 0; g0 < ngs; g0 += tgm) {
-      const int tg = min(tgm, ngs - g0);
-      if (!mbar_wait(&full_bar[s], phase)) {
-        atomicExch(&g_error, 2);
-        return;
-      }
-      dispatch_tile<NT>(k0, np, stages + s * kStageBytes, tg, gp, g0, digits, a.digit_stride, ndrows, inv_scale,
-                        gsum, ngs, two_c, mt, lane, acc);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-      if (++s == kStages) {
-        s = 0;
-        phase ^= 1u;
-      }
-    }
-    // combine the two group parities of each m-tile
-    if (gp == 1) {
+    if (h.slot != cur_slot) {
+      cur_slot = h.slot;
+      const Slot& sl = slots[h.slot];
+      gstride = sl.ngroups;
+      gc_lane = sl.gconst + 8u * (uint32_t)(t * sl.ngroups);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        xfer[mt][nt][0][lane] = acc[nt][0];
-        xfer[mt][nt][1][lane] = acc[nt][1];
+        const int row = 8 * nt + g;
+        const bool liveb = row < 2 * a.batch;
+        dlane[nt] = liveb ? sl.digits + (uint32_t)(row * sl.stride + 32 * t) : smem_u32(zeros + 32 * t);
+        dstep[nt] = liveb ? 128u : 0u;
       }
     }
-    named_bar(2 + mt, 64);
-    if (gp == 0) {
+    if (h.flags & kFirst) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
+      cfac = cfac_of(h.k0, h.np);
+    }
+    dispatch_tile<NT>(h.k0, h.np, smem_base + s * kStageBytes, h.tg, dlane, dstep, gc_lane, gstride, h.g0, cfac, r0,
+                      t, acc);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    if (!(h.flags & kLast)) continue;
+
+    // ---- unit done: this warp's 16 rows are final (or a slice partial)
+    if (h.slices == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        acc[nt][0] += xfer[mt][nt][0][lane];
-        acc[nt][1] += xfer[mt][nt][1][lane];
-      }
-    }
-    named_bar(2 + mt, 64);
-    const size_t ystride = (size_t)64 * P.nblocks;
-    if (P.slices == 1) {
-      if (gp == 0) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int bb = 4 * nt + t;
-          if (bb < a.batch) {
-            float* y0 = P.y + (size_t)bb * ystride + row_base + g;
-            if (a.mode == 0) {
-              y0[0] = acc[nt][0];
-              y0[8] = acc[nt][1];
-            } else {
-              y0[0] += acc[nt][0];
-              y0[8] += acc[nt][1];
-            }
+        const int bb = 4 * nt + t;
+        if (bb < a.batch) {
+          float* y0 = h.y + (size_t)bb * ystride + row_base + g;
+          if (a.mode == 0) {
+            y0[0] = acc[nt][0];
+            y0[8] = acc[nt][1];
+          } else {
+            y0[0] += acc[nt][0];
+            y0[8] += acc[nt][1];
           }
         }
       }
     } else {
-      // partial for this slice, then the last slice to finish reduces in slice order
-      if (gp == 0) {
+      // partial for this slice; the last team to finish the block adds the slices in order
+      const Slot& P = slots[h.slot];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int bb = 4 * nt + t;
-          if (bb < a.batch) {
-            float* pp = P.partial + (((size_t)c.j * P.nblocks + c.b) * a.batch + bb) * 64 + 16 * mt + g;
-            pp[0] = acc[nt][0];
-            pp[8] = acc[nt][1];
-          }
+      for (int nt = 0; nt < NT; ++nt) {
+        const int bb = 4 * nt + t;
+        if (bb < a.batch) {
+          float* pp = P.partial + (((size_t)h.j * P.nblocks + h.b) * a.batch + bb) * 64 + 16 * mt + g;
+          pp[0] = acc[nt][0];
+          pp[8] = acc[nt][1];
         }
       }
       __threadfence();
-      named_bar(1, 32 * kConsumerWarps);
-      if (threadIdx.x == 0) s_ticket = (int)atomicAdd(&P.tickets[c.b], 1u);
-      named_bar(1, 32 * kConsumerWarps);
-      if (s_ticket == P.slices - 1) {
+      named_bar(2 + team, kTeamThreads);
+      if (tt == 0) s_ticket[team] = (int)atomicAdd(&P.tickets[h.b], 1u);
+      named_bar(2 + team, kTeamThreads);
+      if (s_ticket[team] == P.slices - 1) {
         __threadfence();
-        for (int e = threadIdx.x; e < a.batch * 64; e += 32 * kConsumerWarps) {
+        for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
           const int bb = e / 64, r = e % 64;
           float sum = 0.f;
           for (int jj = 0; jj < P.slices; ++jj)
-            sum += __ldcg(P.partial + (((size_t)jj * P.nblocks + c.b) * a.batch + bb) * 64 + r);
-          float* yy = P.y + (size_t)bb * ystride + 64 * c.b + r;
+            sum += __ldcg(P.partial + (((size_t)jj * P.nblocks + h.b) * a.batch + bb) * 64 + r);
+          float* yy = h.y + (size_t)bb * ystride + 64 * h.b + r;
           if (a.mode == 0)
             *yy = sum;
           else
             *yy += sum;
         }
-        if (threadIdx.x == 0) P.tickets[c.b] = 0u;
+        if (tt == 0) P.tickets[h.b] = 0u;
       }
+      named_bar(2 + team, kTeamThreads);
     }
   }
 }
@@ -453,20 +640,15 @@ struct Plan {
   int slices, slice_groups;
 };
 
-static int digit_stride_for(int slice_groups) { return 128 * slice_groups + 16; }
-
-// Dynamic shared memory: stages, activation digits (2 rows per batch entry),
-// and per (padded batch, group) the inverse scale and the group sum.
-static size_t smem_bytes(int batch, int slice_groups) {
+static size_t slot_bytes(int batch, int ngroups) {
   const int nt = (batch + 3) / 4;
-  return (size_t)kStages * kStageBytes + (size_t)2 * batch * digit_stride_for(slice_groups) +
-         (size_t)4 * nt * slice_groups * 8;
+  return (size_t)2 * batch * (128 * ngroups + 16) + (size_t)8 * 4 * nt * ngroups;
 }
 
-// Widest column slice (in 128-column groups) whose digits fit next to the stages.
+// Widest column slice (in 128-column groups) whose digits fit in one slot.
 static int max_groups_fit(int batch) {
   const int nt = (batch + 3) / 4;
-  const long avail = (long)kSmemLimit - (long)kStages * kStageBytes - 32L * batch;
+  const long avail = (long)kDigitBudget - 32L * batch;
   return (int)std::max(1L, avail / (256L * batch + 32L * nt));
 }
 
@@ -474,9 +656,9 @@ static int max_groups_fit(int batch) {
 // groups, and a slice narrow enough for the activation digits to fit in smem.
 static Plan plan_single(int nblocks, int G, int batch, int nsm) {
   Plan pl;
-  int max_sg = max_groups_fit(batch);
-  int s_mem = (G + max_sg - 1) / max_sg;
-  int s_fill = (2 * nsm + nblocks - 1) / nblocks;
+  const int max_sg = max_groups_fit(batch);
+  const int s_mem = (G + max_sg - 1) / max_sg;
+  const int s_fill = (2 * nsm + nblocks - 1) / nblocks;
   int s = std::max(s_mem, std::min(s_fill, std::max(1, G / 4)));
   s = std::min(s, G);
   pl.slice_groups = (G + s - 1) / s;
@@ -486,39 +668,65 @@ static Plan plan_single(int nblocks, int G, int batch, int nsm) {
 
 static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
   if (pl.slices <= 1) return 0;
-  size_t tickets = ((size_t)nblocks * 4 + 255) / 256 * 256;
+  const size_t tickets = ((size_t)nblocks * 4 + 255) / 256 * 256;
   return tickets + (size_t)pl.slices * nblocks * batch * 64 * 4;
 }
 
+// Contiguous cost-balanced unit ranges, one per CTA (cost ~ columns read). A range is also
+// closed early when the digits of its distinct (problem, slice) pairs would overflow shared
+// memory, at kMaxSlots pairs, or at the level-cache size; such cuts can make more ranges than
+// SMs (a second, partial wave).
 template <int MAXP>
-static void partition(Args<MAXP>& a, int nsm) {
-  // cost of a unit ~ columns it reads; contiguous cost-balanced ranges per CTA
+static bool partition(Args<MAXP>& a, int nsm) {
   double total = 0;
   for (int i = 0; i < a.nproblems; ++i) total += (double)a.p[i].nblocks * a.p[i].G;
-  int units = a.p[a.nproblems - 1].unit_begin + a.p[a.nproblems - 1].nblocks * a.p[a.nproblems - 1].slices;
-  int ncta = std::min(nsm, units);
-  ncta = std::max(1, std::min(ncta, kMaxCtas));
-  a.ncta = ncta;
-  int c = 0;
+  const Problem& L = a.p[a.nproblems - 1];
+  const int units = L.unit_begin + L.nblocks * L.slices;
+  const int target = std::max(1, std::min(nsm, units));
+  const double per_cta = total / target;
+  int n = 0;
   a.cta_begin[0] = 0;
-  double acc = 0;
-  for (int i = 0; i < a.nproblems && c < ncta; ++i) {
+  double acc = 0;      // cumulative cost from the first unit
+  size_t dig = 0;      // digit bytes of the current range
+  int nslots = 0, count = 0;
+  for (int i = 0; i < a.nproblems; ++i) {
     const Problem& P = a.p[i];
-    const int nu = P.nblocks * P.slices;
-    const double per = (double)P.G / P.slices;
-    for (int k = 0; k < nu; ++k) {
-      acc += per;
-      const int u = P.unit_begin + k + 1;
-      while (c + 1 < ncta && acc >= total * (c + 1) / ncta) a.cta_begin[++c] = u;
+    for (int j = 0; j < P.slices; ++j) {
+      const int ng = std::min(P.slice_groups, P.G - j * P.slice_groups);
+      const size_t sb = slot_bytes(a.batch, ng);
+      const double cost = (double)ng;
+      for (int b = 0; b < P.nblocks; ++b) {
+        const int u = P.unit_begin + j * P.nblocks + b;
+        bool cut = false;
+        if (count > 0) {
+          if (n + 1 < target && acc + 0.5 * cost > per_cta * (n + 1)) cut = true;
+          if (b == 0 && (dig + sb > (size_t)kDigitBudget || nslots == kMaxSlots)) cut = true;
+          if (count == kLevelCache) cut = true;
+        }
+        if (cut) {
+          if (n + 1 >= kMaxCtas) return false;
+          a.cta_begin[++n] = u;
+          dig = 0;
+          nslots = 0;
+          count = 0;
+        }
+        if (b == 0 || count == 0) {
+          dig += sb;
+          ++nslots;
+        }
+        acc += cost;
+        ++count;
+      }
     }
   }
-  while (c + 1 < ncta) a.cta_begin[++c] = units;
-  a.cta_begin[ncta] = units;
+  a.cta_begin[++n] = units;
+  a.ncta = n;
+  return true;
 }
 
 template <int MAXP, int NT>
 static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
-  const size_t smem = smem_bytes(a.batch, a.max_slice_groups);
+  const size_t smem = (size_t)kSmemLimit;
   auto kern = plane_gemv_kernel<MAXP, NT>;
   FL_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                 "cudaFuncSetAttribute(plane_gemv)");
@@ -566,8 +774,6 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   a.nproblems = 1;
   a.batch = batch;
   a.mode = mode;
-  a.max_slice_groups = pl.slice_groups;
-  a.digit_stride = digit_stride_for(pl.slice_groups);
   Problem& P = a.p[0];
   P.store = w->store;
   P.lv_from = lv_from;
@@ -587,7 +793,7 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
     P.tickets = nullptr;
     P.partial = nullptr;
   }
-  partition(a, nsm);
+  if (!partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: layer too large for one launch", what);
   return launch_nt(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -626,7 +832,7 @@ extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int
   a.nproblems = n;
   a.batch = batch;
   a.mode = mode;
-  int max_g = 0, unit = 0;
+  int unit = 0;
   for (int i = 0; i < n; ++i) {
     const fl_gemv_problem& q = problems[i];
     fl_status st = gemv::check_weight(&q.w, what);
@@ -652,12 +858,9 @@ extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int
     P.slice_groups = G;
     P.unit_begin = unit;
     unit += P.nblocks;
-    max_g = std::max(max_g, G);
   }
-  a.max_slice_groups = max_g;
-  a.digit_stride = gemv::digit_stride_for(max_g);
   const int nsm = device_sm_count();
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
-  gemv::partition(a, nsm);
+  if (!gemv::partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: problems too large for one launch", what);
   return gemv::launch_nt(a, static_cast<cudaStream_t>(stream));
 }

@@ -23,8 +23,9 @@
 namespace fl {
 namespace kq {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kConsumerWarps = 16;
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kThreads = kConsumers + 32;
 constexpr int kStages = 4;
 constexpr int kStageBytes = 37888;
 constexpr int kMaxCtas = 512;
@@ -61,6 +62,16 @@ struct Args {
 
 __device__ int g_error;
 
+enum : int { kTileData = 0, kTileEnd = 2 };
+enum : int { kFirst = 1, kLast = 2, kNewX = 4 };
+struct TileHdr {
+  int kind, flags;
+  int p, j, b;
+  int sb0;   // first super-block of the tile within the slice
+  int tsb;   // super-blocks in the tile
+  int off;   // byte offset of the first record inside each row slot
+};
+
 struct Cursor {
   int p, j, b, u;
 };
@@ -90,7 +101,6 @@ __device__ __forceinline__ void cursor_next(const Args<MAXP>& a, Cursor& c) {
   }
 }
 
-__device__ __forceinline__ int slice_sb0(const Problem& P, int j) { return j * P.slice_sb; }
 __device__ __forceinline__ int slice_nsb(const Problem& P, int j) { return min(P.slice_sb, P.nsb - j * P.slice_sb); }
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
@@ -102,6 +112,7 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t h) {
 }
 
 __device__ __forceinline__ int byte_u(uint32_t w, int j) { return (int)__byte_perm(w, 0u, 0x4440u | (uint32_t)j); }
+
 // Byte j of w, sign-extended. Uses PTX prmt directly: its selector's top bit
 // replicates the selected byte's sign, which __byte_perm does not expose.
 __device__ __forceinline__ int byte_s(uint32_t w, int j) {
@@ -112,139 +123,135 @@ __device__ __forceinline__ int byte_s(uint32_t w, int j) {
   return (int)r;
 }
 
-// ---------------------------------------------------------------- Q4_K: one super-block, one m-tile
+__device__ __forceinline__ uint32_t lds_u32(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+  return v;
+}
+
+// ---------------------------------------------------------------- Q4_K: half (4 sub-blocks) of one super-block
 template <int NT>
-__device__ __forceinline__ void q4k_superblock(const uint8_t* rec0, const uint8_t* rec1, const int8_t* digits,
-                                               int digit_stride, int ndrows, int colg, const float* inv_scale,
-                                               const int32_t* gsum, int ngroups, int gidx0, int lane,
-                                               float (&acc)[NT][2]) {
-  const int g = lane >> 2, t = lane & 3;
-  const uint4 h0 = *reinterpret_cast<const uint4*>(rec0);
-  const uint4 h1 = *reinterpret_cast<const uint4*>(rec1);
+__device__ __forceinline__ void q4k_half(const uint8_t* rec0, const uint8_t* rec1, int half, const int8_t* const (&dl)[NT],
+                                         const int (&dstep)[NT], int colg, const float* inv_scale, const int32_t* gsum,
+                                         int gstride, int gi, int t, float (&acc)[NT][2]) {
+  const uint4 h0 = lds_v4(rec0);
+  const uint4 h1 = lds_v4(rec1);
   const float d0 = half_bits_to_float(h0.x), dm0 = half_bits_to_float(h0.x >> 16);
   const float d1 = half_bits_to_float(h1.x), dm1 = half_bits_to_float(h1.x >> 16);
-  const uint32_t sc0a = h0.y & 0x3F3F3F3Fu, sc0b = h0.z & 0x3F3F3F3Fu;
-  const uint32_t sc1a = h1.y & 0x3F3F3F3Fu, sc1b = h1.z & 0x3F3F3F3Fu;
+  const uint32_t S0 = half ? h0.z : h0.y, S1 = half ? h1.z : h1.y;
+  const uint32_t sc0 = S0 & 0x3F3F3F3Fu, sc1 = S1 & 0x3F3F3F3Fu;
   // mn_j bytes: low 2 bits from the top of byte j, high 4 bits from nibble j
-  auto mn_bytes = [](uint32_t S, uint32_t M16) -> uint32_t {
-    const uint32_t t1 = M16 & 0x0F0Fu, t2 = (M16 >> 4) & 0x0F0Fu;
-    const uint32_t nib = __byte_perm(t1, t2, 0x5140u);
-    return ((S >> 6) & 0x03030303u) | (nib << 2);
-  };
-  const uint32_t mn0a = mn_bytes(h0.y, h0.w & 0xFFFFu), mn0b = mn_bytes(h0.z, h0.w >> 16);
-  const uint32_t mn1a = mn_bytes(h1.y, h1.w & 0xFFFFu), mn1b = mn_bytes(h1.z, h1.w >> 16);
+  const uint32_t M0 = half ? (h0.w >> 16) : (h0.w & 0xFFFFu), M1 = half ? (h1.w >> 16) : (h1.w & 0xFFFFu);
+  const uint32_t mn0 = ((S0 >> 6) & 0x03030303u) | (__byte_perm(M0 & 0x0F0Fu, (M0 >> 4) & 0x0F0Fu, 0x5140u) << 2);
+  const uint32_t mn1 = ((S1 >> 6) & 0x03030303u) | (__byte_perm(M1 & 0x0F0Fu, (M1 >> 4) & 0x0F0Fu, 0x5140u) << 2);
+  uint32_t q0[4], q1[4];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    int32_t ai[NT][4];
+  for (int jj = 0; jj < 4; ++jj) {
+    const int j = 4 * half + jj;
+    q0[jj] = lds_u32(rec0 + 16 + 16 * j + 4 * t);
+    q1[jj] = lds_u32(rec1 + 16 + 16 * j + 4 * t);
+  }
+  int32_t ai[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = 0;
+  for (int nt = 0; nt < NT; ++nt) ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = 0;
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int j = 4 * half + jj;
-      const uint32_t q0 = *reinterpret_cast<const uint32_t*>(rec0 + 16 + 16 * j + 4 * t);
-      const uint32_t q1 = *reinterpret_cast<const uint32_t*>(rec1 + 16 + 16 * j + 4 * t);
-      const uint32_t a0 = q0 & 0x0F0F0F0Fu, a2 = (q0 >> 4) & 0x0F0F0F0Fu;
-      const uint32_t a1 = q1 & 0x0F0F0F0Fu, a3 = (q1 >> 4) & 0x0F0F0F0Fu;
-      const int s0 = byte_u(half ? sc0b : sc0a, jj), s1 = byte_u(half ? sc1b : sc1a, jj);
+  for (int jj = 0; jj < 4; ++jj) {
+    const int j = 4 * half + jj;
+    const uint32_t a0 = q0[jj] & 0x0F0F0F0Fu, a2 = (q0[jj] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t a1 = q1[jj] & 0x0F0F0F0Fu, a3 = (q1[jj] >> 4) & 0x0F0F0F0Fu;
+    const int s0 = byte_u(sc0, jj), s1 = byte_u(sc1, jj);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint2 bb = *reinterpret_cast<const uint2*>(dl[nt] + dstep[nt] * (colg + 32 * j));
+      int32_t C[4] = {0, 0, 0, 0};
+      mma_u8s8(C, a0, a1, a2, a3, bb.x, bb.y);
+      ai[nt][0] += s0 * C[0];
+      ai[nt][1] += s0 * C[1];
+      ai[nt][2] += s1 * C[2];
+      ai[nt][3] += s1 * C[3];
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int bb = 4 * nt + t;
+    const float isc = inv_scale[bb * gstride + gi];
+    // sums over the 32-column sub-blocks from the 16-column sums
+    const int4 Xa = *reinterpret_cast<const int4*>(gsum + (bb * gstride + gi) * 8);
+    const int4 Xb = *reinterpret_cast<const int4*>(gsum + (bb * gstride + gi) * 8 + 4);
+    const int32_t X0 = Xa.x + Xa.y, X1 = Xa.z + Xa.w, X2 = Xb.x + Xb.y, X3 = Xb.z + Xb.w;
+    const int32_t mx0 = byte_u(mn0, 0) * X0 + byte_u(mn0, 1) * X1 + byte_u(mn0, 2) * X2 + byte_u(mn0, 3) * X3;
+    const int32_t mx1 = byte_u(mn1, 0) * X0 + byte_u(mn1, 1) * X1 + byte_u(mn1, 2) * X2 + byte_u(mn1, 3) * X3;
+    const float v0 = fmaf(256.f, (float)ai[nt][0], (float)ai[nt][1]);
+    const float v1 = fmaf(256.f, (float)ai[nt][2], (float)ai[nt][3]);
+    acc[nt][0] = fmaf(isc, fmaf(d0, v0, -dm0 * (float)mx0), acc[nt][0]);
+    acc[nt][1] = fmaf(isc, fmaf(d1, v1, -dm1 * (float)mx1), acc[nt][1]);
+  }
+}
+
+// ---------------------------------------------------------------- Q6_K: half (8 sub-blocks of 16) of one super-block
+template <int NT>
+__device__ __forceinline__ void q6k_half(const uint8_t* rec0, const uint8_t* rec1, int odd, int half,
+                                         const int8_t* const (&dl)[NT], const int (&dstep)[NT], int colg,
+                                         const float* inv_scale, const int32_t* gsum, int gstride, int gi, int t,
+                                         float (&acc)[NT][2]) {
+  const uint8_t* qa0 = rec0 + (odd ? 2 : 0);
+  const uint8_t* qa1 = rec1 + (odd ? 2 : 0);
+  const uint8_t* sc0p = rec0 + (odd ? 194 : 192);
+  const uint8_t* sc1p = rec1 + (odd ? 194 : 192);
+  const float d0 = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec0 + (odd ? 0 : 208)));
+  const float d1 = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec1 + (odd ? 0 : 208)));
+  int32_t ai[NT][4], ao[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = ao[nt][0] = ao[nt][1] = 0;
+#pragma unroll
+  for (int mm = 0; mm < 2; ++mm) {
+    const int m = 2 * half + mm;
+    const uint8_t* w0 = qa0 + 48 * t + 12 * m;
+    const uint8_t* w1 = qa1 + 48 * t + 12 * m;
+    const uint32_t A0 = lds_u32(w0), B0 = lds_u32(w0 + 4), C0 = lds_u32(w0 + 8);
+    const uint32_t A1 = lds_u32(w1), B1 = lds_u32(w1 + 4), C1 = lds_u32(w1 + 8);
+    const uint32_t scw0 = lds_u32(sc0p + 4 * m), scw1 = lds_u32(sc1p + 4 * m);
+    uint32_t op0[4], op1[4];
+    op0[0] = (A0 & 0x0F0F0F0Fu) | (C0 & 0x30303030u);
+    op0[1] = ((A0 >> 4) & 0x0F0F0F0Fu) | ((C0 >> 2) & 0x30303030u);
+    op0[2] = (B0 & 0x0F0F0F0Fu) | ((C0 << 4) & 0x30303030u);
+    op0[3] = ((B0 >> 4) & 0x0F0F0F0Fu) | ((C0 << 2) & 0x30303030u);
+    op1[0] = (A1 & 0x0F0F0F0Fu) | (C1 & 0x30303030u);
+    op1[1] = ((A1 >> 4) & 0x0F0F0F0Fu) | ((C1 >> 2) & 0x30303030u);
+    op1[2] = (B1 & 0x0F0F0F0Fu) | ((C1 << 4) & 0x30303030u);
+    op1[3] = ((B1 >> 4) & 0x0F0F0F0Fu) | ((C1 << 2) & 0x30303030u);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int j = 4 * m + s;  // sub-block of 16 weights
+      const int s0 = byte_s(scw0, s), s1 = byte_s(scw1, s);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int row = 8 * nt + g;
-        uint2 bb = make_uint2(0u, 0u);
-        if (row < ndrows) bb = *reinterpret_cast<const uint2*>(digits + (size_t)row * digit_stride + colg + 32 * j + 8 * t);
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(dl[nt] + dstep[nt] * (colg + 16 * j));
         int32_t C[4] = {0, 0, 0, 0};
-        mma_u8s8(C, a0, a1, a2, a3, bb.x, bb.y);
+        mma_u8s8_k16(C, op0[s], op1[s], b0);
         ai[nt][0] += s0 * C[0];
         ai[nt][1] += s0 * C[1];
         ai[nt][2] += s1 * C[2];
         ai[nt][3] += s1 * C[3];
+        const int32_t X = gsum[((4 * nt + t) * gstride + gi) * 8 + (j & 7)];
+        ao[nt][0] += s0 * X;
+        ao[nt][1] += s1 * X;
       }
-    }
-    const int gi = gidx0 + half;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int bb = 4 * nt + t;
-      const float isc = inv_scale[bb * ngroups + gi];
-      const int32_t* X = gsum + (bb * ngroups + gi) * 4;  // 32-column sub-block sums
-      const uint32_t m0 = half ? mn0b : mn0a, m1 = half ? mn1b : mn1a;
-      int32_t mx0 = 0, mx1 = 0;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        mx0 += byte_u(m0, jj) * X[jj];
-        mx1 += byte_u(m1, jj) * X[jj];
-      }
-      const float v0 = fmaf(256.f, (float)ai[nt][0], (float)ai[nt][1]);
-      const float v1 = fmaf(256.f, (float)ai[nt][2], (float)ai[nt][3]);
-      acc[nt][0] = fmaf(isc, fmaf(d0, v0, -dm0 * (float)mx0), acc[nt][0]);
-      acc[nt][1] = fmaf(isc, fmaf(d1, v1, -dm1 * (float)mx1), acc[nt][1]);
     }
   }
-}
-
-// ---------------------------------------------------------------- Q6_K: one super-block, one m-tile
-template <int NT>
-__device__ __forceinline__ void q6k_superblock(const uint8_t* rec0, const uint8_t* rec1, int odd, const int8_t* digits,
-                                               int digit_stride, int ndrows, int colg, const float* inv_scale,
-                                               const int32_t* gsum, int ngroups, int gidx0, int lane,
-                                               float (&acc)[NT][2]) {
-  const int g = lane >> 2, t = lane & 3;
-  const uint8_t* qa0 = rec0 + (odd ? 2 : 0);
-  const uint8_t* qa1 = rec1 + (odd ? 2 : 0);
-  const uint32_t* sc0w = reinterpret_cast<const uint32_t*>(rec0 + (odd ? 194 : 192));
-  const uint32_t* sc1w = reinterpret_cast<const uint32_t*>(rec1 + (odd ? 194 : 192));
-  const float d0 = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec0 + (odd ? 0 : 208)));
-  const float d1 = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec1 + (odd ? 0 : 208)));
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    int32_t ai[NT][4], ao[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = ao[nt][0] = ao[nt][1] = 0;
-    const int gi = gidx0 + half;
-#pragma unroll
-    for (int mm = 0; mm < 2; ++mm) {
-      const int m = 2 * half + mm;
-      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(qa0 + 48 * t + 12 * m);
-      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(qa1 + 48 * t + 12 * m);
-      const uint32_t A0 = w0[0], B0 = w0[1], C0 = w0[2];
-      const uint32_t A1 = w1[0], B1 = w1[1], C1 = w1[2];
-      uint32_t op0[4], op1[4];
-      op0[0] = (A0 & 0x0F0F0F0Fu) | (C0 & 0x30303030u);
-      op0[1] = ((A0 >> 4) & 0x0F0F0F0Fu) | ((C0 >> 2) & 0x30303030u);
-      op0[2] = (B0 & 0x0F0F0F0Fu) | ((C0 << 4) & 0x30303030u);
-      op0[3] = ((B0 >> 4) & 0x0F0F0F0Fu) | ((C0 << 2) & 0x30303030u);
-      op1[0] = (A1 & 0x0F0F0F0Fu) | (C1 & 0x30303030u);
-      op1[1] = ((A1 >> 4) & 0x0F0F0F0Fu) | ((C1 >> 2) & 0x30303030u);
-      op1[2] = (B1 & 0x0F0F0F0Fu) | ((C1 << 4) & 0x30303030u);
-      op1[3] = ((B1 >> 4) & 0x0F0F0F0Fu) | ((C1 << 2) & 0x30303030u);
-      const uint32_t scw0 = sc0w[m], scw1 = sc1w[m];
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int j = 4 * m + s;  // sub-block (16 weights)
-        const int s0 = byte_s(scw0, s), s1 = byte_s(scw1, s);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int row = 8 * nt + g;
-          uint32_t b0 = 0u;
-          if (row < ndrows) b0 = *reinterpret_cast<const uint32_t*>(digits + (size_t)row * digit_stride + colg + 16 * j + 4 * t);
-          int32_t C[4] = {0, 0, 0, 0};
-          mma_u8s8_k16(C, op0[s], op1[s], b0);
-          ai[nt][0] += s0 * C[0];
-          ai[nt][1] += s0 * C[1];
-          ai[nt][2] += s1 * C[2];
-          ai[nt][3] += s1 * C[3];
-          const int32_t X = gsum[(( 4 * nt + t) * ngroups + gi) * 8 + (j & 7)];
-          ao[nt][0] += s0 * X;
-          ao[nt][1] += s1 * X;
-        }
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const float isc = inv_scale[(4 * nt + t) * ngroups + gi];
-      const float v0 = fmaf(256.f, (float)ai[nt][0], fmaf(-32.f, (float)ao[nt][0], (float)ai[nt][1]));
-      const float v1 = fmaf(256.f, (float)ai[nt][2], fmaf(-32.f, (float)ao[nt][1], (float)ai[nt][3]));
-      acc[nt][0] = fmaf(isc * d0, v0, acc[nt][0]);
-      acc[nt][1] = fmaf(isc * d1, v1, acc[nt][1]);
-    }
+  for (int nt = 0; nt < NT; ++nt) {
+    const float isc = inv_scale[(4 * nt + t) * gstride + gi];
+    const float v0 = fmaf(256.f, (float)ai[nt][0], fmaf(-32.f, (float)ao[nt][0], (float)ai[nt][1]));
+    const float v1 = fmaf(256.f, (float)ai[nt][2], fmaf(-32.f, (float)ao[nt][1], (float)ai[nt][3]));
+    acc[nt][0] = fmaf(isc * d0, v0, acc[nt][0]);
+    acc[nt][1] = fmaf(isc * d1, v1, acc[nt][1]);
   }
 }
 
@@ -252,7 +259,8 @@ template <int MAXP, int NT>
 __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ float xfer[4][NT][2][32];
+  __shared__ TileHdr hdr[kStages];
+  __shared__ __align__(16) uint8_t zeros[160];
   __shared__ int s_ticket;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -264,7 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   const int max_groups = 2 * a.max_slice_sb;
   float* inv_scale = reinterpret_cast<float*>(smem + kStages * kStageBytes + (size_t)ndrows * a.digit_stride);
   int32_t* gsum = reinterpret_cast<int32_t*>(inv_scale + 4 * NT * max_groups);
+  float* xfer = reinterpret_cast<float*>(gsum + 4 * NT * max_groups * 8);  // [4 mt][3][NT][64]
 
+  if (threadIdx.x < 40) reinterpret_cast<uint32_t*>(zeros)[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -275,15 +285,16 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   __syncthreads();
 
   if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer (all 32 lanes issue copies)
+    // ------------------------------------------------------------ producer warp: all lanes issue row copies
     int s = 0;
     uint32_t phase = 0, issued = 0;
+    int last_p = -1, last_j = -1;
     Cursor c = cursor_at(a, u_begin);
     for (; c.u < u_end; cursor_next(a, c)) {
       const Problem& P = a.p[c.p];
       const bool q4 = P.type == FL_GGML_Q4_K;
       const int rec = q4 ? 144 : 210, tsbm = q4 ? kQ4Tsb : kQ6Tsb, slot = q4 ? kQ4Slot : kQ6Slot;
-      const int sb0s = slice_sb0(P, c.j), nsbs = slice_nsb(P, c.j);
+      const int sb0s = c.j * P.slice_sb, nsbs = slice_nsb(P, c.j);
       for (int t0 = 0; t0 < nsbs; t0 += tsbm) {
         const int tsb = min(tsbm, nsbs - t0);
         if (issued >= (uint32_t)kStages) {
@@ -300,7 +311,24 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
         const size_t e_off = (start_off + (size_t)rec * tsb + 15) & ~(size_t)15;
         const uint32_t row_bytes = (uint32_t)(e_off - a_off);
         uint8_t* st = stages + s * kStageBytes;
-        if (lane == 0) mbar_expect_tx(&full_bar[s], row_bytes * 64u);
+        if (lane == 0) {
+          TileHdr& h = hdr[s];
+          h.kind = kTileData;
+          int fl = (t0 == 0 ? kFirst : 0) | (t0 + tsb >= nsbs ? kLast : 0);
+          if (t0 == 0 && (c.p != last_p || c.j != last_j)) fl |= kNewX;
+          h.flags = fl;
+          h.p = c.p;
+          h.j = c.j;
+          h.b = c.b;
+          h.sb0 = t0;
+          h.tsb = tsb;
+          h.off = (int)(start_off - a_off);
+          mbar_expect_tx(&full_bar[s], row_bytes * 64u);
+        }
+        if (t0 == 0) {
+          last_p = c.p;
+          last_j = c.j;
+        }
         __syncwarp();
         for (int r = lane; r < 64; r += 32) {
           const uint8_t* src = P.blocks + (size_t)(64 * c.b + r) * P.nsb * rec + a_off;
@@ -313,86 +341,110 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
         }
       }
     }
+    if (issued >= (uint32_t)kStages) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&empty_bar[s], phase ^ 1u);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return;
+    }
+    if (lane == 0) {
+      hdr[s].kind = kTileEnd;
+      mbar_arrive(&full_bar[s]);
+    }
     return;
   }
 
-  // -------------------------------------------------------------- consumers
-  const int mt = warp & 3, sp = warp >> 2;
+  // -------------------------------------------------------------- consumer warps
+  const int mt = warp & 3, sq = warp >> 2;
   const int g = lane >> 2, t = lane & 3;
+  const int r0 = 16 * mt + g;
+  const int8_t* dl_perm[NT];
+  const int8_t* dl_nat[NT];
+  int dstep[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int row = 8 * nt + g;
+    const bool live = row < ndrows;
+    dl_perm[nt] = live ? digits + (size_t)row * a.digit_stride + 8 * t : reinterpret_cast<const int8_t*>(zeros) + 8 * t;
+    dl_nat[nt] = live ? digits + (size_t)row * a.digit_stride + 4 * t : reinterpret_cast<const int8_t*>(zeros) + 4 * t;
+    dstep[nt] = live ? 1 : 0;
+  }
+  float acc[NT][2];
+  int gstride = 2;
   int s = 0;
   uint32_t phase = 0;
-  int cur_p = -1, cur_j = -1;
-  Cursor c = cursor_at(a, u_begin);
-  for (; c.u < u_end; cursor_next(a, c)) {
-    const Problem& P = a.p[c.p];
+  for (;;) {
+    if (!mbar_wait(&full_bar[s], phase)) {
+      if (lane == 0) atomicExch(&g_error, 2);
+      return;
+    }
+    const TileHdr h = hdr[s];
+    if (h.kind == kTileEnd) break;
+    const Problem& P = a.p[h.p];
     const bool q4 = P.type == FL_GGML_Q4_K;
-    const int rec = q4 ? 144 : 210, tsbm = q4 ? kQ4Tsb : kQ6Tsb, slot = q4 ? kQ4Slot : kQ6Slot;
-    const int sb0s = slice_sb0(P, c.j), nsbs = slice_nsb(P, c.j);
-    const int ngroups = 2 * nsbs;
-    if (c.p != cur_p || c.j != cur_j) {
-      named_bar(1, 32 * kConsumerWarps);
+    if (h.flags & kNewX) {
+      named_bar(1, kConsumers);
+      gstride = 2 * slice_nsb(P, h.j);
       XDigitView v;
       v.digits = digits;
       v.inv_scale = inv_scale;
       v.gsum = gsum;
       v.stride = a.digit_stride;
-      v.ngroups = ngroups;
-      build_x_digits(P.x, P.nsb * 256, a.batch, 4 * NT, 256 * sb0s, v, q4 ? 4 : 8, threadIdx.x,
-                     32 * kConsumerWarps, q4 ? 1 : 0);
-      named_bar(1, 32 * kConsumerWarps);
-      cur_p = c.p;
-      cur_j = c.j;
+      v.ngroups = gstride;
+      build_x_digits(P.x, P.nsb * 256, a.batch, 4 * NT, 256 * h.j * P.slice_sb, v, 8, threadIdx.x, kConsumers,
+                     q4 ? 1 : 0);
+      named_bar(1, kConsumers);
     }
-    float acc[NT][2];
+    if (h.flags & kFirst) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-    const int r0 = 16 * mt + g;
-    for (int t0 = 0; t0 < nsbs; t0 += tsbm) {
-      const int tsb = min(tsbm, nsbs - t0);
-      if (!mbar_wait(&full_bar[s], phase)) {
-        if (lane == 0) atomicExch(&g_error, 2);
-        return;
-      }
-      const uint8_t* st = stages + s * kStageBytes;
-      const int off = (int)(((size_t)rec * (sb0s + t0)) & 15);
-      for (int k = sp; k < tsb; k += 2) {
-        const uint8_t* rec0 = st + slot * r0 + off + rec * k;
-        const uint8_t* rec1 = st + slot * (r0 + 8) + off + rec * k;
-        const int sbs = t0 + k;  // super-block index within the slice
-        if (q4)
-          q4k_superblock<NT>(rec0, rec1, digits, a.digit_stride, ndrows, 256 * sbs, inv_scale, gsum, ngroups,
-                             2 * sbs, lane, acc);
-        else
-          q6k_superblock<NT>(rec0, rec1, (sb0s + sbs) & 1, digits, a.digit_stride, ndrows, 256 * sbs, inv_scale,
-                             gsum, ngroups, 2 * sbs, lane, acc);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-      if (++s == kStages) {
-        s = 0;
-        phase ^= 1u;
-      }
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
     }
-    if (sp == 1) {
+    const uint8_t* st = stages + s * kStageBytes;
+    const int rec = q4 ? 144 : 210, slot = q4 ? kQ4Slot : kQ6Slot;
+    // work items of the tile: (super-block k, half) = 2 tsb halves, item hh = 2 k + half
+    for (int hh = sq; hh < 2 * h.tsb; hh += 4) {
+      const int k = hh >> 1, half = hh & 1;
+      const uint8_t* rec0 = st + slot * r0 + h.off + rec * k;
+      const uint8_t* rec1 = rec0 + slot * 8;
+      const int sbs = h.sb0 + k;
+      const int gi = 2 * sbs + half;
+      if (q4)
+        q4k_half<NT>(rec0, rec1, half, dl_perm, dstep, 256 * sbs, inv_scale, gsum, gstride, gi, t, acc);
+      else
+        q6k_half<NT>(rec0, rec1, (h.j * P.slice_sb + sbs) & 1, half, dl_nat, dstep, 256 * sbs, inv_scale, gsum,
+                     gstride, gi, t, acc);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    if (++s == kStages) {
+      s = 0;
+      phase ^= 1u;
+    }
+    if (!(h.flags & kLast)) continue;
+
+    float* xf = xfer + (size_t)mt * 3 * NT * 64;
+    if (sq > 0) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        xfer[mt][nt][0][lane] = acc[nt][0];
-        xfer[mt][nt][1][lane] = acc[nt][1];
+        xf[((sq - 1) * NT + nt) * 64 + lane] = acc[nt][0];
+        xf[((sq - 1) * NT + nt) * 64 + 32 + lane] = acc[nt][1];
       }
     }
-    named_bar(2 + mt, 64);
-    if (sp == 0) {
+    named_bar(2 + mt, 128);
+    if (sq == 0) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        acc[nt][0] += xfer[mt][nt][0][lane];
-        acc[nt][1] += xfer[mt][nt][1][lane];
-      }
+      for (int q = 0; q < 3; ++q)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[nt][0] += xf[(q * NT + nt) * 64 + lane];
+          acc[nt][1] += xf[(q * NT + nt) * 64 + 32 + lane];
+        }
     }
-    named_bar(2 + mt, 64);
+    named_bar(2 + mt, 128);
     const size_t ystride = (size_t)64 * P.nblocks;
-    const int row_base = 64 * c.b + 16 * mt;
+    const int row_base = 64 * h.b + 16 * mt;
     if (P.slices == 1) {
-      if (sp == 0) {
+      if (sq == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int bb = 4 * nt + t;
@@ -404,32 +456,33 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
         }
       }
     } else {
-      if (sp == 0) {
+      if (sq == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int bb = 4 * nt + t;
           if (bb < a.batch) {
-            float* pp = P.partial + (((size_t)c.j * P.nblocks + c.b) * a.batch + bb) * 64 + 16 * mt + g;
+            float* pp = P.partial + (((size_t)h.j * P.nblocks + h.b) * a.batch + bb) * 64 + 16 * mt + g;
             pp[0] = acc[nt][0];
             pp[8] = acc[nt][1];
           }
         }
       }
       __threadfence();
-      named_bar(1, 32 * kConsumerWarps);
-      if (threadIdx.x == 0) s_ticket = (int)atomicAdd(&P.tickets[c.b], 1u);
-      named_bar(1, 32 * kConsumerWarps);
+      named_bar(1, kConsumers);
+      if (threadIdx.x == 0) s_ticket = (int)atomicAdd(&P.tickets[h.b], 1u);
+      named_bar(1, kConsumers);
       if (s_ticket == P.slices - 1) {
         __threadfence();
-        for (int e = threadIdx.x; e < a.batch * 64; e += 32 * kConsumerWarps) {
+        for (int e = threadIdx.x; e < a.batch * 64; e += kConsumers) {
           const int bb = e / 64, r = e % 64;
           float sum = 0.f;
           for (int jj = 0; jj < P.slices; ++jj)
-            sum += __ldcg(P.partial + (((size_t)jj * P.nblocks + c.b) * a.batch + bb) * 64 + r);
-          P.y[(size_t)bb * ystride + 64 * c.b + r] = sum;
+            sum += __ldcg(P.partial + (((size_t)jj * P.nblocks + h.b) * a.batch + bb) * 64 + r);
+          P.y[(size_t)bb * ystride + 64 * h.b + r] = sum;
         }
-        if (threadIdx.x == 0) P.tickets[c.b] = 0u;
+        if (threadIdx.x == 0) P.tickets[h.b] = 0u;
       }
+      named_bar(1, kConsumers);
     }
   }
 }
@@ -440,16 +493,17 @@ struct Plan {
   int slices, slice_sb;
 };
 
-// Dynamic shared memory: stages, activation digits, and per (padded batch,
-// 128-column group) the inverse scale plus up to 8 sub-group sums.
+// Dynamic shared memory: stages, activation digits, per (padded batch, 128-column group)
+// the inverse scale plus 8 sub-group sums, and the cross-warp transfer of row sums.
 static size_t smem_bytes(int batch, int slice_sb) {
   const int nt = (batch + 3) / 4;
-  return (size_t)kStages * kStageBytes + (size_t)2 * batch * (256 * slice_sb + 16) + (size_t)4 * nt * (2 * slice_sb) * 36;
+  return (size_t)kStages * kStageBytes + (size_t)2 * batch * (256 * slice_sb + 16) +
+         (size_t)4 * nt * (2 * slice_sb) * 36 + (size_t)3072 * nt;
 }
 
 static int max_sb_fit(int batch) {
   const int nt = (batch + 3) / 4;
-  const long avail = (long)kSmemLimit - (long)kStages * kStageBytes - 32L * batch;
+  const long avail = (long)kSmemLimit - (long)kStages * kStageBytes - 32L * batch - 3072L * nt;
   return (int)std::max(1L, avail / (512L * batch + 288L * nt));
 }
 

@@ -86,20 +86,6 @@ struct Args {
 
 __device__ int g_error;  // set when a bounded wait runs out (never expected)
 
-enum : int { kTileData = 0, kTileZero = 1, kTileEnd = 2 };
-enum : int { kFirst = 1, kLast = 2 };
-
-struct __align__(16) TileHdr {
-  int kind, flags;
-  int p, j, b;       // problem, slice, block
-  int k0, np;        // plane range read
-  int g0, tg;        // first group of the tile within the slice, groups in the tile
-  int slot;          // activation-digit slot of (p, j)
-  int slices;        // column slices of the problem
-  int ystride;       // 64 * nblocks = out
-  float* y;          // output of the problem
-};
-
 // One (problem, column slice) touched by a CTA: the units [u0, u1) of the CTA's range (relative
 // to its first unit) are its blocks b0, b0 + 1, ...; everything the producer and consumers need
 // is copied here once, so the hot loops never index the kernel-parameter problem table.
@@ -349,7 +335,6 @@ template <int MAXP, int NT>
 __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ TileHdr hdr[kStages];
   __shared__ Slot slots[kMaxSlots];
   __shared__ uint8_t lvc[kLevelCache];
   __shared__ __align__(16) uint8_t zeros[160];
@@ -414,105 +399,67 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   }
   __syncthreads();
 
+  // Level cache: plane ranges of the CTA's units, read once by the producer threads.
+  if (warp >= kConsumerWarps) {
+    const int nsl = s_nslots;
+    int si = 0;
+    for (int k = threadIdx.x - kConsumers; k < nunits && k < kLevelCache; k += 32 * kProducerWarps) {
+      while (si + 1 < nsl && k >= slots[si].u1) ++si;
+      const Slot& sl = slots[si];
+      lvc[k] = (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, sl.b0 + (k - sl.u0));
+    }
+  }
+  __syncthreads();
+
+  // Team t (producer warp t and consumer warps 4t..4t+3) walks units t, t + kTeams, ... of the
+  // range; both sides derive the same tile sequence from the slot table and the level cache,
+  // so the only hand-offs are the full / empty barriers of the team's two stages.
+  const int nsl = s_nslots;
   if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producer warps
-    const int nsl = s_nslots;
-    // 1. plane ranges of the CTA's units into the level cache (all producer threads)
-    {
-      int si = 0;
-      for (int k = threadIdx.x - kConsumers; k < nunits && k < kLevelCache; k += 32 * kProducerWarps) {
-        while (si + 1 < nsl && k >= slots[si].u1) ++si;
-        const Slot& sl = slots[si];
-        lvc[k] = (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, sl.b0 + (k - sl.u0));
-      }
-    }
-    named_bar(6, 32 * kProducerWarps);
     if (lane != 0) return;
-    // 2. producer warp t walks team t's units t, t + kTeams, ... of the range
     const int team = warp - kConsumerWarps;
-    int issued = 0;
-    auto claim = [&](int& s) -> bool {
-      s = kTeamStages * team + (issued % kTeamStages);
-      if (issued >= kTeamStages) {
-        const uint32_t ph = (uint32_t)((issued / kTeamStages - 1) & 1);
-        if (!mbar_wait(&empty_bar[s], ph)) {
-          atomicExch(&g_error, 1);
-          return false;
-        }
-      }
-      return true;
-    };
-    bool ok = true;
-    int si = 0;
-    for (int k = team; k < nunits && ok; k += kTeams) {
+    int issued = 0, si = 0;
+    for (int k = team; k < nunits; k += kTeams) {
       while (si + 1 < nsl && k >= slots[si].u1) ++si;
       const Slot& sl = slots[si];
       const int b = sl.b0 + (k - sl.u0);
       const int pr = (k < kLevelCache) ? (int)lvc[k] : plane_range(a.mode, sl.lv_from, sl.lv_to, b);
       const int k0 = pr >> 4, np = pr & 15;
-      int s;
-      if (np == 0) {
-        if (a.mode == 0 && sl.j == 0 && (ok = claim(s))) {
-          TileHdr& h = hdr[s];
-          h.kind = kTileZero;
-          h.flags = kFirst | kLast;
-          h.p = sl.p;
-          h.j = sl.j;
-          h.b = b;
-          h.slot = si;
-          h.ystride = 64 * sl.nblocks;
-          h.y = sl.y;
-          mbar_arrive(&full_bar[s]);
-          ++issued;
-        }
-        continue;
-      }
+      if (np == 0) continue;
       const int tgm = tile_groups(np);
       const int ngs = sl.ngroups;
-      const uint8_t* blk = sl.store + (size_t)b * 8448u * sl.G;
-      for (int g0 = 0; g0 < ngs && ok; g0 += tgm) {
+      const int G = sl.G;
+      const uint8_t* blk = sl.store + (size_t)b * 8448u * G;
+      for (int g0 = 0; g0 < ngs; g0 += tgm) {
         const int tg = min(tgm, ngs - g0);
-        if (!(ok = claim(s))) break;
-        TileHdr& h = hdr[s];
-        h.kind = kTileData;
-        h.flags = (g0 == 0 ? kFirst : 0) | (g0 + tg >= ngs ? kLast : 0);
-        h.p = sl.p;
-        h.j = sl.j;
-        h.b = b;
-        h.k0 = k0;
-        h.np = np;
-        h.g0 = g0;
-        h.tg = tg;
-        h.slot = si;
-        h.slices = sl.slices;
-        h.ystride = 64 * sl.nblocks;
-        h.y = sl.y;
+        const int s = kTeamStages * team + (issued % kTeamStages);
+        if (issued >= kTeamStages &&
+            !mbar_wait(&empty_bar[s], (uint32_t)((issued / kTeamStages - 1) & 1))) {
+          atomicExch(&g_error, 1);
+          return;
+        }
         uint8_t* st = smem + s * kStageBytes;
         const int gg = sl.gfirst + g0;
         const uint32_t bytes = 256u * tg + 2048u * tg * np;
         mbar_expect_tx(&full_bar[s], bytes);
-        if (tg == sl.G && k0 == 0) {
+        if (tg == G && k0 == 0) {
           bulk_g2s(st, blk, bytes, &full_bar[s]);  // the whole depth-d prefix of the block
         } else {
           bulk_g2s(st, blk + 256u * gg, 256u * tg, &full_bar[s]);
           for (int kk = 0; kk < np; ++kk)
-            bulk_g2s(st + 256 * tg + 2048 * tg * kk, blk + 256u * sl.G + 2048u * ((size_t)sl.G * (k0 + kk) + gg),
+            bulk_g2s(st + 256 * tg + 2048 * tg * kk, blk + 256u * G + 2048u * ((size_t)G * (k0 + kk) + gg),
                      2048u * tg, &full_bar[s]);
         }
         ++issued;
       }
-    }
-    int s;
-    if (ok && claim(s)) {
-      hdr[s].kind = kTileEnd;
-      mbar_arrive(&full_bar[s]);
     }
     return;
   }
 
   // ------------------------------------------------------------------ consumer warps
   // 1. activation digits of every (problem, slice) the range touches
-  for (int i = 0; i < s_nslots; ++i) {
+  for (int i = 0; i < nsl; ++i) {
     const Slot& sl = slots[i];
     build_slot(sl.x, sl.G * 128, a.batch, 4 * NT, 128 * sl.gfirst, sl, threadIdx.x, kConsumers);
   }
@@ -524,44 +471,32 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   const int g = lane >> 2, t = lane & 3;
   const int r0 = 16 * mt + g;
   const uint32_t smem_base = smem_u32(smem);
-  float acc[NT][2];
-  float cfac = 0.f;
-  int cur_slot = -1;
   uint32_t dlane[NT], dstep[NT], gc_lane = 0;
-  int gstride = 1;
-  for (int k = 0;; ++k) {
-    const int s = kTeamStages * team + (k % kTeamStages);
-    if (!mbar_wait(&full_bar[s], (uint32_t)((k / kTeamStages) & 1))) {
-      if (lane == 0) atomicExch(&g_error, 2);
-      return;
-    }
-    TileHdr h;
-    {
-      const uint4* hv = reinterpret_cast<const uint4*>(&hdr[s]);
-      uint4* dv = reinterpret_cast<uint4*>(&h);
+  int cur_slot = -1, si = 0, used = 0;
+  for (int k = team; k < nunits; k += kTeams) {
+    while (si + 1 < nsl && k >= slots[si].u1) ++si;
+    const Slot& sl = slots[si];
+    const int b = sl.b0 + (k - sl.u0);
+    const int pr = (k < kLevelCache) ? (int)lvc[k] : plane_range(a.mode, sl.lv_from, sl.lv_to, b);
+    const int k0 = pr >> 4, np = pr & 15;
+    const size_t ystride = (size_t)64 * sl.nblocks;
+    const int row_base = 64 * b + 16 * mt;
+    float* const y = sl.y;
+    if (np == 0) {  // ZERO block (depth mode): its rows are 0; a residual adds nothing
+      if (a.mode == 0 && sl.j == 0) {
 #pragma unroll
-      for (int q = 0; q < (int)(sizeof(TileHdr) / 16); ++q) dv[q] = hv[q];
-    }
-    if (h.kind == kTileEnd) break;
-    const size_t ystride = (size_t)h.ystride;
-    const int row_base = 64 * h.b + 16 * mt;
-    if (h.kind == kTileZero) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int bb = 4 * nt + t;
-        if (bb < a.batch) {
-          h.y[(size_t)bb * ystride + row_base + g] = 0.f;
-          h.y[(size_t)bb * ystride + row_base + g + 8] = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+          const int bb = 4 * nt + t;
+          if (bb < a.batch) {
+            y[(size_t)bb * ystride + row_base + g] = 0.f;
+            y[(size_t)bb * ystride + row_base + g + 8] = 0.f;
+          }
         }
       }
       continue;
     }
-    if (h.slot != cur_slot) {
-      cur_slot = h.slot;
-      const Slot& sl = slots[h.slot];
-      gstride = sl.ngroups;
+    if (si != cur_slot) {
+      cur_slot = si;
       gc_lane = sl.gconst + 8u * (uint32_t)(t * sl.ngroups);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -571,24 +506,33 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         dstep[nt] = liveb ? 128u : 0u;
       }
     }
-    if (h.flags & kFirst) {
+    const int gstride = sl.ngroups;
+    const float cfac = cfac_of(k0, np);
+    float acc[NT][2];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-      cfac = cfac_of(h.k0, h.np);
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
+    const int tgm = tile_groups(np);
+    for (int g0 = 0; g0 < sl.ngroups; g0 += tgm) {
+      const int tg = min(tgm, sl.ngroups - g0);
+      const int s = kTeamStages * team + (used % kTeamStages);
+      if (!mbar_wait(&full_bar[s], (uint32_t)((used / kTeamStages) & 1))) {
+        if (lane == 0) atomicExch(&g_error, 2);
+        return;
+      }
+      dispatch_tile<NT>(k0, np, smem_base + s * kStageBytes, tg, dlane, dstep, gc_lane, gstride, g0, cfac, r0, t,
+                        acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+      ++used;
     }
-    dispatch_tile<NT>(h.k0, h.np, smem_base + s * kStageBytes, h.tg, dlane, dstep, gc_lane, gstride, h.g0, cfac, r0,
-                      t, acc);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
-    if (!(h.flags & kLast)) continue;
 
     // ---- unit done: this warp's 16 rows are final (or a slice partial)
-    if (h.slices == 1) {
+    if (sl.slices == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int bb = 4 * nt + t;
         if (bb < a.batch) {
-          float* y0 = h.y + (size_t)bb * ystride + row_base + g;
+          float* y0 = y + (size_t)bb * ystride + row_base + g;
           if (a.mode == 0) {
             y0[0] = acc[nt][0];
             y0[8] = acc[nt][1];
@@ -600,34 +544,33 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       }
     } else {
       // partial for this slice; the last team to finish the block adds the slices in order
-      const Slot& P = slots[h.slot];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int bb = 4 * nt + t;
         if (bb < a.batch) {
-          float* pp = P.partial + (((size_t)h.j * P.nblocks + h.b) * a.batch + bb) * 64 + 16 * mt + g;
+          float* pp = sl.partial + (((size_t)sl.j * sl.nblocks + b) * a.batch + bb) * 64 + 16 * mt + g;
           pp[0] = acc[nt][0];
           pp[8] = acc[nt][1];
         }
       }
       __threadfence();
       named_bar(2 + team, kTeamThreads);
-      if (tt == 0) s_ticket[team] = (int)atomicAdd(&P.tickets[h.b], 1u);
+      if (tt == 0) s_ticket[team] = (int)atomicAdd(&sl.tickets[b], 1u);
       named_bar(2 + team, kTeamThreads);
-      if (s_ticket[team] == P.slices - 1) {
+      if (s_ticket[team] == sl.slices - 1) {
         __threadfence();
         for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
           const int bb = e / 64, r = e % 64;
           float sum = 0.f;
-          for (int jj = 0; jj < P.slices; ++jj)
-            sum += __ldcg(P.partial + (((size_t)jj * P.nblocks + h.b) * a.batch + bb) * 64 + r);
-          float* yy = h.y + (size_t)bb * ystride + 64 * h.b + r;
+          for (int jj = 0; jj < sl.slices; ++jj)
+            sum += __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + bb) * 64 + r);
+          float* yy = y + (size_t)bb * ystride + 64 * b + r;
           if (a.mode == 0)
             *yy = sum;
           else
             *yy += sum;
         }
-        if (tt == 0) P.tickets[h.b] = 0u;
+        if (tt == 0) sl.tickets[b] = 0u;
       }
       named_bar(2 + team, kTeamThreads);
     }

@@ -52,7 +52,7 @@ constexpr int kStages = kTeams * kTeamStages;
 constexpr int kStageBytes = 18432;
 constexpr int kMaxCtas = 1024;
 constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
-constexpr int kLevelCache = 4096;     // units per CTA whose plane ranges are cached in smem
+constexpr int kLevelCache = 4096;     // most units per CTA; all their plane ranges are cached in smem
 constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
 constexpr int kDigitBudget = kSmemLimit - kStages * kStageBytes;
 
@@ -81,6 +81,7 @@ struct Args {
   int mode;            // 0 depth (y =), 1 residual (y +=)
   int ncta;
   int cta_begin[kMaxCtas + 1];
+  int cta_slice[kMaxCtas];  // first (problem, slice) pair of the CTA, counted in order, << 7 | pairs touched
   Problem p[MAXP];
 };
 
@@ -95,6 +96,7 @@ struct __align__(16) Slot {
   int p, j, u0, u1, b0;
   int nblocks, G, ngroups, slices, gfirst;  // gfirst = first group of the slice in the row
   int stride;
+  int it0;           // first (batch row, group) digit item of the slot in the CTA's item count
   uint32_t digits;   // smem address
   uint32_t gconst;   // smem address
   const uint8_t* store;
@@ -105,35 +107,6 @@ struct __align__(16) Slot {
   float* partial;
   uint32_t* tickets;
 };
-
-struct UnitCursor {
-  int p, j, b, u;
-};
-
-template <int MAXP>
-__device__ __forceinline__ UnitCursor cursor_at(const Args<MAXP>& a, int u) {
-  int p = 0;
-  while (p + 1 < a.nproblems && a.p[p + 1].unit_begin <= u) ++p;
-  const int local = u - a.p[p].unit_begin;
-  UnitCursor c;
-  c.p = p;
-  c.j = local / a.p[p].nblocks;
-  c.b = local % a.p[p].nblocks;
-  c.u = u;
-  return c;
-}
-
-template <int MAXP>
-__device__ __forceinline__ void cursor_next(const Args<MAXP>& a, UnitCursor& c) {
-  ++c.u;
-  if (++c.b == a.p[c.p].nblocks) {
-    c.b = 0;
-    if (++c.j == a.p[c.p].slices) {
-      c.j = 0;
-      ++c.p;
-    }
-  }
-}
 
 __device__ __forceinline__ int slice_ng(const Problem& P, int j) {
   return min(P.slice_groups, P.G - j * P.slice_groups);
@@ -146,8 +119,15 @@ __host__ __device__ constexpr uint32_t plane_mask(int k, int i) {
              : ((0x03030303u << ((6 - 2 * k + 2 * i) & 7)) | (0x03030303u >> (32 - ((6 - 2 * k + 2 * i) & 7))));
 }
 
+// Named barriers: 0 is __syncthreads; team t uses kBarTeam0 + t.
+enum : int { kBarTeam0 = 2, kBarProducers = 6, kBarLevels = 7 };
+
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
@@ -182,46 +162,85 @@ __device__ __forceinline__ float cfac_of(int k0, int np) {
   return 0.5f * (float)(cb2 - ca2);
 }
 
-// Digits of columns [col0, col0 + 128 ngroups) of x into one slot (see fl_common.cuh for the
-// number format). Called by nthreads consumer threads, tid in [0, nthreads).
-__device__ __forceinline__ void build_slot(const uint16_t* __restrict__ x, int in, int batch, int batch_pad, int col0,
-                                           const Slot& sl, int tid, int nthreads) {
+// Digit items of every slot (one item = 128 columns of one batch row) by nthreads consumer
+// threads, tid in [0, nthreads): one warp per item, four items' loads in flight per warp.
+// See fl_common.cuh for the number format.
+__device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, int g, int lane) {
+  const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+  // group max |x| (the bit patterns of non-negative floats order like the values)
+  uint32_t mb = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mb = max(mb, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+  mb = __reduce_max_sync(0xffffffffu, mb);
+  int E = 0;  // m = mant * 2^E, mant in [0.5, 1)
+  if (mb >= 0x00800000u)
+    E = (int)(mb >> 23) - 126;
+  else if (mb != 0u)
+    frexpf(__uint_as_float(mb), &E);
+  const int sigma = (mb != 0u) ? (14 - E) : 0;
+  // v = rint(x 2^sigma): a power-of-two scale is exact, so one multiply when 2^sigma is normal
+  const bool direct = sigma >= -126 && sigma <= 127;
+  const float scale = __uint_as_float((uint32_t)(sigma + 127) << 23);
+  uint32_t hw = 0, lw = 0;
+  int part = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int vv = __float2int_rn(direct ? f[i] * scale : ldexpf(f[i], sigma));
+    const int h = (vv + 128) >> 8;
+    const int l = vv - 256 * h;
+    hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
+    lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
+    part += vv;
+  }
+  const uint32_t dh = sl.digits + (uint32_t)((2 * b) * sl.stride + 128 * g + 4 * lane);
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh), "r"(hw) : "memory");
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)sl.stride), "r"(lw) : "memory");
+  part = __reduce_add_sync(0xffffffffu, part);
+  if (lane == 0) {
+    const uint32_t gc = sl.gconst + 8u * (uint32_t)(b * sl.ngroups + g);
+    asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(ldexpf(1.0f, -sigma)), "f"(ldexpf((float)part, -sigma))
+                 : "memory");
+  }
+}
+
+__device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int batch, int batch_pad, int tid,
+                                             int nthreads) {
   const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
-  for (int item = wid; item < batch_pad * sl.ngroups; item += nw) {
-    const int b = item / sl.ngroups, g = item % sl.ngroups;
-    const uint32_t gc = sl.gconst + 8u * (uint32_t)item;
-    if (b >= batch) {
-      if (lane == 0) asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(0.f), "f"(0.f) : "memory");
-      continue;
+  const Slot& last = slots[nsl - 1];
+  const int total = last.it0 + batch * last.ngroups;
+  int si = 0;
+  for (int it0 = wid; it0 < total; it0 += 4 * nw) {
+    uint2 raw[4];
+    int sq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int it = it0 + q * nw;
+      sq[q] = -1;
+      if (it < total) {
+        while (si + 1 < nsl && it >= slots[si + 1].it0) ++si;
+        const Slot& sl = slots[si];
+        const int local = it - sl.it0, b = local / sl.ngroups, g = local % sl.ngroups;
+        raw[q] = __ldg(reinterpret_cast<const uint2*>(sl.x + (size_t)b * sl.G * 128 + 128 * (sl.gfirst + g) +
+                                                      4 * lane));
+        sq[q] = si;
+      }
     }
-    const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)b * in + col0 + 128 * g + 4 * lane);
-    const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-    float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    int E = 0;
-    if (m > 0.f) frexpf(m, &E);
-    const int sigma = (m > 0.f) ? (14 - E) : 0;
-    uint32_t hw = 0, lw = 0;
-    int part = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int vv = __float2int_rn(ldexpf(f[i], sigma));
-      const int h = (vv + 128) >> 8;
-      const int l = vv - 256 * h;
-      hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
-      lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
-      part += vv;
+    for (int q = 0; q < 4; ++q) {
+      if (sq[q] >= 0) {
+        const Slot& sl = slots[sq[q]];
+        const int local = it0 + q * nw - sl.it0;
+        convert_item(raw[q], sl, local / sl.ngroups, local % sl.ngroups, lane);
+      }
     }
-    const uint32_t dh = sl.digits + (uint32_t)((2 * b) * sl.stride + 128 * g + 4 * lane);
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh), "r"(hw) : "memory");
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)sl.stride), "r"(lw) : "memory");
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane == 0)
-      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(ldexpf(1.0f, -sigma)),
-                   "f"(ldexpf((float)part, -sigma))
+  }
+  // padded batch rows read zero constants
+  for (int i = 0; i < nsl; ++i) {
+    const Slot& sl = slots[i];
+    for (int e = tid; e < (batch_pad - batch) * sl.ngroups; e += nthreads)
+      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(sl.gconst + 8u * (uint32_t)(batch * sl.ngroups + e)),
+                   "f"(0.f), "f"(0.f)
                    : "memory");
   }
 }
@@ -229,17 +248,19 @@ __device__ __forceinline__ void build_slot(const uint16_t* __restrict__ x, int i
 // One tile for one warp: all tg groups of the tile for rows r0 = 16 mt + g and r0 + 8.
 // Per group: plane words, activation digits, code bytes by mask/or/rotate, 4 k32 MMAs per
 // N-tile in two independent chains, then the group's scale and constant part in fp32.
-template <int K0, int NP, int NT>
-__device__ __forceinline__ void tile_compute(uint32_t stage, int tg, const uint32_t (&dlane)[NT],
+template <int K0, int NP, int NT, bool FULL>
+__device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const uint32_t (&dlane)[NT],
                                              const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
                                              int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
   constexpr int TG = tile_groups(NP);
+  // A full tile has a compile-time group count, so the groups' loads and MMAs interleave freely.
+  const int tg = FULL ? TG : tg_arg;
   const uint32_t planes = stage + 256u * tg;
   const uint32_t wrow = planes + 32u * r0 + 8u * t;
   const uint32_t srow = stage + 4u * r0;
 #pragma unroll
   for (int gl = 0; gl < TG; ++gl) {
-    if (gl < tg) {
+    if (FULL || gl < tg) {
       const int gs = slice_goff + gl;
       uint2 W[NP][2];
 #pragma unroll
@@ -305,8 +326,11 @@ template <int NT>
 __device__ __forceinline__ void dispatch_tile(int k0, int np, uint32_t stage, int tg, const uint32_t (&dlane)[NT],
                                               const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
                                               int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
-#define FL_TILE(K0_, NP_) \
-  tile_compute<K0_, NP_, NT>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc)
+#define FL_TILE(K0_, NP_)                                                                            \
+  if (tg == tile_groups(NP_))                                                                        \
+    tile_compute<K0_, NP_, NT, true>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc); \
+  else                                                                                               \
+    tile_compute<K0_, NP_, NT, false>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc)
   switch (k0 * 8 + np) {
     case 0 * 8 + 1: FL_TILE(0, 1); break;
     case 0 * 8 + 2: FL_TILE(0, 2); break;
@@ -353,70 +377,93 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       mbar_init(&empty_bar[s], kTeamWarps);
     }
     fence_mbar_init();
-    // one slot per distinct (problem, slice) of the range, digits laid out back to back
-    uint32_t off = 0;
-    int n = 0;
+  }
+  if (warp == 0) {
+    // Slot table: lane i fills slot i, the i-th (problem, slice) pair from the CTA's first one
+    // (a multi-problem launch has one slice per problem); digit areas laid out back to back.
     const uint32_t base = smem_u32(smem + kStages * kStageBytes);
-    UnitCursor c = cursor_at(a, u_begin);
-    int u = u_begin;
-    while (u < u_end && n < kMaxSlots) {
-      const Problem& P = a.p[c.p];
-      const int slice_end = P.unit_begin + (c.j + 1) * P.nblocks;  // first unit after this slice
+    const int s0 = a.cta_slice[blockIdx.x] >> 7, nsl_cta = a.cta_slice[blockIdx.x] & 127;
+    uint32_t carry = 0;
+    int items = 0, n = 0;
+    for (int i0 = 0; i0 < nsl_cta; i0 += 32) {
+      const int i = i0 + lane;
+      const bool live = i < nsl_cta;
       Slot sl;
-      sl.p = c.p;
-      sl.j = c.j;
-      sl.u0 = u - u_begin;
-      sl.u1 = min(u_end, slice_end) - u_begin;
-      sl.b0 = c.b;
-      sl.nblocks = P.nblocks;
-      sl.G = P.G;
-      sl.ngroups = slice_ng(P, c.j);
-      sl.slices = P.slices;
-      sl.gfirst = c.j * P.slice_groups;
-      sl.stride = 128 * sl.ngroups + 16;
-      sl.digits = base + off;
-      off += 2 * a.batch * sl.stride;
-      sl.gconst = base + off;
-      off += 8 * 4 * NT * sl.ngroups;
-      sl.store = P.store;
-      sl.lv_from = P.lv_from;
-      sl.lv_to = P.lv_to;
-      sl.x = P.x;
-      sl.y = P.y;
-      sl.partial = P.partial;
-      sl.tickets = P.tickets;
-      slots[n++] = sl;
-      u = min(u_end, slice_end);
-      if (u < u_end) {
-        c.b = 0;
-        if (++c.j == P.slices) {
-          c.j = 0;
-          ++c.p;
+      uint32_t bytes = 0;
+      int nit = 0;
+      if (live) {
+        const int p = (a.nproblems == 1) ? 0 : s0 + i;
+        const int j = (a.nproblems == 1) ? s0 + i : 0;
+        const Problem& P = a.p[p];
+        const int slice_start = P.unit_begin + j * P.nblocks;
+        const int first = max(slice_start, u_begin);
+        sl.p = p;
+        sl.j = j;
+        sl.u0 = first - u_begin;
+        sl.u1 = min(u_end, slice_start + P.nblocks) - u_begin;
+        sl.b0 = first - slice_start;
+        sl.nblocks = P.nblocks;
+        sl.G = P.G;
+        sl.ngroups = slice_ng(P, j);
+        sl.slices = P.slices;
+        sl.gfirst = j * P.slice_groups;
+        sl.stride = 128 * sl.ngroups + 16;
+        sl.store = P.store;
+        sl.lv_from = P.lv_from;
+        sl.lv_to = P.lv_to;
+        sl.x = P.x;
+        sl.y = P.y;
+        sl.partial = P.partial;
+        sl.tickets = P.tickets;
+        bytes = (uint32_t)(2 * a.batch * sl.stride + 8 * 4 * NT * sl.ngroups);
+        nit = a.batch * sl.ngroups;
+      }
+      uint32_t incl = bytes;
+      int iincl = nit;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        const int w = __shfl_up_sync(0xffffffffu, iincl, o);
+        if (lane >= o) {
+          incl += v;
+          iincl += w;
         }
       }
+      if (live) {
+        sl.digits = base + carry + incl - bytes;
+        sl.gconst = sl.digits + (uint32_t)(2 * a.batch * sl.stride);
+        sl.it0 = items + iincl - nit;
+        slots[i] = sl;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+      items += __shfl_sync(0xffffffffu, iincl, 31);
+      n += __popc(__ballot_sync(0xffffffffu, live));
     }
-    s_nslots = n;
+    if (lane == 0) s_nslots = n;
   }
   __syncthreads();
 
-  // Level cache: plane ranges of the CTA's units, read once by the producer threads.
-  if (warp >= kConsumerWarps) {
-    const int nsl = s_nslots;
-    int si = 0;
-    for (int k = threadIdx.x - kConsumers; k < nunits && k < kLevelCache; k += 32 * kProducerWarps) {
-      while (si + 1 < nsl && k >= slots[si].u1) ++si;
-      const Slot& sl = slots[si];
-      lvc[k] = (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, sl.b0 + (k - sl.u0));
-    }
-  }
-  __syncthreads();
-
+  // Before any weight copy is in flight (they would queue ahead of these small reads): the
+  // producer threads read the level bytes into the level cache while the consumer threads read
+  // the activations. Producers then publish the cache with an arrive on kBarLevels and start
+  // copying; consumers wait on it only once their digits are built.
+  //
   // Team t (producer warp t and consumer warps 4t..4t+3) walks units t, t + kTeams, ... of the
   // range; both sides derive the same tile sequence from the slot table and the level cache,
   // so the only hand-offs are the full / empty barriers of the team's two stages.
   const int nsl = s_nslots;
   if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producer warps
+    {
+      int si = 0;
+      for (int k = threadIdx.x - kConsumers; k < nunits; k += 32 * kProducerWarps) {
+        while (si + 1 < nsl && k >= slots[si].u1) ++si;
+        const Slot& sl = slots[si];
+        lvc[k] = (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, sl.b0 + (k - sl.u0));
+      }
+    }
+    named_bar(kBarProducers, 32 * kProducerWarps);
+    bar_arrive(kBarLevels, kThreads);
     if (lane != 0) return;
     const int team = warp - kConsumerWarps;
     int issued = 0, si = 0;
@@ -424,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       while (si + 1 < nsl && k >= slots[si].u1) ++si;
       const Slot& sl = slots[si];
       const int b = sl.b0 + (k - sl.u0);
-      const int pr = (k < kLevelCache) ? (int)lvc[k] : plane_range(a.mode, sl.lv_from, sl.lv_to, b);
+      const int pr = (int)lvc[k];
       const int k0 = pr >> 4, np = pr & 15;
       if (np == 0) continue;
       const int tgm = tile_groups(np);
@@ -459,11 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
 
   // ------------------------------------------------------------------ consumer warps
   // 1. activation digits of every (problem, slice) the range touches
-  for (int i = 0; i < nsl; ++i) {
-    const Slot& sl = slots[i];
-    build_slot(sl.x, sl.G * 128, a.batch, 4 * NT, 128 * sl.gfirst, sl, threadIdx.x, kConsumers);
-  }
-  named_bar(1, kConsumers);
+  build_digits(slots, nsl, a.batch, 4 * NT, threadIdx.x, kConsumers);
+  named_bar(kBarLevels, kThreads);  // every consumer's digits, and the producers' level cache
 
   // 2. team loop
   const int team = warp / kTeamWarps, mt = warp % kTeamWarps;
@@ -477,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
     while (si + 1 < nsl && k >= slots[si].u1) ++si;
     const Slot& sl = slots[si];
     const int b = sl.b0 + (k - sl.u0);
-    const int pr = (k < kLevelCache) ? (int)lvc[k] : plane_range(a.mode, sl.lv_from, sl.lv_to, b);
+    const int pr = (int)lvc[k];
     const int k0 = pr >> 4, np = pr & 15;
     const size_t ystride = (size_t)64 * sl.nblocks;
     const int row_base = 64 * b + 16 * mt;
@@ -554,9 +598,9 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         }
       }
       __threadfence();
-      named_bar(2 + team, kTeamThreads);
+      named_bar(kBarTeam0 + team, kTeamThreads);
       if (tt == 0) s_ticket[team] = (int)atomicAdd(&sl.tickets[b], 1u);
-      named_bar(2 + team, kTeamThreads);
+      named_bar(kBarTeam0 + team, kTeamThreads);
       if (s_ticket[team] == sl.slices - 1) {
         __threadfence();
         for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
@@ -572,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         }
         if (tt == 0) sl.tickets[b] = 0u;
       }
-      named_bar(2 + team, kTeamThreads);
+      named_bar(kBarTeam0 + team, kTeamThreads);
     }
   }
 }
@@ -629,6 +673,7 @@ static bool partition(Args<MAXP>& a, int nsm) {
   const double per_cta = total / target;
   int n = 0;
   a.cta_begin[0] = 0;
+  a.cta_slice[0] = 0;
   double acc = 0;      // cumulative cost from the first unit
   size_t dig = 0;      // digit bytes of the current range
   int nslots = 0, count = 0;
@@ -648,7 +693,9 @@ static bool partition(Args<MAXP>& a, int nsm) {
         }
         if (cut) {
           if (n + 1 >= kMaxCtas) return false;
+          a.cta_slice[n] |= nslots;
           a.cta_begin[++n] = u;
+          a.cta_slice[n] = ((a.nproblems == 1) ? j : i) << 7;
           dig = 0;
           nslots = 0;
           count = 0;
@@ -662,6 +709,7 @@ static bool partition(Args<MAXP>& a, int nsm) {
       }
     }
   }
+  a.cta_slice[n] |= nslots;
   a.cta_begin[++n] = units;
   a.ncta = n;
   return true;

@@ -170,6 +170,28 @@ FL_API size_t fl_gemv_workspace_bytes(int out, int in, int batch);
 FL_API fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, const uint16_t* x, int batch, float* y,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Depth GEMV without a caller workspace. No counterpart in the pages: an
+ * operational variant of fl_gemv_depth for callers that cannot hand over a
+ * device buffer, e.g. a plugin host that passes only the operation's own
+ * tensors, or a runtime that reserves all device memory up front (an extra
+ * cudaMalloc would fail there, and it may synchronize the device inside the
+ * decode loop). The column-split scratch lives in a fixed array of
+ * FL_GEMV_STATIC_SCRATCH_BYTES inside the library's device image, so this
+ * call allocates nothing.
+ *   - Same arguments and arithmetic as fl_gemv_depth, minus the workspace.
+ *   - Shapes whose split needs more scratch than the array holds
+ *     (fl_gemv_workspace_bytes(out, in, batch) > FL_GEMV_STATIC_SCRATCH_BYTES)
+ *     return FL_ERR_WORKSPACE; use fl_gemv_depth for them.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; each call clears the part that must start at zero on
+ *     its stream before the launch. Calls that overlap on the GPU (two
+ *     streams, or two host threads) race on the array: serialize them. */
+#define FL_GEMV_STATIC_SCRATCH_BYTES (4u << 20)
+FL_API fl_status fl_gemv_depth_static(const fl_plane_weight* w, const uint8_t* levels, const uint16_t* x, int batch,
+                               float* y, void* stream);
+
 /* Escalation residual ([PoD]: redo a step at 8 bits, written as an addition
  * to the low pass):  y[t][r] += sum_c (w_b - w_a)[r][c] x[t][c]  with
  * a = 2 from_levels[blk], b = 2 to_levels[blk], w_0 = 0. Reads only planes

@@ -33,6 +33,7 @@
 //    finish a block (atomic ticket) adds the slices in order. No CTA ever
 //    waits on another; every mbarrier wait is bounded.
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "fl_common.cuh"
@@ -854,4 +855,64 @@ extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
   if (!gemv::partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: problems too large for one launch", what);
   return gemv::launch_nt(a, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- allocation-free variant
+// The column-split scratch of fl_gemv_depth_static: one fixed array in the device image
+// (tickets first, then the slice partials, as in a caller workspace). Its device address is
+// looked up once per device, with that device current, on the first call there.
+namespace fl {
+namespace gemv {
+
+static __device__ __align__(256) uint8_t g_static_scratch[FL_GEMV_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_static_mu;
+static void* g_static_ptr[kMaxDevices];
+
+static fl_status static_scratch(void** ptr, const char* what) {
+  int dev = -1;
+  FL_CHECK_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FL_ERR_CUDA, "%s: device %d out of range", what, dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_static_ptr[dev] = p;
+  }
+  *ptr = g_static_ptr[dev];
+  return FL_OK;
+}
+
+}  // namespace gemv
+}  // namespace fl
+
+extern "C" fl_status fl_gemv_depth_static(const fl_plane_weight* w, const uint8_t* levels, const uint16_t* x,
+                                          int batch, float* y, void* stream) {
+  const char* what = "fl_gemv_depth_static";
+  fl_status st = gemv::check_weight(w, what);
+  if (st != FL_OK) return st;
+  if (batch < 1 || batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..16)", what, batch);
+  const int nsm = device_sm_count();
+  if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
+  const int nblocks = w->out / 64;
+  const gemv::Plan pl = gemv::plan_single(nblocks, w->in / 128, batch, nsm);
+  const size_t need = gemv::workspace_for(pl, nblocks, batch);
+  if (need > (size_t)FL_GEMV_STATIC_SCRATCH_BYTES)
+    return fail(FL_ERR_WORKSPACE,
+                "%s: out=%d in=%d batch=%d needs %zu bytes of scratch, the built-in array holds %zu "
+                "(use fl_gemv_depth with a caller workspace)",
+                what, w->out, w->in, batch, need, (size_t)FL_GEMV_STATIC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (need > 0) {
+    st = gemv::static_scratch(&scratch, what);
+    if (st != FL_OK) return st;
+    // the split's tickets start at zero; the partials are written before they are read
+    const size_t tickets = ((size_t)nblocks * 4 + 255) / 256 * 256;
+    FL_CHECK_CUDA(cudaMemsetAsync(scratch, 0, tickets, static_cast<cudaStream_t>(stream)),
+                  "cudaMemsetAsync(static scratch tickets)");
+  }
+  return gemv::single(w, levels, nullptr, x, batch, y, scratch, need > 0 ? (size_t)FL_GEMV_STATIC_SCRATCH_BYTES : 0,
+                      stream, 0, what);
 }

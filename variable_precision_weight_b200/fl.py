@@ -25,6 +25,7 @@ FL_MAX_STOPS = 16
 FL_MAX_PROBLEMS = 256
 FL_GGML_Q4_K = 12
 FL_GGML_Q6_K = 14
+FL_GEMV_STATIC_SCRATCH_BYTES = 4 << 20
 STATUS = {0: "FL_OK", -1: "FL_ERR_ARG", -2: "FL_ERR_SHAPE", -3: "FL_ERR_UNSUPPORTED", -4: "FL_ERR_ALIGN",
           -5: "FL_ERR_CUDA", -6: "FL_ERR_WORKSPACE"}
 
@@ -64,6 +65,7 @@ _sigs = {
     "fl_level_map": (_I, [_P, _I, _P, _P, _I, C.POINTER(fl_lens_params), _P, _P, _P]),
     "fl_gemv_workspace_bytes": (_S, [_I, _I, _I]),
     "fl_gemv_depth": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P, _S, _P]),
+    "fl_gemv_depth_static": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P]),
     "fl_gemv_residual": (_I, [C.POINTER(fl_plane_weight), _P, _P, _P, _I, _P, _P, _S, _P]),
     "fl_gemv_batched": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, _P]),
     "fl_logit_gate": (_I, [_P, _I, _I, _F, _F, _P, _P, _P, _P, _P]),
@@ -150,6 +152,10 @@ def fl_gemv_depth(w: fl_plane_weight, levels, x, batch: int, y, workspace=None, 
                   stream=None) -> None:
     _check(_lib.fl_gemv_depth(C.byref(w), _ptr(levels), _ptr(x), batch, _ptr(y), _ptr(workspace), workspace_bytes,
                               _stream(stream)))
+
+
+def fl_gemv_depth_static(w: fl_plane_weight, levels, x, batch: int, y, stream=None) -> None:
+    _check(_lib.fl_gemv_depth_static(C.byref(w), _ptr(levels), _ptr(x), batch, _ptr(y), _stream(stream)))
 
 
 def fl_gemv_residual(w: fl_plane_weight, from_levels, to_levels, x, batch: int, y, workspace=None,

@@ -558,7 +558,9 @@ def run_fl(args, rank, world, local_rank):
                      "traffic": tr["bytes_per_launch"] if tr else None,
                      "kernel": "plane_gemv_kernel (fl_gemv_batched, 197 problems, D4)",
                      "us_per_launch": tk * 1e6, "bytes_per_launch": step.bytes_d4,
-                     "share_of_step": tk / (t / args.steps) if t > 0 else None},
+                     # plane GEMV launches per step (the D4 pass plus the escalated steps' residual
+                     # pass, both full reads of the store) x time per launch / step time
+                     "share_of_step": (1 + n_esc / args.steps) * tk / (t / args.steps) if t > 0 else None},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": step.h2d_bytes,
                 "d2h_bytes_per_step": 32, "steps": e2e_steps,

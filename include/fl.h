@@ -235,15 +235,17 @@ FL_API fl_status fl_logit_gate(const float* logits, int vocab, int batch, float 
 /* ========================================================================= */
 /* K-quant GEMV ([Ember]: Q4_K / Q6_K native kernels, dequantize only at     */
 /* block granularity inside the product, per-tensor dispatch, unsupported    */
-/* types fail). Records of 256 weights, row-major [out][in / 256]; the value */
-/* rules are GGUF's, the byte layout is this library's own with the GGUF     */
-/* byte counts:                                                              */
+/* types fail). Records of 256 weights stored block-tiled: 64-row blocks,   */
+/* then super-blocks, then the block's 64 rows, i.e. record number           */
+/* ((r / 64) * (in / 256) + sb) * 64 + r % 64 holds row r, super-block sb,   */
+/* so 64 rows x k super-blocks is one contiguous range. The value rules are  */
+/* GGUF's; the byte layout is this library's own with the GGUF byte counts:  */
 /*   Q4_K 144 B, sub-blocks j of 32: [0,2) d fp16, [2,4) dmin fp16,          */
 /*        byte 4 + j = sc_j | (mn_j & 3) << 6, nibble j of the word at 12 =   */
 /*        mn_j >> 2, byte 16 + 16 j + b = q[32 j + b] | q[32 j + 16 + b] << 4;*/
 /*        w = d sc_j q - dmin mn_j.                                          */
-/*   Q6_K 210 B, sub-blocks j of 16, q in 0..63: a record at an even place n */
-/*        in its row is [q area 192][sc_j int8 x16][d fp16], at an odd place */
+/*   Q6_K 210 B, sub-blocks j of 16, q in 0..63: a record of an even row is */
+/*        [q area 192][sc_j int8 x16][d fp16], of an odd row                 */
 /*        [d fp16][q area 192][sc_j int8 x16]; q area: chunk t (48 B) x      */
 /*        group m (12 B = words A, B, C), W(j, L) = 16 j + 4 t + L:          */
 /*        A byte L = lo4 q[W(4m,L)] | lo4 q[W(4m+1,L)] << 4,                 */
@@ -251,8 +253,7 @@ FL_API fl_status fl_logit_gate(const float* logits, int vocab, int batch, float 
 /*        C byte L = hi2 q[W(4m+2,L)] | hi2 q[W(4m+3,L)] << 2                */
 /*                 | hi2 q[W(4m,L)] << 4 | hi2 q[W(4m+1,L)] << 6;            */
 /*        w = d sc_j (q - 32).                                               */
-/* blocks: device, 16-byte aligned; in % 256 == 0, and in % 2048 == 0 for    */
-/* Q6_K (rows then start 16-byte aligned and hold an even record count).     */
+/* blocks: device, 16-byte aligned; out % 64 == 0, in % 256 == 0.           */
 /* ggml_type other than FL_GGML_Q4_K / FL_GGML_Q6_K -> FL_ERR_UNSUPPORTED.    */
 /* Same x / y / workspace rules as fl_gemv_depth.                            */
 /* ========================================================================= */

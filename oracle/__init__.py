@@ -190,8 +190,8 @@ def logit_gate(logits, tau_h: float, tau_m: float):
     return H, M, top2, esc
 
 
-def dequant_superblock(rec: np.ndarray, ggml_type: int, index_in_row: int = 0) -> np.ndarray:
-    """Dequantize one record; a Q6_K record's layout depends on its index in its row."""
+def dequant_superblock(rec: np.ndarray, ggml_type: int, row: int = 0) -> np.ndarray:
+    """Dequantize one record; a Q6_K record's layout depends on the parity of its row."""
     rec = np.ascontiguousarray(rec, np.uint8)
     w = np.empty(256, np.float64)
     if ggml_type == Q4_K:
@@ -199,7 +199,7 @@ def dequant_superblock(rec: np.ndarray, ggml_type: int, index_in_row: int = 0) -
         _load().orc_dequant_q4k(_p(rec), _p(w))
     elif ggml_type == Q6_K:
         assert rec.size == 210
-        _load().orc_dequant_q6k(_p(rec), int(index_in_row) & 1, _p(w))
+        _load().orc_dequant_q6k(_p(rec), int(row) & 1, _p(w))
     else:
         raise ValueError("unsupported type")
     return w

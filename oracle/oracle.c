@@ -387,9 +387,9 @@ ORC_API void orc_logit_gate(const float* logits, int vocab, int batch, double ta
 /*            32 j + b, high nibble = q of weight 32 j + 16 + b              */
 /*   w = d * sc_j * q - dmin * mn_j                                          */
 /* Q6_K, 210 bytes, 16 sub-blocks j of 16 weights, 6-bit q (0..63).          */
-/*   A record's place n in its row decides where the 192-byte q area sits:    */
-/*   n even: [0,192) q, [192,208) sc_j int8, [208,210) d fp16                */
-/*   n odd:  [0,2) d fp16, [2,194) q, [194,210) sc_j int8                    */
+/*   The parity of the record's row decides where the 192-byte q area sits:   */
+/*   even row: [0,192) q, [192,208) sc_j int8, [208,210) d fp16              */
+/*   odd row:  [0,2) d fp16, [2,194) q, [194,210) sc_j int8                  */
 /*   q area: chunk t (0..3) = bytes [48 t, 48 t + 48), group m (0..3) =       */
 /*   12 bytes at 48 t + 12 m = words A, B, C; with W(j, L) = 16 j + 4 t + L:  */
 /*     A byte L = lo4 q[W(4m, L)]   | lo4 q[W(4m+1, L)] << 4                  */
@@ -442,6 +442,10 @@ ORC_API void orc_dequant_q6k(const uint8_t* blk, int odd, double* w) {
 #define ORC_Q4_K 12
 #define ORC_Q6_K 14
 
+/* Storage order of a tensor's records (ours; the pages fix only a record's   */
+/* content): 64-row blocks, then super-blocks, then the block's 64 rows, so   */
+/* the record of (row r, super-block sb) is number                            */
+/*   ((r / 64) * nsb + sb) * 64 + r % 64.                                     */
 /* y[t][r] = sum_c w[r][c] x[t][c], each super-block dequantized then dotted.*/
 ORC_API int orc_gemv_kquant(const uint8_t* blocks, int type, int out, int in, const uint16_t* x, int batch,
                             double* y, double* mass, int nthreads) {
@@ -460,11 +464,11 @@ ORC_API int orc_gemv_kquant(const uint8_t* blocks, int type, int out, int in, co
     double acc[16], am[16];
     for (int t = 0; t < batch; ++t) acc[t] = am[t] = 0.0;
     for (int sb = 0; sb < nsb; ++sb) {
-      const uint8_t* blk = blocks + ((size_t)r * nsb + sb) * rec;
+      const uint8_t* blk = blocks + (((size_t)(r / 64) * nsb + sb) * 64 + r % 64) * rec;
       if (type == ORC_Q4_K)
         orc_dequant_q4k(blk, w);
       else
-        orc_dequant_q6k(blk, sb & 1, w);
+        orc_dequant_q6k(blk, r & 1, w);
       for (int t = 0; t < batch; ++t)
         for (int i = 0; i < 256; ++i) {
           double xv = bf16_to_double(x[(size_t)t * in + 256 * sb + i]);

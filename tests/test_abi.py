@@ -72,7 +72,8 @@ def test_host_side_rejections(fl):
     assert _status(fl, fl.fl_gemv_residual, w, 16, None, 16, 1, 16, None, 0, s0) == ERR_ARG
     assert _status(fl, fl.fl_gemv_kquant, 16, 13, 64, 256, 16, 1, 16, None, 0, s0) == ERR_UNSUP   # Q5_K
     assert _status(fl, fl.fl_gemv_kquant, 16, 10, 64, 256, 16, 1, 16, None, 0, s0) == ERR_UNSUP   # Q2_K
-    assert _status(fl, fl.fl_gemv_kquant, 16, 14, 64, 256, 16, 1, 16, None, 0, s0) == ERR_SHAPE   # Q6_K in % 2048
+    assert _status(fl, fl.fl_gemv_kquant, 16, 14, 32, 256, 16, 1, 16, None, 0, s0) == ERR_SHAPE   # out % 64
+    assert _status(fl, fl.fl_gemv_kquant, 16, 12, 64, 384, 16, 1, 16, None, 0, s0) == ERR_SHAPE   # in % 256
     assert _status(fl, fl.fl_logit_gate, 16, 151937, 1, 0.0, 0.0, 16, 16, 16, 16, s0) == ERR_SHAPE
     assert _status(fl, fl.fl_logit_gate, 16, 1024, 0, 0.0, 0.0, 16, 16, 16, 16, s0) == ERR_SHAPE
     p = fl.lens_params(0.3, 0.75, 1, 4, [0.5], 0)                  # kappa - gamma = 2 stops needed

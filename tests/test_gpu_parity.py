@@ -303,6 +303,7 @@ def test_logit_gate_closed_forms(env):
 @pytest.mark.parametrize("ggml_type,out,inn,batch", [
     (12, 512, 2048, 1), (12, 192, 8192, 3), (12, 64, 256, 1), (12, 128, 1280, 5), (12, 256, 2048, 16),
     (14, 512, 2048, 1), (14, 192, 8192, 4), (14, 128, 4096, 8), (14, 64, 2048, 16),
+    (14, 128, 1280, 3), (14, 64, 768, 1),
 ])
 def test_kquant_vs_oracle(env, orc, ggml_type, out, inn, batch):
     torch, fl = env

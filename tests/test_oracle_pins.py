@@ -376,11 +376,22 @@ def test_kquant_saturation_and_zero_scale(orc):
     assert np.all(orc.dequant_superblock(odd, orc.Q6_K, 1) == 2.0 * 127 * 31)
 
 
+def _records_by_row(blocks, out, inn, nbytes):
+    """Block-tiled records [out / 64][nsb][64][bytes] -> [out][nsb][bytes]."""
+    nsb = inn // 256
+    return blocks.reshape(out // 64, nsb, 64, nbytes).transpose(0, 2, 1, 3).reshape(out, nsb, nbytes)
+
+
+def _dequant_tensor(orc, blocks, t, out, inn):
+    rec = _records_by_row(blocks, out, inn, orc.RECORD_BYTES[t])
+    return np.stack([np.concatenate([orc.dequant_superblock(rec[r, k], t, r) for k in range(inn // 256)])
+                     for r in range(out)])
+
+
 def test_kquant_roundtrip_against_source_weights(orc):
-    w = synth.gaussian_weights(8, 2048, 7, 17)
+    w = synth.gaussian_weights(64, 2048, 7, 17)
     for t in (orc.Q4_K, orc.Q6_K):
-        rec = synth.encode_kquant(w, t).reshape(-1, orc.RECORD_BYTES[t])
-        wr = np.concatenate([orc.dequant_superblock(r, t, i % 8) for i, r in enumerate(rec)]).reshape(w.shape)
+        wr = _dequant_tensor(orc, synth.encode_kquant(w, t), t, 64, 2048)
         rel = np.sqrt(((wr - w) ** 2).mean() / (w ** 2).mean())
         assert rel < (0.12 if t == orc.Q4_K else 0.04)
         sub = 32 if t == orc.Q4_K else 16
@@ -389,15 +400,13 @@ def test_kquant_roundtrip_against_source_weights(orc):
 
 
 def test_kquant_gemv_is_dequant_then_matmul(orc):
-    out, inn = 96, 2048
+    out, inn = 128, 1280
     w = synth.gaussian_weights(out, inn, 7, 18)
     x = synth.bf16_normal((3, inn), 7, 19)
     xf = synth.bf16_bits_to_f32(x).astype(np.float64)
     for t in (orc.Q4_K, orc.Q6_K):
         blocks = synth.encode_kquant(w, t)
-        rec = blocks.reshape(-1, orc.RECORD_BYTES[t])
-        W = np.concatenate([orc.dequant_superblock(r, t, i % (inn // 256))
-                            for i, r in enumerate(rec)]).reshape(out, inn)
+        W = _dequant_tensor(orc, blocks, t, out, inn)
         y = orc.gemv_kquant(blocks, t, out, inn, x)
         assert np.allclose(y, xf @ W.T, rtol=1e-12, atol=1e-12)
     with pytest.raises(ValueError):

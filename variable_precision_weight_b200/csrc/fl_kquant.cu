@@ -6,15 +6,16 @@
 //   Q4_K:  y[t][r] = sum_sb sum_j ( d sc_j sum_{c in j} q_c x_c  -  dmin mn_j sum_{c in j} x_c )
 //   Q6_K:  y[t][r] = sum_sb sum_j   d sc_j sum_{c in j} (q_c - 32) x_c
 //
-// Same B200 structure as the plane-store GEMV: one persistent CTA per SM, a
-// producer warp whose 32 lanes issue per-row 1-D bulk copies of a tile (64
-// rows x a few super-blocks) into a 4-stage shared-memory ring, and eight
-// consumer warps (4 m-tiles x 2 super-block parities). Codes become u8
-// tensor-core operands with one or two mask/shift operations per four
-// weights (the record layouts are built for it); each sub-block is one
-// mma.sync (m16n8k32 for Q4_K's 32-weight sub-blocks, m16n8k16 for Q6_K's
-// 16-weight ones) against the activations' int8 digits; the sub-block scale
-// is applied to the int32 result with an integer multiply-add, and each
+// Same B200 structure as the plane-store GEMV. A unit is one 64-row block times a column
+// slice; one persistent CTA per SM takes a contiguous range of units. Four teams, each a
+// producer warp (one lane issues copies) and four consumer warps (one per 16-row m-tile),
+// walk units t, t + 4, ... of the range through the team's two shared-memory stages. The
+// records are stored block-tiled, so a tile (64 rows x 2 Q4_K super-blocks = 18432 B, or
+// 64 rows x 1 Q6_K super-block = 13440 B) is one contiguous 1-D bulk copy. Codes become u8
+// tensor-core operands with one or two mask/shift operations per four weights (the record
+// layouts are built for it); each sub-block is one mma.sync (m16n8k32 for Q4_K's 32-weight
+// sub-blocks, m16n8k16 for Q6_K's 16-weight ones) against the activations' int8 digits; the
+// sub-block scale is applied to the int32 result with an integer multiply-add, and each
 // 128-column half of a super-block is converted to fp32 once.
 #include <algorithm>
 
@@ -23,88 +24,74 @@
 namespace fl {
 namespace kq {
 
-constexpr int kConsumerWarps = 16;
+constexpr int kTeams = 4;
+constexpr int kTeamWarps = 4;
+constexpr int kTeamThreads = 32 * kTeamWarps;
+constexpr int kConsumerWarps = kTeams * kTeamWarps;
 constexpr int kConsumers = 32 * kConsumerWarps;
-constexpr int kThreads = kConsumers + 32;
-constexpr int kStages = 4;
-constexpr int kStageBytes = 37888;
-constexpr int kMaxCtas = 512;
-constexpr int kSmemLimit = 232448 - 6144;  // opt-in shared memory per block on B200, less static use
-constexpr int kQ4Tsb = 4;          // super-blocks per Q4_K tile
-constexpr int kQ4Slot = 592;       // bytes per row in a Q4_K tile (4 records + 16 B pad against bank conflicts)
-constexpr int kQ6Tsb = 2;          // super-blocks per Q6_K tile
-constexpr int kQ6Slot = 432;       // bytes per row in a Q6_K tile (2 records, 16-byte rounded copy)
+constexpr int kProducerWarps = kTeams;  // producer warp t feeds team t
+constexpr int kThreads = kConsumers + 32 * kProducerWarps;
+constexpr int kTeamStages = 2;
+constexpr int kStages = kTeams * kTeamStages;
+constexpr int kStageBytes = 18432;  // 64 rows x 2 Q4_K records
+constexpr int kMaxCtas = 1024;
+constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
+constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
+constexpr int kDigitBudget = kSmemLimit - kStages * kStageBytes;
+
+__host__ __device__ constexpr int rec_bytes(int type) { return type == FL_GGML_Q4_K ? 144 : 210; }
+__host__ __device__ constexpr int tile_sb(int type) { return type == FL_GGML_Q4_K ? 2 : 1; }
 
 struct Problem {
   const uint8_t* blocks;
   const uint16_t* x;
   float* y;
-  float* partial;
-  uint32_t* tickets;
-  int type;          // FL_GGML_Q4_K or FL_GGML_Q6_K
-  int nblocks;       // out / 64
-  int nsb;           // in / 256
+  float* partial;      // [slices][nblocks][batch][64] when slices > 1
+  uint32_t* tickets;   // [nblocks] when slices > 1
+  int type;            // FL_GGML_Q4_K or FL_GGML_Q6_K
+  int nblocks;         // out / 64
+  int nsb;             // in / 256
   int slices;
-  int slice_sb;      // super-blocks per slice
-  int unit_begin;
+  int slice_sb;        // super-blocks per slice (last slice shorter)
+  int unit_begin;      // first global unit index of this problem
 };
 
 template <int MAXP>
 struct Args {
   int nproblems;
   int batch;
-  int digit_stride;
-  int max_slice_sb;
   int ncta;
   int cta_begin[kMaxCtas + 1];
+  int cta_slice[kMaxCtas];  // first (problem, slice) pair of the CTA, counted in order, << 7 | pairs touched
   Problem p[MAXP];
 };
 
-__device__ int g_error;
+__device__ int g_error;  // set when a bounded wait runs out (never expected)
 
-enum : int { kTileData = 0, kTileEnd = 2 };
-enum : int { kFirst = 1, kLast = 2, kNewX = 4 };
-struct TileHdr {
-  int kind, flags;
-  int p, j, b;
-  int sb0;   // first super-block of the tile within the slice
-  int tsb;   // super-blocks in the tile
-  int off;   // byte offset of the first record inside each row slot
+// One (problem, column slice) touched by a CTA; see the plane-store GEMV for the scheme.
+// Activation digits: rows 2b / 2b+1 hold the hi / lo digits of batch row b (stride bytes per
+// row, Q4_K slots in the permuted order its MMA fragments read); per (padded batch row,
+// 128-column group): iscale = 2^-sigma and gsum = 8 sums of 16 columns.
+struct __align__(16) Slot {
+  int p, j, u0, u1, b0;
+  int nblocks, nsb, nsbs, slices, sbfirst;  // nsbs = super-blocks of the slice
+  int type, stride, it0, ngroups;           // ngroups = 2 nsbs
+  uint32_t digits, iscale, gsum;            // smem addresses
+  const uint8_t* blocks;
+  const uint16_t* x;
+  float* y;
+  float* partial;
+  uint32_t* tickets;
 };
 
-struct Cursor {
-  int p, j, b, u;
-};
-
-template <int MAXP>
-__device__ __forceinline__ Cursor cursor_at(const Args<MAXP>& a, int u) {
-  int p = 0;
-  while (p + 1 < a.nproblems && a.p[p + 1].unit_begin <= u) ++p;
-  const int local = u - a.p[p].unit_begin;
-  Cursor c;
-  c.p = p;
-  c.j = local / a.p[p].nblocks;
-  c.b = local % a.p[p].nblocks;
-  c.u = u;
-  return c;
-}
-
-template <int MAXP>
-__device__ __forceinline__ void cursor_next(const Args<MAXP>& a, Cursor& c) {
-  ++c.u;
-  if (++c.b == a.p[c.p].nblocks) {
-    c.b = 0;
-    if (++c.j == a.p[c.p].slices) {
-      c.j = 0;
-      ++c.p;
-    }
-  }
-}
-
-__device__ __forceinline__ int slice_nsb(const Problem& P, int j) { return min(P.slice_sb, P.nsb - j * P.slice_sb); }
+enum : int { kBarTeam0 = 2, kBarX = 6, kBarDigits = 7 };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ float half_bits_to_float(uint32_t h) {
@@ -123,22 +110,145 @@ __device__ __forceinline__ int byte_s(uint32_t w, int j) {
   return (int)r;
 }
 
-__device__ __forceinline__ uint32_t lds_u32(const uint8_t* p) {
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
   uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 
-__device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
   return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ int4 lds_s4(uint32_t a) {
+  int4 v;
+  asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+__device__ __forceinline__ int slice_nsb(const Problem& P, int j) { return min(P.slice_sb, P.nsb - j * P.slice_sb); }
+
+// ---------------------------------------------------------------- activation digits
+// One item = 128 columns of one batch row (see fl_common.cuh for the number format),
+// converted by one warp; the Q4_K slots store each word at the place its m16n8k32 B
+// fragment reads it.
+__device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, int g, int lane) {
+  const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+  uint32_t mb = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mb = max(mb, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+  mb = __reduce_max_sync(0xffffffffu, mb);
+  int E = 0;  // max |x| = mant * 2^E, mant in [0.5, 1)
+  if (mb >= 0x00800000u)
+    E = (int)(mb >> 23) - 126;
+  else if (mb != 0u)
+    frexpf(__uint_as_float(mb), &E);
+  const int sigma = (mb != 0u) ? (14 - E) : 0;
+  const bool direct = sigma >= -126 && sigma <= 127;
+  const float scale = __uint_as_float((uint32_t)(sigma + 127) << 23);
+  uint32_t hw = 0, lw = 0;
+  int part = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int vv = __float2int_rn(direct ? f[i] * scale : ldexpf(f[i], sigma));
+    const int h = (vv + 128) >> 8;
+    const int l = vv - 256 * h;
+    hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
+    lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
+    part += vv;
+  }
+  const int wpos = (sl.type == FL_GGML_Q4_K) ? (8 * (lane >> 3) + 2 * (lane & 3) + ((lane >> 2) & 1)) : lane;
+  const uint32_t dh = sl.digits + (uint32_t)((2 * b) * sl.stride + 128 * g + 4 * wpos);
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh), "r"(hw) : "memory");
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)sl.stride), "r"(lw) : "memory");
+  // sums of 16 columns (4 lanes each)
+  part += __shfl_xor_sync(0xffffffffu, part, 1);
+  part += __shfl_xor_sync(0xffffffffu, part, 2);
+  const int item = b * sl.ngroups + g;
+  if ((lane & 3) == 0)
+    asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + 4u * (uint32_t)(8 * item + (lane >> 2))), "r"(part)
+                 : "memory");
+  if (lane == 0)
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)item), "f"(ldexpf(1.0f, -sigma))
+                 : "memory");
+}
+
+// All consumer threads; every thread arrives once on kBarX after its first loads are issued,
+// which lets the producers start the weight copies behind them.
+__device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int batch, int batch_pad, int tid,
+                                             int nthreads) {
+  const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
+  const Slot& last = slots[nsl - 1];
+  const int total = last.it0 + batch * last.ngroups;
+  int si = 0;
+  for (int round = 0, it0 = wid; round == 0 || it0 < total; ++round, it0 += 4 * nw) {
+    uint2 raw[4];
+    int sq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int it = it0 + q * nw;
+      sq[q] = -1;
+      if (it < total) {
+        while (si + 1 < nsl && it >= slots[si + 1].it0) ++si;
+        const Slot& sl = slots[si];
+        const int local = it - sl.it0, b = local / sl.ngroups, g = local % sl.ngroups;
+        raw[q] = __ldg(reinterpret_cast<const uint2*>(sl.x + (size_t)b * sl.nsb * 256 + 256 * sl.sbfirst + 128 * g +
+                                                      4 * lane));
+        sq[q] = si;
+      }
+    }
+    if (round == 0) bar_arrive(kBarX, kThreads);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (sq[q] >= 0) {
+        const Slot& sl = slots[sq[q]];
+        const int local = it0 + q * nw - sl.it0;
+        convert_item(raw[q], sl, local / sl.ngroups, local % sl.ngroups, lane);
+      }
+    }
+  }
+  // padded batch rows read zero scales and sums
+  for (int i = 0; i < nsl; ++i) {
+    const Slot& sl = slots[i];
+    const int n = (batch_pad - batch) * sl.ngroups;
+    for (int e = tid; e < 9 * n; e += nthreads) {
+      const int item = batch * sl.ngroups + e % n;
+      if (e < n)
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)item), "f"(0.f) : "memory");
+      else
+        asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + 4u * (uint32_t)(8 * item + (e / n - 1))), "r"(0)
+                     : "memory");
+    }
+  }
 }
 
 // ---------------------------------------------------------------- Q4_K: half (4 sub-blocks) of one super-block
+// rec0 / rec1: records of rows r0 and r0 + 8; dl: digit rows (+ 8 t, permuted); colg: first
+// column of the super-block in the slice; gi: 128-column group of the half in the slice.
 template <int NT>
-__device__ __forceinline__ void q4k_half(const uint8_t* rec0, const uint8_t* rec1, int half, const int8_t* const (&dl)[NT],
-                                         const int (&dstep)[NT], int colg, const float* inv_scale, const int32_t* gsum,
+__device__ __forceinline__ void q4k_half(uint32_t rec0, uint32_t rec1, int half, const uint32_t (&dl)[NT],
+                                         const uint32_t (&dstep)[NT], int colg, uint32_t iscale, uint32_t gsum,
                                          int gstride, int gi, int t, float (&acc)[NT][2]) {
   const uint4 h0 = lds_v4(rec0);
   const uint4 h1 = lds_v4(rec1);
@@ -154,8 +264,8 @@ __device__ __forceinline__ void q4k_half(const uint8_t* rec0, const uint8_t* rec
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
     const int j = 4 * half + jj;
-    q0[jj] = lds_u32(rec0 + 16 + 16 * j + 4 * t);
-    q1[jj] = lds_u32(rec1 + 16 + 16 * j + 4 * t);
+    q0[jj] = lds_u32(rec0 + 16u + 16u * j + 4u * t);
+    q1[jj] = lds_u32(rec1 + 16u + 16u * j + 4u * t);
   }
   int32_t ai[NT][4];
 #pragma unroll
@@ -168,7 +278,7 @@ __device__ __forceinline__ void q4k_half(const uint8_t* rec0, const uint8_t* rec
     const int s0 = byte_u(sc0, jj), s1 = byte_u(sc1, jj);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const uint2 bb = *reinterpret_cast<const uint2*>(dl[nt] + dstep[nt] * (colg + 32 * j));
+      const uint2 bb = lds_v2(dl[nt] + dstep[nt] * (uint32_t)(colg + 32 * j));
       int32_t C[4] = {0, 0, 0, 0};
       mma_u8s8(C, a0, a1, a2, a3, bb.x, bb.y);
       ai[nt][0] += s0 * C[0];
@@ -179,11 +289,11 @@ __device__ __forceinline__ void q4k_half(const uint8_t* rec0, const uint8_t* rec
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int bb = 4 * nt + t;
-    const float isc = inv_scale[bb * gstride + gi];
+    const int item = (4 * nt + t) * gstride + gi;
+    const float isc = lds_f32(iscale + 4u * (uint32_t)item);
     // sums over the 32-column sub-blocks from the 16-column sums
-    const int4 Xa = *reinterpret_cast<const int4*>(gsum + (bb * gstride + gi) * 8);
-    const int4 Xb = *reinterpret_cast<const int4*>(gsum + (bb * gstride + gi) * 8 + 4);
+    const int4 Xa = lds_s4(gsum + 32u * (uint32_t)item);
+    const int4 Xb = lds_s4(gsum + 32u * (uint32_t)item + 16u);
     const int32_t X0 = Xa.x + Xa.y, X1 = Xa.z + Xa.w, X2 = Xb.x + Xb.y, X3 = Xb.z + Xb.w;
     const int32_t mx0 = byte_u(mn0, 0) * X0 + byte_u(mn0, 1) * X1 + byte_u(mn0, 2) * X2 + byte_u(mn0, 3) * X3;
     const int32_t mx1 = byte_u(mn1, 0) * X0 + byte_u(mn1, 1) * X1 + byte_u(mn1, 2) * X2 + byte_u(mn1, 3) * X3;
@@ -195,28 +305,26 @@ __device__ __forceinline__ void q4k_half(const uint8_t* rec0, const uint8_t* rec
 }
 
 // ---------------------------------------------------------------- Q6_K: half (8 sub-blocks of 16) of one super-block
+// odd: the rows' parity (their records' layout); dl: digit rows (+ 4 t, natural order).
 template <int NT>
-__device__ __forceinline__ void q6k_half(const uint8_t* rec0, const uint8_t* rec1, int odd, int half,
-                                         const int8_t* const (&dl)[NT], const int (&dstep)[NT], int colg,
-                                         const float* inv_scale, const int32_t* gsum, int gstride, int gi, int t,
-                                         float (&acc)[NT][2]) {
-  const uint8_t* qa0 = rec0 + (odd ? 2 : 0);
-  const uint8_t* qa1 = rec1 + (odd ? 2 : 0);
-  const uint8_t* sc0p = rec0 + (odd ? 194 : 192);
-  const uint8_t* sc1p = rec1 + (odd ? 194 : 192);
-  const float d0 = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec0 + (odd ? 0 : 208)));
-  const float d1 = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec1 + (odd ? 0 : 208)));
+__device__ __forceinline__ void q6k_half(uint32_t rec0, uint32_t rec1, int odd, int half, const uint32_t (&dl)[NT],
+                                         const uint32_t (&dstep)[NT], int colg, uint32_t iscale, uint32_t gsum,
+                                         int gstride, int gi, int t, float (&acc)[NT][2]) {
+  const uint32_t qa0 = rec0 + (odd ? 2u : 0u), qa1 = rec1 + (odd ? 2u : 0u);
+  const uint32_t sc0p = rec0 + (odd ? 194u : 192u), sc1p = rec1 + (odd ? 194u : 192u);
+  const float d0 = half_bits_to_float(lds_u16(rec0 + (odd ? 0u : 208u)));
+  const float d1 = half_bits_to_float(lds_u16(rec1 + (odd ? 0u : 208u)));
   int32_t ai[NT][4], ao[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = ao[nt][0] = ao[nt][1] = 0;
 #pragma unroll
   for (int mm = 0; mm < 2; ++mm) {
     const int m = 2 * half + mm;
-    const uint8_t* w0 = qa0 + 48 * t + 12 * m;
-    const uint8_t* w1 = qa1 + 48 * t + 12 * m;
-    const uint32_t A0 = lds_u32(w0), B0 = lds_u32(w0 + 4), C0 = lds_u32(w0 + 8);
-    const uint32_t A1 = lds_u32(w1), B1 = lds_u32(w1 + 4), C1 = lds_u32(w1 + 8);
-    const uint32_t scw0 = lds_u32(sc0p + 4 * m), scw1 = lds_u32(sc1p + 4 * m);
+    const uint32_t w0 = qa0 + 48u * t + 12u * m;
+    const uint32_t w1 = qa1 + 48u * t + 12u * m;
+    const uint32_t A0 = lds_u32(w0), B0 = lds_u32(w0 + 4u), C0 = lds_u32(w0 + 8u);
+    const uint32_t A1 = lds_u32(w1), B1 = lds_u32(w1 + 4u), C1 = lds_u32(w1 + 8u);
+    const uint32_t scw0 = lds_u32(sc0p + 4u * m), scw1 = lds_u32(sc1p + 4u * m);
     uint32_t op0[4], op1[4];
     op0[0] = (A0 & 0x0F0F0F0Fu) | (C0 & 0x30303030u);
     op0[1] = ((A0 >> 4) & 0x0F0F0F0Fu) | ((C0 >> 2) & 0x30303030u);
@@ -232,14 +340,14 @@ __device__ __forceinline__ void q6k_half(const uint8_t* rec0, const uint8_t* rec
       const int s0 = byte_s(scw0, s), s1 = byte_s(scw1, s);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(dl[nt] + dstep[nt] * (colg + 16 * j));
+        const uint32_t b0 = lds_u32(dl[nt] + dstep[nt] * (uint32_t)(colg + 16 * j));
         int32_t C[4] = {0, 0, 0, 0};
         mma_u8s8_k16(C, op0[s], op1[s], b0);
         ai[nt][0] += s0 * C[0];
         ai[nt][1] += s0 * C[1];
         ai[nt][2] += s1 * C[2];
         ai[nt][3] += s1 * C[3];
-        const int32_t X = gsum[((4 * nt + t) * gstride + gi) * 8 + (j & 7)];
+        const int32_t X = (int32_t)lds_u32(gsum + 4u * (uint32_t)(((4 * nt + t) * gstride + gi) * 8 + (j & 7)));
         ao[nt][0] += s0 * X;
         ao[nt][1] += s1 * X;
       }
@@ -247,7 +355,7 @@ __device__ __forceinline__ void q6k_half(const uint8_t* rec0, const uint8_t* rec
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float isc = inv_scale[(4 * nt + t) * gstride + gi];
+    const float isc = lds_f32(iscale + 4u * (uint32_t)((4 * nt + t) * gstride + gi));
     const float v0 = fmaf(256.f, (float)ai[nt][0], fmaf(-32.f, (float)ao[nt][0], (float)ai[nt][1]));
     const float v1 = fmaf(256.f, (float)ai[nt][2], fmaf(-32.f, (float)ao[nt][1], (float)ai[nt][3]));
     acc[nt][0] = fmaf(isc * d0, v0, acc[nt][0]);
@@ -255,234 +363,249 @@ __device__ __forceinline__ void q6k_half(const uint8_t* rec0, const uint8_t* rec
   }
 }
 
+// One tile for one warp (rows r0 and r0 + 8 of the 64): TSB Q4_K super-blocks, the tile's
+// first at super-block s0 of the slice.
+template <int NT, int TSB>
+__device__ __forceinline__ void tile_q4(uint32_t stage, const uint32_t (&dl)[NT], const uint32_t (&dstep)[NT],
+                                        uint32_t iscale, uint32_t gsum, int gstride, int s0, int r0, int t,
+                                        float (&acc)[NT][2]) {
+#pragma unroll
+  for (int k = 0; k < TSB; ++k) {
+    const uint32_t rec0 = stage + (uint32_t)((64 * k + r0) * 144);
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+      q4k_half<NT>(rec0, rec0 + 8u * 144u, half, dl, dstep, 256 * (s0 + k), iscale, gsum, gstride,
+                   2 * (s0 + k) + half, t, acc);
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ void tile_q6(uint32_t stage, const uint32_t (&dl)[NT], const uint32_t (&dstep)[NT],
+                                        uint32_t iscale, uint32_t gsum, int gstride, int s0, int r0, int t,
+                                        float (&acc)[NT][2]) {
+  const uint32_t rec0 = stage + (uint32_t)(r0 * 210);
+#pragma unroll
+  for (int half = 0; half < 2; ++half)
+    q6k_half<NT>(rec0, rec0 + 8u * 210u, r0 & 1, half, dl, dstep, 256 * s0, iscale, gsum, gstride, 2 * s0 + half, t,
+                 acc);
+}
+
 template <int MAXP, int NT>
 __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ TileHdr hdr[kStages];
+  __shared__ Slot slots[kMaxSlots];
   __shared__ __align__(16) uint8_t zeros[160];
-  __shared__ int s_ticket;
+  __shared__ int s_ticket[kTeams];
+  __shared__ int s_nslots;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u_begin = a.cta_begin[blockIdx.x], u_end = a.cta_begin[blockIdx.x + 1];
   if (u_begin >= u_end) return;
-  uint8_t* stages = smem;
-  int8_t* digits = reinterpret_cast<int8_t*>(smem + kStages * kStageBytes);
-  const int ndrows = 2 * a.batch;
-  const int max_groups = 2 * a.max_slice_sb;
-  float* inv_scale = reinterpret_cast<float*>(smem + kStages * kStageBytes + (size_t)ndrows * a.digit_stride);
-  int32_t* gsum = reinterpret_cast<int32_t*>(inv_scale + 4 * NT * max_groups);
-  float* xfer = reinterpret_cast<float*>(gsum + 4 * NT * max_groups * 8);  // [4 mt][3][NT][64]
+  const int nunits = u_end - u_begin;
 
   if (threadIdx.x < 40) reinterpret_cast<uint32_t*>(zeros)[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kConsumerWarps);
+      mbar_init(&empty_bar[s], kTeamWarps);
     }
     fence_mbar_init();
   }
-  __syncthreads();
-
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer warp: all lanes issue row copies
-    int s = 0;
-    uint32_t phase = 0, issued = 0;
-    int last_p = -1, last_j = -1;
-    Cursor c = cursor_at(a, u_begin);
-    for (; c.u < u_end; cursor_next(a, c)) {
-      const Problem& P = a.p[c.p];
-      const bool q4 = P.type == FL_GGML_Q4_K;
-      const int rec = q4 ? 144 : 210, tsbm = q4 ? kQ4Tsb : kQ6Tsb, slot = q4 ? kQ4Slot : kQ6Slot;
-      const int sb0s = c.j * P.slice_sb, nsbs = slice_nsb(P, c.j);
-      for (int t0 = 0; t0 < nsbs; t0 += tsbm) {
-        const int tsb = min(tsbm, nsbs - t0);
-        if (issued >= (uint32_t)kStages) {
-          bool ok = true;
-          if (lane == 0) ok = mbar_wait(&empty_bar[s], phase ^ 1u);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) {
-            if (lane == 0) atomicExch(&g_error, 1);
-            return;
-          }
-        }
-        const size_t start_off = (size_t)rec * (sb0s + t0);
-        const size_t a_off = start_off & ~(size_t)15;
-        const size_t e_off = (start_off + (size_t)rec * tsb + 15) & ~(size_t)15;
-        const uint32_t row_bytes = (uint32_t)(e_off - a_off);
-        uint8_t* st = stages + s * kStageBytes;
-        if (lane == 0) {
-          TileHdr& h = hdr[s];
-          h.kind = kTileData;
-          int fl = (t0 == 0 ? kFirst : 0) | (t0 + tsb >= nsbs ? kLast : 0);
-          if (t0 == 0 && (c.p != last_p || c.j != last_j)) fl |= kNewX;
-          h.flags = fl;
-          h.p = c.p;
-          h.j = c.j;
-          h.b = c.b;
-          h.sb0 = t0;
-          h.tsb = tsb;
-          h.off = (int)(start_off - a_off);
-          mbar_expect_tx(&full_bar[s], row_bytes * 64u);
-        }
-        if (t0 == 0) {
-          last_p = c.p;
-          last_j = c.j;
-        }
-        __syncwarp();
-        for (int r = lane; r < 64; r += 32) {
-          const uint8_t* src = P.blocks + (size_t)(64 * c.b + r) * P.nsb * rec + a_off;
-          bulk_g2s(st + slot * r, src, row_bytes, &full_bar[s]);
-        }
-        ++issued;
-        if (++s == kStages) {
-          s = 0;
-          phase ^= 1u;
+  if (warp == 0) {
+    // Slot table: lane i fills slot i, the i-th (problem, slice) pair from the CTA's first one
+    // (a multi-problem launch has one slice per problem); digit areas laid out back to back.
+    const uint32_t base = smem_u32(smem + kStages * kStageBytes);
+    const int s0 = a.cta_slice[blockIdx.x] >> 7, nsl_cta = a.cta_slice[blockIdx.x] & 127;
+    uint32_t carry = 0;
+    int items = 0, n = 0;
+    for (int i0 = 0; i0 < nsl_cta; i0 += 32) {
+      const int i = i0 + lane;
+      const bool live = i < nsl_cta;
+      Slot sl;
+      uint32_t bytes = 0;
+      int nit = 0;
+      if (live) {
+        const int p = (a.nproblems == 1) ? 0 : s0 + i;
+        const int j = (a.nproblems == 1) ? s0 + i : 0;
+        const Problem& P = a.p[p];
+        const int slice_start = P.unit_begin + j * P.nblocks;
+        const int first = max(slice_start, u_begin);
+        sl.p = p;
+        sl.j = j;
+        sl.u0 = first - u_begin;
+        sl.u1 = min(u_end, slice_start + P.nblocks) - u_begin;
+        sl.b0 = first - slice_start;
+        sl.nblocks = P.nblocks;
+        sl.nsb = P.nsb;
+        sl.nsbs = slice_nsb(P, j);
+        sl.slices = P.slices;
+        sl.sbfirst = j * P.slice_sb;
+        sl.type = P.type;
+        sl.ngroups = 2 * sl.nsbs;
+        sl.stride = 128 * sl.ngroups + 16;
+        sl.blocks = P.blocks;
+        sl.x = P.x;
+        sl.y = P.y;
+        sl.partial = P.partial;
+        sl.tickets = P.tickets;
+        bytes = (uint32_t)(2 * a.batch * sl.stride + 36 * 4 * NT * sl.ngroups);
+        nit = a.batch * sl.ngroups;
+      }
+      uint32_t incl = bytes;
+      int iincl = nit;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        const int w = __shfl_up_sync(0xffffffffu, iincl, o);
+        if (lane >= o) {
+          incl += v;
+          iincl += w;
         }
       }
+      if (live) {
+        sl.digits = base + carry + incl - bytes;
+        sl.iscale = sl.digits + (uint32_t)(2 * a.batch * sl.stride);
+        sl.gsum = sl.iscale + (uint32_t)(4 * 4 * NT * sl.ngroups);
+        sl.it0 = items + iincl - nit;
+        slots[i] = sl;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+      items += __shfl_sync(0xffffffffu, iincl, 31);
+      n += __popc(__ballot_sync(0xffffffffu, live));
     }
-    if (issued >= (uint32_t)kStages) {
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&empty_bar[s], phase ^ 1u);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) return;
-    }
-    if (lane == 0) {
-      hdr[s].kind = kTileEnd;
-      mbar_arrive(&full_bar[s]);
+    if (lane == 0) s_nslots = n;
+  }
+  __syncthreads();
+
+  // Team t (producer warp t and consumer warps 4t..4t+3) walks units t, t + kTeams, ... of the
+  // range; both sides derive the same tile sequence from the slot table, so the only hand-offs
+  // are the full / empty barriers of the team's two stages. The producers start copying once
+  // every consumer has issued its activation reads (kBarX), so those small reads do not queue
+  // behind the weight stream.
+  const int nsl = s_nslots;
+  if (warp >= kConsumerWarps) {
+    // ---------------------------------------------------------------- producer warps
+    named_bar(kBarX, kThreads);
+    if (lane != 0) return;
+    const int team = warp - kConsumerWarps;
+    int issued = 0, si = 0;
+    for (int k = team; k < nunits; k += kTeams) {
+      while (si + 1 < nsl && k >= slots[si].u1) ++si;
+      const Slot& sl = slots[si];
+      const int b = sl.b0 + (k - sl.u0);
+      const int rec = rec_bytes(sl.type), tsbm = tile_sb(sl.type);
+      const uint8_t* src = sl.blocks + ((size_t)b * sl.nsb + sl.sbfirst) * 64u * rec;
+      for (int s0 = 0; s0 < sl.nsbs; s0 += tsbm) {
+        const int tsb = min(tsbm, sl.nsbs - s0);
+        const int s = kTeamStages * team + (issued % kTeamStages);
+        if (issued >= kTeamStages &&
+            !mbar_wait(&empty_bar[s], (uint32_t)((issued / kTeamStages - 1) & 1))) {
+          atomicExch(&g_error, 1);
+          return;
+        }
+        const uint32_t bytes = (uint32_t)(tsb * 64 * rec);
+        mbar_expect_tx(&full_bar[s], bytes);
+        bulk_g2s(smem + s * kStageBytes, src + (size_t)s0 * 64u * rec, bytes, &full_bar[s]);
+        ++issued;
+      }
     }
     return;
   }
 
-  // -------------------------------------------------------------- consumer warps
-  const int mt = warp & 3, sq = warp >> 2;
+  // ------------------------------------------------------------------ consumer warps
+  // 1. activation digits of every (problem, slice) the range touches
+  build_digits(slots, nsl, a.batch, 4 * NT, threadIdx.x, kConsumers);
+  named_bar(kBarDigits, kConsumers);
+
+  // 2. team loop
+  const int team = warp / kTeamWarps, mt = warp % kTeamWarps;
+  const int tt = threadIdx.x % kTeamThreads;
   const int g = lane >> 2, t = lane & 3;
   const int r0 = 16 * mt + g;
-  const int8_t* dl_perm[NT];
-  const int8_t* dl_nat[NT];
-  int dstep[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int row = 8 * nt + g;
-    const bool live = row < ndrows;
-    dl_perm[nt] = live ? digits + (size_t)row * a.digit_stride + 8 * t : reinterpret_cast<const int8_t*>(zeros) + 8 * t;
-    dl_nat[nt] = live ? digits + (size_t)row * a.digit_stride + 4 * t : reinterpret_cast<const int8_t*>(zeros) + 4 * t;
-    dstep[nt] = live ? 1 : 0;
-  }
-  float acc[NT][2];
-  int gstride = 2;
-  int s = 0;
-  uint32_t phase = 0;
-  for (;;) {
-    if (!mbar_wait(&full_bar[s], phase)) {
-      if (lane == 0) atomicExch(&g_error, 2);
-      return;
-    }
-    const TileHdr h = hdr[s];
-    if (h.kind == kTileEnd) break;
-    const Problem& P = a.p[h.p];
-    const bool q4 = P.type == FL_GGML_Q4_K;
-    if (h.flags & kNewX) {
-      named_bar(1, kConsumers);
-      gstride = 2 * slice_nsb(P, h.j);
-      XDigitView v;
-      v.digits = digits;
-      v.inv_scale = inv_scale;
-      v.gsum = gsum;
-      v.stride = a.digit_stride;
-      v.ngroups = gstride;
-      build_x_digits(P.x, P.nsb * 256, a.batch, 4 * NT, 256 * h.j * P.slice_sb, v, 8, threadIdx.x, kConsumers,
-                     q4 ? 1 : 0);
-      named_bar(1, kConsumers);
-    }
-    if (h.flags & kFirst) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-    }
-    const uint8_t* st = stages + s * kStageBytes;
-    const int rec = q4 ? 144 : 210, slot = q4 ? kQ4Slot : kQ6Slot;
-    // work items of the tile: (super-block k, half) = 2 tsb halves, item hh = 2 k + half
-    for (int hh = sq; hh < 2 * h.tsb; hh += 4) {
-      const int k = hh >> 1, half = hh & 1;
-      const uint8_t* rec0 = st + slot * r0 + h.off + rec * k;
-      const uint8_t* rec1 = rec0 + slot * 8;
-      const int sbs = h.sb0 + k;
-      const int gi = 2 * sbs + half;
-      if (q4)
-        q4k_half<NT>(rec0, rec1, half, dl_perm, dstep, 256 * sbs, inv_scale, gsum, gstride, gi, t, acc);
-      else
-        q6k_half<NT>(rec0, rec1, (h.j * P.slice_sb + sbs) & 1, half, dl_nat, dstep, 256 * sbs, inv_scale, gsum,
-                     gstride, gi, t, acc);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
-    if (++s == kStages) {
-      s = 0;
-      phase ^= 1u;
-    }
-    if (!(h.flags & kLast)) continue;
-
-    float* xf = xfer + (size_t)mt * 3 * NT * 64;
-    if (sq > 0) {
+  const uint32_t smem_base = smem_u32(smem);
+  uint32_t dl[NT], dstep[NT];
+  int cur_slot = -1, si = 0, used = 0;
+  for (int k = team; k < nunits; k += kTeams) {
+    while (si + 1 < nsl && k >= slots[si].u1) ++si;
+    const Slot& sl = slots[si];
+    const int b = sl.b0 + (k - sl.u0);
+    const bool q4 = sl.type == FL_GGML_Q4_K;
+    if (si != cur_slot) {
+      cur_slot = si;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        xf[((sq - 1) * NT + nt) * 64 + lane] = acc[nt][0];
-        xf[((sq - 1) * NT + nt) * 64 + 32 + lane] = acc[nt][1];
+        const int row = 8 * nt + g;
+        const bool liveb = row < 2 * a.batch;
+        const uint32_t lane_off = q4 ? 8u * t : 4u * t;
+        dl[nt] = (liveb ? sl.digits + (uint32_t)(row * sl.stride) : smem_u32(zeros)) + lane_off;
+        dstep[nt] = liveb ? 1u : 0u;
       }
     }
-    named_bar(2 + mt, 128);
-    if (sq == 0) {
+    const uint32_t iscale = sl.iscale, gsum = sl.gsum;
+    const int gstride = sl.ngroups;
+    float acc[NT][2];
 #pragma unroll
-      for (int q = 0; q < 3; ++q)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[nt][0] += xf[(q * NT + nt) * 64 + lane];
-          acc[nt][1] += xf[(q * NT + nt) * 64 + 32 + lane];
-        }
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
+    const int tsbm = q4 ? 2 : 1;
+    for (int s0 = 0; s0 < sl.nsbs; s0 += tsbm) {
+      const int s = kTeamStages * team + (used % kTeamStages);
+      if (!mbar_wait(&full_bar[s], (uint32_t)((used / kTeamStages) & 1))) {
+        if (lane == 0) atomicExch(&g_error, 2);
+        return;
+      }
+      const uint32_t stage = smem_base + s * kStageBytes;
+      if (!q4)
+        tile_q6<NT>(stage, dl, dstep, iscale, gsum, gstride, s0, r0, t, acc);
+      else if (s0 + 2 <= sl.nsbs)
+        tile_q4<NT, 2>(stage, dl, dstep, iscale, gsum, gstride, s0, r0, t, acc);
+      else
+        tile_q4<NT, 1>(stage, dl, dstep, iscale, gsum, gstride, s0, r0, t, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+      ++used;
     }
-    named_bar(2 + mt, 128);
-    const size_t ystride = (size_t)64 * P.nblocks;
-    const int row_base = 64 * h.b + 16 * mt;
-    if (P.slices == 1) {
-      if (sq == 0) {
+
+    // ---- unit done: this warp's 16 rows are final (or a slice partial)
+    const size_t ystride = (size_t)64 * sl.nblocks;
+    const int row_base = 64 * b + 16 * mt;
+    if (sl.slices == 1) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int bb = 4 * nt + t;
-          if (bb < a.batch) {
-            float* y0 = P.y + (size_t)bb * ystride + row_base + g;
-            y0[0] = acc[nt][0];
-            y0[8] = acc[nt][1];
-          }
+      for (int nt = 0; nt < NT; ++nt) {
+        const int bb = 4 * nt + t;
+        if (bb < a.batch) {
+          float* y0 = sl.y + (size_t)bb * ystride + row_base + g;
+          y0[0] = acc[nt][0];
+          y0[8] = acc[nt][1];
         }
       }
     } else {
-      if (sq == 0) {
+      // partial for this slice; the last team to finish the block adds the slices in order
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int bb = 4 * nt + t;
-          if (bb < a.batch) {
-            float* pp = P.partial + (((size_t)h.j * P.nblocks + h.b) * a.batch + bb) * 64 + 16 * mt + g;
-            pp[0] = acc[nt][0];
-            pp[8] = acc[nt][1];
-          }
+      for (int nt = 0; nt < NT; ++nt) {
+        const int bb = 4 * nt + t;
+        if (bb < a.batch) {
+          float* pp = sl.partial + (((size_t)sl.j * sl.nblocks + b) * a.batch + bb) * 64 + 16 * mt + g;
+          pp[0] = acc[nt][0];
+          pp[8] = acc[nt][1];
         }
       }
       __threadfence();
-      named_bar(1, kConsumers);
-      if (threadIdx.x == 0) s_ticket = (int)atomicAdd(&P.tickets[h.b], 1u);
-      named_bar(1, kConsumers);
-      if (s_ticket == P.slices - 1) {
+      named_bar(kBarTeam0 + team, kTeamThreads);
+      if (tt == 0) s_ticket[team] = (int)atomicAdd(&sl.tickets[b], 1u);
+      named_bar(kBarTeam0 + team, kTeamThreads);
+      if (s_ticket[team] == sl.slices - 1) {
         __threadfence();
-        for (int e = threadIdx.x; e < a.batch * 64; e += kConsumers) {
+        for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
           const int bb = e / 64, r = e % 64;
           float sum = 0.f;
-          for (int jj = 0; jj < P.slices; ++jj)
-            sum += __ldcg(P.partial + (((size_t)jj * P.nblocks + h.b) * a.batch + bb) * 64 + r);
-          P.y[(size_t)bb * ystride + 64 * h.b + r] = sum;
+          for (int jj = 0; jj < sl.slices; ++jj)
+            sum += __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + bb) * 64 + r);
+          sl.y[(size_t)bb * ystride + 64 * b + r] = sum;
         }
-        if (threadIdx.x == 0) P.tickets[h.b] = 0u;
+        if (tt == 0) sl.tickets[b] = 0u;
       }
-      named_bar(1, kConsumers);
+      named_bar(kBarTeam0 + team, kTeamThreads);
     }
   }
 }
@@ -493,20 +616,21 @@ struct Plan {
   int slices, slice_sb;
 };
 
-// Dynamic shared memory: stages, activation digits, per (padded batch, 128-column group)
-// the inverse scale plus 8 sub-group sums, and the cross-warp transfer of row sums.
-static size_t smem_bytes(int batch, int slice_sb) {
+// Shared memory of one slot's activation digits, scales and 16-column sums.
+static size_t slot_bytes(int batch, int nsbs) {
   const int nt = (batch + 3) / 4;
-  return (size_t)kStages * kStageBytes + (size_t)2 * batch * (256 * slice_sb + 16) +
-         (size_t)4 * nt * (2 * slice_sb) * 36 + (size_t)3072 * nt;
+  return (size_t)2 * batch * (256 * nsbs + 16) + (size_t)36 * 4 * nt * (2 * nsbs);
 }
 
+// Widest column slice (in super-blocks) whose digits fit in one slot.
 static int max_sb_fit(int batch) {
   const int nt = (batch + 3) / 4;
-  const long avail = (long)kSmemLimit - (long)kStages * kStageBytes - 32L * batch - 3072L * nt;
+  const long avail = (long)kDigitBudget - 32L * batch;
   return (int)std::max(1L, avail / (512L * batch + 288L * nt));
 }
 
+// Column split for a single tensor: enough units to fill the GPU, slices of whole
+// super-blocks, and a slice narrow enough for the activation digits to fit in smem.
 static Plan plan_single(int nblocks, int nsb, int batch, int nsm) {
   Plan pl;
   const int max_sb = max_sb_fit(batch);
@@ -525,35 +649,63 @@ static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
   return tickets + (size_t)pl.slices * nblocks * batch * 64 * 4;
 }
 
+// Contiguous byte-balanced unit ranges, one per CTA. A range is also closed early when the
+// digits of its distinct (problem, slice) pairs would overflow shared memory or at kMaxSlots
+// pairs; such cuts can make more ranges than SMs (a second, partial wave).
 template <int MAXP>
-static void partition(Args<MAXP>& a, int nsm) {
+static bool partition(Args<MAXP>& a, int nsm) {
   double total = 0;
-  for (int i = 0; i < a.nproblems; ++i)
-    total += (double)a.p[i].nblocks * a.p[i].nsb * (a.p[i].type == FL_GGML_Q4_K ? 144 : 210);
+  for (int i = 0; i < a.nproblems; ++i) total += (double)a.p[i].nblocks * a.p[i].nsb * rec_bytes(a.p[i].type);
   const Problem& L = a.p[a.nproblems - 1];
   const int units = L.unit_begin + L.nblocks * L.slices;
-  int ncta = std::max(1, std::min(std::min(nsm, units), kMaxCtas));
-  a.ncta = ncta;
-  int c = 0;
+  const int target = std::max(1, std::min(nsm, units));
+  const double per_cta = total / target;
+  int n = 0;
   a.cta_begin[0] = 0;
+  a.cta_slice[0] = 0;
   double acc = 0;
-  for (int i = 0; i < a.nproblems && c < ncta; ++i) {
+  size_t dig = 0;
+  int nslots = 0, count = 0;
+  for (int i = 0; i < a.nproblems; ++i) {
     const Problem& P = a.p[i];
-    const int nu = P.nblocks * P.slices;
-    const double per = (double)P.nsb * (P.type == FL_GGML_Q4_K ? 144 : 210) / P.slices;
-    for (int k = 0; k < nu; ++k) {
-      acc += per;
-      const int u = P.unit_begin + k + 1;
-      while (c + 1 < ncta && acc >= total * (c + 1) / ncta) a.cta_begin[++c] = u;
+    for (int j = 0; j < P.slices; ++j) {
+      const int ns = std::min(P.slice_sb, P.nsb - j * P.slice_sb);
+      const size_t sb = slot_bytes(a.batch, ns);
+      const double cost = (double)ns * rec_bytes(P.type);
+      for (int b = 0; b < P.nblocks; ++b) {
+        const int u = P.unit_begin + j * P.nblocks + b;
+        bool cut = false;
+        if (count > 0) {
+          if (n + 1 < target && acc + 0.5 * cost > per_cta * (n + 1)) cut = true;
+          if (b == 0 && (dig + sb > (size_t)kDigitBudget || nslots == kMaxSlots)) cut = true;
+        }
+        if (cut) {
+          if (n + 1 >= kMaxCtas) return false;
+          a.cta_slice[n] |= nslots;
+          a.cta_begin[++n] = u;
+          a.cta_slice[n] = ((a.nproblems == 1) ? j : i) << 7;
+          dig = 0;
+          nslots = 0;
+          count = 0;
+        }
+        if (b == 0 || count == 0) {
+          dig += sb;
+          ++nslots;
+        }
+        acc += cost;
+        ++count;
+      }
     }
   }
-  while (c + 1 < ncta) a.cta_begin[++c] = units;
-  a.cta_begin[ncta] = units;
+  a.cta_slice[n] |= nslots;
+  a.cta_begin[++n] = units;
+  a.ncta = n;
+  return true;
 }
 
 template <int MAXP, int NT>
 static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
-  const size_t smem = smem_bytes(a.batch, a.max_slice_sb);
+  const size_t smem = (size_t)kSmemLimit;
   auto kern = kquant_gemv_kernel<MAXP, NT>;
   FL_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                 "cudaFuncSetAttribute(kquant_gemv)");
@@ -577,9 +729,8 @@ static fl_status check_tensor(const void* blocks, int type, int out, int in, con
     return fail(FL_ERR_UNSUPPORTED, "%s: tensor %d has GGUF type %d; the fast path implements Q4_K (12) and Q6_K (14)",
                 what, idx, type);
   if (!blocks) return fail(FL_ERR_ARG, "%s: tensor %d blocks pointer is NULL", what, idx);
-  if (out <= 0 || out % 64 || in <= 0 || in % 256 || (type == FL_GGML_Q6_K && in % 2048))
-    return fail(FL_ERR_SHAPE, "%s: tensor %d out=%d in=%d (out %% 64 == 0, in %% 256 == 0, Q6_K in %% 2048 == 0)",
-                what, idx, out, in);
+  if (out <= 0 || out % 64 || in <= 0 || in % 256)
+    return fail(FL_ERR_SHAPE, "%s: tensor %d out=%d in=%d (out %% 64 == 0, in %% 256 == 0)", what, idx, out, in);
   if (!aligned16(blocks)) return fail(FL_ERR_ALIGN, "%s: tensor %d blocks not 16-byte aligned", what, idx);
   return FL_OK;
 }
@@ -625,8 +776,6 @@ extern "C" fl_status fl_gemv_kquant(const void* blocks, int ggml_type, int out, 
   static thread_local kq::Args<1> a;
   a.nproblems = 1;
   a.batch = batch;
-  a.max_slice_sb = pl.slice_sb;
-  a.digit_stride = 256 * pl.slice_sb + 16;
   kq::Problem& P = a.p[0];
   P.blocks = static_cast<const uint8_t*>(blocks);
   P.x = x;
@@ -645,7 +794,7 @@ extern "C" fl_status fl_gemv_kquant(const void* blocks, int ggml_type, int out, 
     P.tickets = nullptr;
     P.partial = nullptr;
   }
-  kq::partition(a, nsm);
+  if (!kq::partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: tensor too large for one launch", what);
   return kq::launch_nt(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -657,7 +806,7 @@ extern "C" fl_status fl_gemv_kquant_batched(const fl_kquant_problem* problems, i
   static thread_local kq::Args<FL_MAX_PROBLEMS> a;
   a.nproblems = n;
   a.batch = batch;
-  int max_sb = 0, unit = 0;
+  int unit = 0;
   for (int i = 0; i < n; ++i) {
     const fl_kquant_problem& q = problems[i];
     fl_status st = kq::check_tensor(q.blocks, q.ggml_type, q.out, q.in, what, i);
@@ -681,12 +830,9 @@ extern "C" fl_status fl_gemv_kquant_batched(const fl_kquant_problem* problems, i
     P.slice_sb = nsb;
     P.unit_begin = unit;
     unit += P.nblocks;
-    max_sb = std::max(max_sb, nsb);
   }
-  a.max_slice_sb = max_sb;
-  a.digit_stride = 256 * max_sb + 16;
   const int nsm = device_sm_count();
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
-  kq::partition(a, nsm);
+  if (!kq::partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: tensors too large for one launch", what);
   return kq::launch_nt(a, static_cast<cudaStream_t>(stream));
 }

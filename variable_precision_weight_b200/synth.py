@@ -86,13 +86,14 @@ def _fp16(a):
 
 
 def encode_q4k(w: np.ndarray) -> np.ndarray:
-    """Encode rows of weights (in % 256 == 0) as 144-byte Q4_K records, row-major.
+    """Encode rows of weights (out % 64 == 0, in % 256 == 0) as 144-byte Q4_K records in
+    block-tiled order (see kquant_tile_order).
 
-    Layout: [0,2) d fp16, [2,4) dmin fp16, byte 4 + j = sc_j | (mn_j & 3) << 6,
+    Record: [0,2) d fp16, [2,4) dmin fp16, byte 4 + j = sc_j | (mn_j & 3) << 6,
     nibble j of the word at 12 = mn_j >> 2, byte 16 + 16 j + b = q[32 j + b] | q[32 j + 16 + b] << 4.
     """
     out, inn = w.shape
-    assert inn % 256 == 0
+    assert inn % 256 == 0 and out % 64 == 0
     sb = w.reshape(-1, 8, 32).astype(np.float32)
     n = sb.shape[0]
     lo = np.minimum(sb.min(axis=2), 0.0).astype(np.float32)
@@ -118,21 +119,24 @@ def encode_q4k(w: np.ndarray) -> np.ndarray:
     nib = (mn >> 2).astype(np.uint8)
     rec[:, 12:16] = nib[:, 0::2] | (nib[:, 1::2] << 4)
     rec[:, 16:144] = (q[:, :, :16] | (q[:, :, 16:] << 4)).reshape(n, 128)
-    return rec.reshape(-1)
+    return kquant_tile_order(rec, out, inn // 256)
 
 
 def encode_q6k(w: np.ndarray) -> np.ndarray:
-    """Encode rows of weights (in % 2048 == 0) as 210-byte Q6_K records, row-major.
+    """Encode rows of weights (out % 64 == 0, in % 256 == 0) as 210-byte Q6_K records in
+    block-tiled order (see kquant_tile_order).
 
-    A record's layout depends on its index n in its row: n even -> [0,192) q, [192,208)
-    int8 scales, [208,210) d; n odd -> [0,2) d, [2,194) q, [194,210) scales. The q area
+    A record's layout depends on the parity of its row: even row -> [0,192) q, [192,208)
+    int8 scales, [208,210) d; odd row -> [0,2) d, [2,194) q, [194,210) scales (in the tiled
+    order an odd row's record starts 2 bytes past a 4-byte boundary, so its q area is
+    4-byte aligned). The q area
     holds, for chunk t (48 bytes) and group m (12 bytes: words A, B, C), with
     W(j, L) = 16 j + 4 t + L: A byte L = lo4 q[W(4m,L)] | lo4 q[W(4m+1,L)] << 4,
     B byte L = lo4 q[W(4m+2,L)] | lo4 q[W(4m+3,L)] << 4, C byte L = hi2 q[W(4m+2,L)]
     | hi2 q[W(4m+3,L)] << 2 | hi2 q[W(4m,L)] << 4 | hi2 q[W(4m+1,L)] << 6.
     """
     out, inn = w.shape
-    assert inn % 2048 == 0, "Q6_K rows must hold a multiple of 8 records"
+    assert inn % 256 == 0 and out % 64 == 0
     sb = w.reshape(-1, 16, 16).astype(np.float32)
     n = sb.shape[0]
     a = (np.abs(sb).max(axis=2) / np.float32(31.0)).astype(np.float32)
@@ -154,7 +158,7 @@ def encode_q6k(w: np.ndarray) -> np.ndarray:
     rec = np.zeros((n, 210), np.uint8)
     scb = sc.astype(np.int8).view(np.uint8)
     db = d16.view(np.uint8).reshape(n, 2)
-    even = (np.arange(n) % 2) == 0                                 # rows hold an even count of records
+    even = ((np.arange(n) // (inn // 256)) % 2) == 0               # record n belongs to row n // (in / 256)
     rec[even, 0:192] = area[even]
     rec[even, 192:208] = scb[even]
     rec[even, 208:210] = db[even]
@@ -162,7 +166,15 @@ def encode_q6k(w: np.ndarray) -> np.ndarray:
     rec[odd, 0:2] = db[odd]
     rec[odd, 2:194] = area[odd]
     rec[odd, 194:210] = scb[odd]
-    return rec.reshape(-1)
+    return kquant_tile_order(rec, out, inn // 256)
+
+
+def kquant_tile_order(rec: np.ndarray, out: int, nsb: int) -> np.ndarray:
+    """Row-major records [out][nsb][bytes] -> block-tiled [out / 64][nsb][64][bytes], flat.
+
+    A tile of 64 rows x k consecutive super-blocks is then one contiguous byte range."""
+    nb = rec.shape[-1]
+    return np.ascontiguousarray(rec.reshape(out // 64, 64, nsb, nb).transpose(0, 2, 1, 3)).reshape(-1)
 
 
 def encode_kquant(w: np.ndarray, ggml_type: int) -> np.ndarray:

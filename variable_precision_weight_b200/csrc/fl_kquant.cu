@@ -148,6 +148,45 @@ __device__ __forceinline__ int4 lds_s4(uint32_t a) {
 
 __device__ __forceinline__ int slice_nsb(const Problem& P, int j) { return min(P.slice_sb, P.nsb - j * P.slice_sb); }
 
+// A slot's digit area, batch rows padded to 4 NT. The padded strides spread the rows that
+// one warp reads together over distinct shared-memory banks.
+//   digits: 2 batch rows of digit_stride bytes (hi, lo)
+//   iscale: [4 NT][ngroups + 1] floats, area rounded up to 16 bytes
+//   gsum:   [4 NT][gsum_row bytes]: per 128-column group 8 int32 sums of 16 columns
+__host__ __device__ constexpr int digit_stride(int ngroups) { return 128 * ngroups + 32; }
+__host__ __device__ constexpr int iscale_row(int ngroups) { return ngroups + 1; }
+__host__ __device__ constexpr int gsum_row(int ngroups) { return 32 * ngroups + 16; }
+__host__ __device__ constexpr int iscale_area(int nt, int ngroups) { return (16 * nt * iscale_row(ngroups) + 15) & ~15; }
+__host__ __device__ constexpr int slot_area(int batch, int nt, int ngroups) {
+  return 2 * batch * digit_stride(ngroups) + iscale_area(nt, ngroups) + 4 * nt * gsum_row(ngroups);
+}
+
+// Rows of the 64-row block held by lane row g of warp mt: Q4_K records (144 B) are
+// bank-conflict free for consecutive rows; Q6_K records (210 B) are when the eight rows of
+// a fragment half are {0, 1, 3, 5} or {7, 2, 4, 6} of an 8-row group plus the same rows 32
+// further on.
+__device__ __forceinline__ int q6_row(int mt, int h, int g) {
+  const int x = g & 3;
+  return 8 * mt + (x == 0 ? (h ? 7 : 0) : 2 * x - 1 + h) + 32 * (g >> 2);
+}
+
+__device__ __forceinline__ uint2 lds_v2_if(uint32_t a, bool p) {
+  uint2 v;
+  asm volatile(
+      "{ .reg .pred q; setp.ne.u32 q, %3, 0; mov.u32 %0, 0; mov.u32 %1, 0; @q ld.shared.v2.u32 {%0,%1}, [%2]; }"
+      : "=r"(v.x), "=r"(v.y)
+      : "r"(a), "r"((uint32_t)p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u32_if(uint32_t a, bool p) {
+  uint32_t v;
+  asm volatile("{ .reg .pred q; setp.ne.u32 q, %2, 0; mov.u32 %0, 0; @q ld.shared.u32 %0, [%1]; }"
+               : "=r"(v)
+               : "r"(a), "r"((uint32_t)p));
+  return v;
+}
+
 // ---------------------------------------------------------------- activation digits
 // One item = 128 columns of one batch row (see fl_common.cuh for the number format),
 // converted by one warp; the Q4_K slots store each word at the place its m16n8k32 B
@@ -185,12 +224,13 @@ __device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, i
   // sums of 16 columns (4 lanes each)
   part += __shfl_xor_sync(0xffffffffu, part, 1);
   part += __shfl_xor_sync(0xffffffffu, part, 2);
-  const int item = b * sl.ngroups + g;
   if ((lane & 3) == 0)
-    asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + 4u * (uint32_t)(8 * item + (lane >> 2))), "r"(part)
+    asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + (uint32_t)(b * gsum_row(sl.ngroups) + 32 * g + (lane & ~3))),
+                 "r"(part)
                  : "memory");
   if (lane == 0)
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)item), "f"(ldexpf(1.0f, -sigma))
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)(b * iscale_row(sl.ngroups) + g)),
+                 "f"(ldexpf(1.0f, -sigma))
                  : "memory");
 }
 
@@ -233,22 +273,27 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
     const Slot& sl = slots[i];
     const int n = (batch_pad - batch) * sl.ngroups;
     for (int e = tid; e < 9 * n; e += nthreads) {
-      const int item = batch * sl.ngroups + e % n;
+      const int b = batch + (e % n) / sl.ngroups, g = (e % n) % sl.ngroups;
       if (e < n)
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)item), "f"(0.f) : "memory");
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)(b * iscale_row(sl.ngroups) + g)),
+                     "f"(0.f)
+                     : "memory");
       else
-        asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + 4u * (uint32_t)(8 * item + (e / n - 1))), "r"(0)
+        asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + (uint32_t)(b * gsum_row(sl.ngroups) + 32 * g +
+                                                                         4 * (e / n - 1))),
+                     "r"(0)
                      : "memory");
     }
   }
 }
 
 // ---------------------------------------------------------------- Q4_K: half (4 sub-blocks) of one super-block
-// rec0 / rec1: records of rows r0 and r0 + 8; dl: digit rows (+ 8 t, permuted); colg: first
+// rec0 / rec1: records of the lane's two rows; dl: digit rows (+ 8 t, permuted), live: whether
+// the lane's digit row is a real batch row (else its B fragment is zero); colg: first
 // column of the super-block in the slice; gi: 128-column group of the half in the slice.
 template <int NT>
 __device__ __forceinline__ void q4k_half(uint32_t rec0, uint32_t rec1, int half, const uint32_t (&dl)[NT],
-                                         const uint32_t (&dstep)[NT], int colg, uint32_t iscale, uint32_t gsum,
+                                         const bool (&live)[NT], int colg, uint32_t iscale, uint32_t gsum,
                                          int gstride, int gi, int t, float (&acc)[NT][2]) {
   const uint4 h0 = lds_v4(rec0);
   const uint4 h1 = lds_v4(rec1);
@@ -278,7 +323,7 @@ __device__ __forceinline__ void q4k_half(uint32_t rec0, uint32_t rec1, int half,
     const int s0 = byte_u(sc0, jj), s1 = byte_u(sc1, jj);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const uint2 bb = lds_v2(dl[nt] + dstep[nt] * (uint32_t)(colg + 32 * j));
+      const uint2 bb = lds_v2_if(dl[nt] + (uint32_t)(colg + 32 * j), live[nt]);
       int32_t C[4] = {0, 0, 0, 0};
       mma_u8s8(C, a0, a1, a2, a3, bb.x, bb.y);
       ai[nt][0] += s0 * C[0];
@@ -289,11 +334,12 @@ __device__ __forceinline__ void q4k_half(uint32_t rec0, uint32_t rec1, int half,
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int item = (4 * nt + t) * gstride + gi;
-    const float isc = lds_f32(iscale + 4u * (uint32_t)item);
+    const int bb = 4 * nt + t;
+    const float isc = lds_f32(iscale + 4u * (uint32_t)(bb * iscale_row(gstride) + gi));
     // sums over the 32-column sub-blocks from the 16-column sums
-    const int4 Xa = lds_s4(gsum + 32u * (uint32_t)item);
-    const int4 Xb = lds_s4(gsum + 32u * (uint32_t)item + 16u);
+    const uint32_t ga = gsum + (uint32_t)(bb * gsum_row(gstride) + 32 * gi);
+    const int4 Xa = lds_s4(ga);
+    const int4 Xb = lds_s4(ga + 16u);
     const int32_t X0 = Xa.x + Xa.y, X1 = Xa.z + Xa.w, X2 = Xb.x + Xb.y, X3 = Xb.z + Xb.w;
     const int32_t mx0 = byte_u(mn0, 0) * X0 + byte_u(mn0, 1) * X1 + byte_u(mn0, 2) * X2 + byte_u(mn0, 3) * X3;
     const int32_t mx1 = byte_u(mn1, 0) * X0 + byte_u(mn1, 1) * X1 + byte_u(mn1, 2) * X2 + byte_u(mn1, 3) * X3;
@@ -307,16 +353,24 @@ __device__ __forceinline__ void q4k_half(uint32_t rec0, uint32_t rec1, int half,
 // ---------------------------------------------------------------- Q6_K: half (8 sub-blocks of 16) of one super-block
 // odd: the rows' parity (their records' layout); dl: digit rows (+ 4 t, natural order).
 template <int NT>
-__device__ __forceinline__ void q6k_half(uint32_t rec0, uint32_t rec1, int odd, int half, const uint32_t (&dl)[NT],
-                                         const uint32_t (&dstep)[NT], int colg, uint32_t iscale, uint32_t gsum,
-                                         int gstride, int gi, int t, float (&acc)[NT][2]) {
-  const uint32_t qa0 = rec0 + (odd ? 2u : 0u), qa1 = rec1 + (odd ? 2u : 0u);
-  const uint32_t sc0p = rec0 + (odd ? 194u : 192u), sc1p = rec1 + (odd ? 194u : 192u);
-  const float d0 = half_bits_to_float(lds_u16(rec0 + (odd ? 0u : 208u)));
-  const float d1 = half_bits_to_float(lds_u16(rec1 + (odd ? 0u : 208u)));
+__device__ __forceinline__ void q6k_half(uint32_t rec0, uint32_t rec1, int odd0, int odd1, int half,
+                                         const uint32_t (&dl)[NT], const bool (&live)[NT], int colg,
+                                         uint32_t iscale, uint32_t gsum, int gstride, int gi, int t,
+                                         float (&acc)[NT][2]) {
+  const uint32_t qa0 = rec0 + (odd0 ? 2u : 0u), qa1 = rec1 + (odd1 ? 2u : 0u);
+  const uint32_t sc0p = rec0 + (odd0 ? 194u : 192u), sc1p = rec1 + (odd1 ? 194u : 192u);
+  const float d0 = half_bits_to_float(lds_u16(rec0 + (odd0 ? 0u : 208u)));
+  const float d1 = half_bits_to_float(lds_u16(rec1 + (odd1 ? 0u : 208u)));
   int32_t ai[NT][4], ao[NT][2];
+  int32_t X[NT][8];  // the half's 16-column sums, per batch row
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = ao[nt][0] = ao[nt][1] = 0;
+  for (int nt = 0; nt < NT; ++nt) {
+    ai[nt][0] = ai[nt][1] = ai[nt][2] = ai[nt][3] = ao[nt][0] = ao[nt][1] = 0;
+    const uint32_t ga = gsum + (uint32_t)((4 * nt + t) * gsum_row(gstride) + 32 * gi);
+    const int4 Xa = lds_s4(ga), Xb = lds_s4(ga + 16u);
+    X[nt][0] = Xa.x; X[nt][1] = Xa.y; X[nt][2] = Xa.z; X[nt][3] = Xa.w;
+    X[nt][4] = Xb.x; X[nt][5] = Xb.y; X[nt][6] = Xb.z; X[nt][7] = Xb.w;
+  }
 #pragma unroll
   for (int mm = 0; mm < 2; ++mm) {
     const int m = 2 * half + mm;
@@ -340,22 +394,21 @@ __device__ __forceinline__ void q6k_half(uint32_t rec0, uint32_t rec1, int odd, 
       const int s0 = byte_s(scw0, s), s1 = byte_s(scw1, s);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t b0 = lds_u32(dl[nt] + dstep[nt] * (uint32_t)(colg + 16 * j));
+        const uint32_t b0 = lds_u32_if(dl[nt] + (uint32_t)(colg + 16 * j), live[nt]);
         int32_t C[4] = {0, 0, 0, 0};
         mma_u8s8_k16(C, op0[s], op1[s], b0);
         ai[nt][0] += s0 * C[0];
         ai[nt][1] += s0 * C[1];
         ai[nt][2] += s1 * C[2];
         ai[nt][3] += s1 * C[3];
-        const int32_t X = (int32_t)lds_u32(gsum + 4u * (uint32_t)(((4 * nt + t) * gstride + gi) * 8 + (j & 7)));
-        ao[nt][0] += s0 * X;
-        ao[nt][1] += s1 * X;
+        ao[nt][0] += s0 * X[nt][j & 7];
+        ao[nt][1] += s1 * X[nt][j & 7];
       }
     }
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float isc = lds_f32(iscale + 4u * (uint32_t)((4 * nt + t) * gstride + gi));
+    const float isc = lds_f32(iscale + 4u * (uint32_t)((4 * nt + t) * iscale_row(gstride) + gi));
     const float v0 = fmaf(256.f, (float)ai[nt][0], fmaf(-32.f, (float)ao[nt][0], (float)ai[nt][1]));
     const float v1 = fmaf(256.f, (float)ai[nt][2], fmaf(-32.f, (float)ao[nt][1], (float)ai[nt][3]));
     acc[nt][0] = fmaf(isc * d0, v0, acc[nt][0]);
@@ -363,31 +416,30 @@ __device__ __forceinline__ void q6k_half(uint32_t rec0, uint32_t rec1, int odd, 
   }
 }
 
-// One tile for one warp (rows r0 and r0 + 8 of the 64): TSB Q4_K super-blocks, the tile's
-// first at super-block s0 of the slice.
+// One tile for one warp (rows row0 / row1 of the 64 per lane): TSB Q4_K super-blocks, the
+// tile's first at super-block s0 of the slice.
 template <int NT, int TSB>
-__device__ __forceinline__ void tile_q4(uint32_t stage, const uint32_t (&dl)[NT], const uint32_t (&dstep)[NT],
-                                        uint32_t iscale, uint32_t gsum, int gstride, int s0, int r0, int t,
+__device__ __forceinline__ void tile_q4(uint32_t stage, const uint32_t (&dl)[NT], const bool (&live)[NT],
+                                        uint32_t iscale, uint32_t gsum, int gstride, int s0, int row0, int row1, int t,
                                         float (&acc)[NT][2]) {
 #pragma unroll
   for (int k = 0; k < TSB; ++k) {
-    const uint32_t rec0 = stage + (uint32_t)((64 * k + r0) * 144);
+    const uint32_t blk = stage + (uint32_t)(64 * 144 * k);
 #pragma unroll
     for (int half = 0; half < 2; ++half)
-      q4k_half<NT>(rec0, rec0 + 8u * 144u, half, dl, dstep, 256 * (s0 + k), iscale, gsum, gstride,
+      q4k_half<NT>(blk + 144u * row0, blk + 144u * row1, half, dl, live, 256 * (s0 + k), iscale, gsum, gstride,
                    2 * (s0 + k) + half, t, acc);
   }
 }
 
 template <int NT>
-__device__ __forceinline__ void tile_q6(uint32_t stage, const uint32_t (&dl)[NT], const uint32_t (&dstep)[NT],
-                                        uint32_t iscale, uint32_t gsum, int gstride, int s0, int r0, int t,
+__device__ __forceinline__ void tile_q6(uint32_t stage, const uint32_t (&dl)[NT], const bool (&live)[NT],
+                                        uint32_t iscale, uint32_t gsum, int gstride, int s0, int row0, int row1, int t,
                                         float (&acc)[NT][2]) {
-  const uint32_t rec0 = stage + (uint32_t)(r0 * 210);
 #pragma unroll
   for (int half = 0; half < 2; ++half)
-    q6k_half<NT>(rec0, rec0 + 8u * 210u, r0 & 1, half, dl, dstep, 256 * s0, iscale, gsum, gstride, 2 * s0 + half, t,
-                 acc);
+    q6k_half<NT>(stage + 210u * row0, stage + 210u * row1, row0 & 1, row1 & 1, half, dl, live, 256 * s0, iscale,
+                 gsum, gstride, 2 * s0 + half, t, acc);
 }
 
 template <int MAXP, int NT>
@@ -395,7 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ Slot slots[kMaxSlots];
-  __shared__ __align__(16) uint8_t zeros[160];
   __shared__ int s_ticket[kTeams];
   __shared__ int s_nslots;
 
@@ -404,7 +455,6 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   if (u_begin >= u_end) return;
   const int nunits = u_end - u_begin;
 
-  if (threadIdx.x < 40) reinterpret_cast<uint32_t*>(zeros)[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -443,13 +493,13 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
         sl.sbfirst = j * P.slice_sb;
         sl.type = P.type;
         sl.ngroups = 2 * sl.nsbs;
-        sl.stride = 128 * sl.ngroups + 16;
+        sl.stride = digit_stride(sl.ngroups);
         sl.blocks = P.blocks;
         sl.x = P.x;
         sl.y = P.y;
         sl.partial = P.partial;
         sl.tickets = P.tickets;
-        bytes = (uint32_t)(2 * a.batch * sl.stride + 36 * 4 * NT * sl.ngroups);
+        bytes = (uint32_t)slot_area(a.batch, NT, sl.ngroups);
         nit = a.batch * sl.ngroups;
       }
       uint32_t incl = bytes;
@@ -466,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       if (live) {
         sl.digits = base + carry + incl - bytes;
         sl.iscale = sl.digits + (uint32_t)(2 * a.batch * sl.stride);
-        sl.gsum = sl.iscale + (uint32_t)(4 * 4 * NT * sl.ngroups);
+        sl.gsum = sl.iscale + (uint32_t)iscale_area(NT, sl.ngroups);
         sl.it0 = items + iincl - nit;
         slots[i] = sl;
       }
@@ -522,9 +572,10 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   const int team = warp / kTeamWarps, mt = warp % kTeamWarps;
   const int tt = threadIdx.x % kTeamThreads;
   const int g = lane >> 2, t = lane & 3;
-  const int r0 = 16 * mt + g;
   const uint32_t smem_base = smem_u32(smem);
-  uint32_t dl[NT], dstep[NT];
+  uint32_t dl[NT];
+  bool live[NT];
+  int row0 = 0, row1 = 0;
   int cur_slot = -1, si = 0, used = 0;
   for (int k = team; k < nunits; k += kTeams) {
     while (si + 1 < nsl && k >= slots[si].u1) ++si;
@@ -535,12 +586,12 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       cur_slot = si;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int row = 8 * nt + g;
-        const bool liveb = row < 2 * a.batch;
-        const uint32_t lane_off = q4 ? 8u * t : 4u * t;
-        dl[nt] = (liveb ? sl.digits + (uint32_t)(row * sl.stride) : smem_u32(zeros)) + lane_off;
-        dstep[nt] = liveb ? 1u : 0u;
+        const int row = 8 * nt + g;  // digit row (2 per batch row) this lane's B fragment reads
+        live[nt] = row < 2 * a.batch;
+        dl[nt] = sl.digits + (uint32_t)(min(row, 2 * a.batch - 1) * sl.stride) + (q4 ? 8u * t : 4u * t);
       }
+      row0 = q4 ? 16 * mt + g : q6_row(mt, 0, g);
+      row1 = q4 ? 16 * mt + g + 8 : q6_row(mt, 1, g);
     }
     const uint32_t iscale = sl.iscale, gsum = sl.gsum;
     const int gstride = sl.ngroups;
@@ -556,11 +607,11 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       }
       const uint32_t stage = smem_base + s * kStageBytes;
       if (!q4)
-        tile_q6<NT>(stage, dl, dstep, iscale, gsum, gstride, s0, r0, t, acc);
+        tile_q6<NT>(stage, dl, live, iscale, gsum, gstride, s0, row0, row1, t, acc);
       else if (s0 + 2 <= sl.nsbs)
-        tile_q4<NT, 2>(stage, dl, dstep, iscale, gsum, gstride, s0, r0, t, acc);
+        tile_q4<NT, 2>(stage, dl, live, iscale, gsum, gstride, s0, row0, row1, t, acc);
       else
-        tile_q4<NT, 1>(stage, dl, dstep, iscale, gsum, gstride, s0, r0, t, acc);
+        tile_q4<NT, 1>(stage, dl, live, iscale, gsum, gstride, s0, row0, row1, t, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);
       ++used;
@@ -568,15 +619,14 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
 
     // ---- unit done: this warp's 16 rows are final (or a slice partial)
     const size_t ystride = (size_t)64 * sl.nblocks;
-    const int row_base = 64 * b + 16 * mt;
     if (sl.slices == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int bb = 4 * nt + t;
         if (bb < a.batch) {
-          float* y0 = sl.y + (size_t)bb * ystride + row_base + g;
-          y0[0] = acc[nt][0];
-          y0[8] = acc[nt][1];
+          float* yb = sl.y + (size_t)bb * ystride + 64 * b;
+          yb[row0] = acc[nt][0];
+          yb[row1] = acc[nt][1];
         }
       }
     } else {
@@ -585,9 +635,9 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       for (int nt = 0; nt < NT; ++nt) {
         const int bb = 4 * nt + t;
         if (bb < a.batch) {
-          float* pp = sl.partial + (((size_t)sl.j * sl.nblocks + b) * a.batch + bb) * 64 + 16 * mt + g;
-          pp[0] = acc[nt][0];
-          pp[8] = acc[nt][1];
+          float* pp = sl.partial + (((size_t)sl.j * sl.nblocks + b) * a.batch + bb) * 64;
+          pp[row0] = acc[nt][0];
+          pp[row1] = acc[nt][1];
         }
       }
       __threadfence();
@@ -617,16 +667,13 @@ struct Plan {
 };
 
 // Shared memory of one slot's activation digits, scales and 16-column sums.
-static size_t slot_bytes(int batch, int nsbs) {
-  const int nt = (batch + 3) / 4;
-  return (size_t)2 * batch * (256 * nsbs + 16) + (size_t)36 * 4 * nt * (2 * nsbs);
-}
+static size_t slot_bytes(int batch, int nsbs) { return (size_t)slot_area(batch, (batch + 3) / 4, 2 * nsbs); }
 
 // Widest column slice (in super-blocks) whose digits fit in one slot.
 static int max_sb_fit(int batch) {
-  const int nt = (batch + 3) / 4;
-  const long avail = (long)kDigitBudget - 32L * batch;
-  return (int)std::max(1L, avail / (512L * batch + 288L * nt));
+  int s = 1;
+  while (slot_bytes(batch, s + 1) <= (size_t)kDigitBudget) ++s;
+  return s;
 }
 
 // Column split for a single tensor: enough units to fill the GPU, slices of whole

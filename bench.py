@@ -36,7 +36,8 @@ sys.path.insert(0, ROOT)
 METRIC = "weight-bytes GB/s and fraction of HBM peak at batch 1; decode-step tokens/s"
 ESC_RATE = 0.16
 WORKLOAD = ("qwen3-0.6b-shaped decode step: 197 GEMVs (28 layers x q,k,v,o,gate,up,down + tied head "
-            "1024x151936) read at D4 from the plane store, logit gate over 151936 logits, seeded 16% of steps "
+            "1024x151936) read at D4 from the plane store, logit gate over 151936 logits fused into the same launch, "
+            "seeded 16% of steps "
             "escalate D4->D8 via residual planes + gate; batch 1")
 
 
@@ -217,29 +218,27 @@ class DecodeStep:
         self.prob_d4 = fl.gemv_problems(items)
         self.prob_res = fl.gemv_problems(items_r)
         self.n = len(items)
-        # gate outputs (one buffer so one device->host copy reads the step's result)
+        # gate outputs (one buffer so one device->host copy reads the step's result); the gate
+        # runs fused into the batched GEMV over the head's outputs (problem n - 1)
         self.gate = torch.zeros(8, dtype=torch.int32, device="cuda")
         self.tau_h, self.tau_m = 11.8, 1e-6
+        wsb = fl.fl_gemv_gate_workspace_bytes(1)
+        self.gate_ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+        g = self.gate
+        self.spec = fl.gate_spec(self.n - 1, self.tau_h, self.tau_m, g[0:1].view(torch.float32),
+                                 g[1:2].view(torch.float32), g[2:4], g[4:5].view(torch.uint8)[0:1], self.gate_ws, wsb)
         gx = synth.bf16_normal((tot_in,), seed, 99)
         self.x.copy_(torch.from_numpy(gx.view("int16")))
 
-    def _gate(self):
-        fl, g = self.fl, self.gate
-        ent, mar = g[0:1].view(self.torch.float32), g[1:2].view(self.torch.float32)
-        top2 = g[2:4]
-        esc = g[4:5].view(self.torch.uint8)[0:1]
-        fl.fl_logit_gate(self.head_logits, self.vocab, 1, self.tau_h, self.tau_m, ent, mar, top2, esc)
-
     def low_pass(self):
-        self.fl.fl_gemv_batched(self.prob_d4, self.n, 1, 0)
-        self._gate()
+        self.fl.fl_gemv_batched_gate(self.prob_d4, self.n, 1, 0, self.spec)
 
     def escalate(self):
-        self.fl.fl_gemv_batched(self.prob_res, self.n, 1, 1)
-        self._gate()
+        self.fl.fl_gemv_batched_gate(self.prob_res, self.n, 1, 1, self.spec)
 
     def gemv_only(self):
-        self.fl.fl_gemv_batched(self.prob_d4, self.n, 1, 0)
+        # the step's dominant kernel as the step runs it (D4 pass, gate fused)
+        self.fl.fl_gemv_batched_gate(self.prob_d4, self.n, 1, 0, self.spec)
 
     def capture(self):
         torch = self.torch
@@ -556,7 +555,7 @@ def run_fl(args, rank, world, local_rank):
         "tokens_per_s": tok_s, "hbm_frac": value / world / peak, "peak_gbs": peak, "peak_kind": peak_kind,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": tr["bytes_per_launch"] if tr else None,
-                     "kernel": "plane_gemv_kernel (fl_gemv_batched, 197 problems, D4)",
+                     "kernel": "plane_gemv_kernel (fl_gemv_batched_gate, 197 problems, D4, logit gate fused)",
                      "us_per_launch": tk * 1e6, "bytes_per_launch": step.bytes_d4,
                      # plane GEMV launches per step (the D4 pass plus the escalated steps' residual
                      # pass, both full reads of the store) x time per launch / step time
@@ -565,7 +564,7 @@ def run_fl(args, rank, world, local_rank):
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": step.h2d_bytes,
                 "d2h_bytes_per_step": 32, "steps": e2e_steps,
                 "tokens_per_s": world * e2e_steps / te},
-        "gpu_launches": 2 * args.steps + 2 * n_esc,
+        "gpu_launches": args.steps + n_esc,
         "clocks": clk.summary(),
         "kernels": extra,
     }

@@ -217,6 +217,35 @@ typedef struct {
 
 FL_API fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream);
 
+/* fl_gemv_batched with the logit gate fused in ([PoD] abstract: the gate reads the
+ * distribution the low-precision step produced). Problem `problem`'s outputs y[t][0..out)
+ * are the logits of batch row t; as its blocks are produced, each CTA folds them into
+ * entropy / top-2 partials, and the last CTA to finish merges them and writes
+ * entropy / margin / top2 / escalate exactly as fl_logit_gate defines them (equal up to
+ * fp32 summation order). In mode 1 the gate reads the updated y. y is written as by
+ * fl_gemv_batched. No counterpart of the separate launch is needed.
+ * entropy, margin  device, fp32 [batch]      top2  device, int32 [batch][2]
+ * escalate         device, uint8 [batch]
+ * workspace        device, >= fl_gemv_gate_workspace_bytes(batch) bytes, 16-byte
+ *                  aligned, ZERO-FILLED before first use; every completed launch leaves
+ *                  its counter at zero. Launches sharing a workspace must not overlap. */
+typedef struct {
+  int problem;
+  float tau_h;
+  float tau_m;
+  float* entropy;
+  float* margin;
+  int32_t* top2;
+  uint8_t* escalate;
+  void* workspace;
+  size_t workspace_bytes;
+} fl_gate_spec;
+
+FL_API size_t fl_gemv_gate_workspace_bytes(int batch);
+
+FL_API fl_status fl_gemv_batched_gate(const fl_gemv_problem* problems, int n, int batch, int mode,
+                               const fl_gate_spec* gate, void* stream);
+
 /* ========================================================================= */
 /* Uncertainty gate ([PoD]: redo at 8 bits when the low-precision output     */
 /* distribution looks uncertain: entropy above a threshold or a small        */

@@ -223,6 +223,59 @@ def test_batched_problems(env, orc):
         check_close(y.cpu().numpy(), yref, mass, f"batched {o}x{n}")
 
 
+@pytest.mark.parametrize("batch,gate_index", [(1, 3), (3, 1)])
+def test_batched_gate_fused(env, orc, batch, gate_index):
+    """Gate fused into the batched GEMV: y as the oracle, gate outputs as the oracle's gate on
+    the GPU's own logits, for the depth pass and then the residual pass to D8."""
+    torch, fl = env
+    shapes = [(1024, 1024), (8192, 1024), (2048, 2048), (1024, 3072)]
+    items, layers, keep = [], [], []
+    for i, (o, n) in enumerate(shapes):
+        q, s = synth.int8_layer(o, n, 91, i)
+        lv = synth.seeded_levels(o // 64, 92, i)     # the logits include ZERO and D8 blocks
+        x = synth.bf16_normal((batch, n), 93, i)
+        st = pack_gpu(torch, fl, q, s)
+        y = torch.zeros((batch, o), dtype=torch.float32, device="cuda")
+        lvd, xd, to = dev(torch, lv), dev(torch, x), torch.full((o // 64,), 4, dtype=torch.uint8, device="cuda")
+        keep += [st, lvd, xd, y, to]
+        items.append((st, o, n, lvd, to, xd, y))
+        layers.append((q, s, lv, x))
+    arr = fl.gemv_problems(items)
+    V = shapes[gate_index][0]
+    wsb = fl.fl_gemv_gate_workspace_bytes(batch)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    e = torch.empty(batch, dtype=torch.float32, device="cuda")
+    m = torch.empty(batch, dtype=torch.float32, device="cuda")
+    t2 = torch.empty((batch, 2), dtype=torch.int32, device="cuda")
+    es = torch.empty(batch, dtype=torch.uint8, device="cuda")
+    for mode in (0, 1):
+        tau_h, tau_m = 8.5, 1e-4
+        spec = fl.gate_spec(gate_index, tau_h, tau_m, e, m, t2, es, ws, wsb)
+        fl.fl_gemv_batched_gate(arr, len(items), batch, mode, spec)
+        torch.cuda.synchronize()
+        for i, ((q, s, lv, x), it) in enumerate(zip(layers, items)):
+            to_lv = np.full_like(lv, 4) if mode == 1 else lv
+            yref, mass = orc.gemv_depth(q, s, to_lv, x, with_mass=True)
+            check_close(it[6].cpu().numpy(), yref, mass, f"fused-gate batch mode {mode} problem {i}")
+        z = items[gate_index][6].cpu().numpy()
+        H, M, top2, esc = orc.logit_gate(z, tau_h, tau_m)
+        ge, gm, gt, gs = e.cpu().numpy(), m.cpu().numpy(), t2.cpu().numpy(), es.cpu().numpy()
+        assert np.array_equal(gt, top2), (mode, gt, top2)
+        assert np.allclose(ge, H, rtol=1e-5, atol=1e-6), (mode, ge, H)
+        assert np.allclose(gm, M, rtol=1e-5, atol=1e-7), (mode, gm, M)
+        band = (np.abs(H - tau_h) <= 1e-4 * abs(tau_h) + 1e-6) | (np.abs(M - tau_m) <= 1e-6)
+        assert np.array_equal(gs[~band], esc[~band])
+        assert np.array_equal(gs, ((ge > np.float32(tau_h)) | (gm < np.float32(tau_m))).astype(np.uint8))
+        assert int(ws[:4].view(torch.int32).item()) == 0, "gate counter not left at zero"
+        # the standalone gate over the same logits agrees
+        e2, m2 = torch.empty_like(e), torch.empty_like(m)
+        t22, es2 = torch.empty_like(t2), torch.empty_like(es)
+        fl.fl_logit_gate(items[gate_index][6], V, batch, tau_h, tau_m, e2, m2, t22, es2)
+        torch.cuda.synchronize()
+        assert np.array_equal(t22.cpu().numpy(), gt)
+        assert np.allclose(e2.cpu().numpy(), ge, rtol=1e-5, atol=1e-6)
+
+
 # ----------------------------------------------------------------------------- level map
 
 def test_level_map_bit_exact(env, orc, golden):

@@ -37,6 +37,7 @@
 #include <vector>
 
 #include "fl_common.cuh"
+#include "fl_gate_merge.cuh"
 
 namespace fl {
 namespace gemv {
@@ -83,6 +84,16 @@ struct Args {
   int ncta;
   int cta_begin[kMaxCtas + 1];
   int cta_slice[kMaxCtas];  // first (problem, slice) pair of the CTA, counted in order, << 7 | pairs touched
+  // fused logit gate over problem gate_p's outputs (gate_p < 0: none)
+  int gate_p;
+  float tau_h, tau_m;
+  float* entropy;
+  float* margin;
+  int32_t* top2;
+  uint8_t* escalate;
+  uint32_t* gate_ticket;   // launch counter, zero between launches
+  GateRec* gate_part;      // [kMaxCtas][FL_MAX_BATCH] per-CTA partials
+  int gate_cta0, gate_ncta;  // the CTAs whose unit ranges hold gate-problem units
   Problem p[MAXP];
 };
 
@@ -121,7 +132,7 @@ __host__ __device__ constexpr uint32_t plane_mask(int k, int i) {
 }
 
 // Named barriers: 0 is __syncthreads; team t uses kBarTeam0 + t.
-enum : int { kBarTeam0 = 2, kBarProducers = 6, kBarLevels = 7 };
+enum : int { kBarGate = 1, kBarTeam0 = 2, kBarProducers = 6, kBarLevels = 7 };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -348,6 +359,131 @@ __device__ __forceinline__ void dispatch_tile(int k0, int np, uint32_t stage, in
 #undef FL_TILE
 }
 
+// ---------------------------------------------------------------- fused logit gate
+// Per consumer warp and batch row, a running partial (in dynamic shared memory at gw) over
+// the gate problem's outputs this warp produced; merged per CTA by the last warp to finish,
+// per launch by the last CTA to finish (atomic counters, no waiting).
+
+__device__ __forceinline__ GateRec ldcg_rec(const GateRec* p) {
+  const float4 u = __ldcg(reinterpret_cast<const float4*>(p));
+  const int4 w = __ldcg(reinterpret_cast<const int4*>(p) + 1);
+  GateRec r;
+  r.m = u.x;
+  r.S = u.y;
+  r.T = u.z;
+  r.v2 = u.w;
+  r.i1 = w.x;
+  r.i2 = w.y;
+  r.pad0 = r.pad1 = 0;
+  return r;
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Warp 0 publishes the CTA's partials (lane bb holds batch row bb's): lane 0 stores them and
+// takes the launch counter with one acquire-release atomic; the last CTA merges every CTA's
+// partials in CTA order and writes the gate outputs.
+template <int MAXP>
+__device__ __forceinline__ void gate_publish(const Args<MAXP>& a, const GateRec& mine, int lane) {
+  GateRec* part = a.gate_part + (size_t)(blockIdx.x - a.gate_cta0) * FL_MAX_BATCH;
+  int last = 0;
+  for (int bb = 0; bb < a.batch; ++bb) {
+    GateRec r;
+    r.m = __shfl_sync(0xffffffffu, mine.m, bb);
+    r.S = __shfl_sync(0xffffffffu, mine.S, bb);
+    r.T = __shfl_sync(0xffffffffu, mine.T, bb);
+    r.v2 = __shfl_sync(0xffffffffu, mine.v2, bb);
+    r.i1 = __shfl_sync(0xffffffffu, mine.i1, bb);
+    r.i2 = __shfl_sync(0xffffffffu, mine.i2, bb);
+    r.pad0 = r.pad1 = 0;
+    if (lane == 0) part[bb] = r;
+  }
+  if (lane == 0) last = (atom_add_acq_rel(a.gate_ticket, 1u) == (uint32_t)(a.gate_ncta - 1));
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  for (int bb = 0; bb < a.batch; ++bb) {
+    // lane 0 acquired the counter; the others' loads are ordered after it by the warp sync
+    __syncwarp();
+    GateRec r = empty_rec();
+    for (int c = lane; c < a.gate_ncta; c += 32) r = merge2(r, ldcg_rec(&a.gate_part[(size_t)c * FL_MAX_BATCH + bb]));
+    r = warp_merge(r);
+    if (lane == 0)
+      gate_outputs(r, a.tau_h, a.tau_m, a.entropy + bb, a.margin + bb, a.top2 + 2 * bb, a.escalate + bb);
+  }
+  if (lane == 0) *a.gate_ticket = 0u;
+}
+
+// All consumer threads of a CTA that holds gate-problem units, after the CTA's outputs are
+// written: the CTA's rows of that problem are one contiguous range [r0, r1) (still in L2).
+// Every thread loads its strided share (up to kGateLoads values per batch row at once), takes
+// the top-2 and S, T relative to its own max; warps merge (redux / shuffles), then warp 0
+// merges the warps (one lane per warp) and publishes. gws: [kConsumerWarps][batch] in smem.
+constexpr int kGateLoads = 8;
+template <int MAXP>
+__device__ __forceinline__ void gate_cta_reduce(const Args<MAXP>& a, const float* y, size_t ystride, int r0, int r1,
+                                                GateRec* gws, int tid, int warp, int lane) {
+  for (int bb = 0; bb < a.batch; ++bb) {
+    const float* yr = y + (size_t)bb * ystride;
+    GateRec r = empty_rec();
+    for (int base = r0 + tid; base < r1; base += kGateLoads * kConsumers) {
+      float v[kGateLoads];
+#pragma unroll
+      for (int j = 0; j < kGateLoads; ++j) {
+        const int k = base + j * kConsumers;
+        v[j] = (k < r1) ? __ldcg(yr + k) : -INFINITY;
+      }
+      GateRec q = empty_rec();
+      float a1 = -INFINITY, a2 = -INFINITY;
+      int j1 = 0x7fffffff, j2 = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < kGateLoads; ++j) {
+        const int k = base + j * kConsumers;
+        if (k < r1 && better(v[j], k, a2, j2)) {
+          if (better(v[j], k, a1, j1)) {
+            a2 = a1;
+            j2 = j1;
+            a1 = v[j];
+            j1 = k;
+          } else {
+            a2 = v[j];
+            j2 = k;
+          }
+        }
+      }
+      q.m = a1;
+      q.i1 = j1;
+      q.v2 = a2;
+      q.i2 = j2;
+      float S = 0.f, T = 0.f;
+#pragma unroll
+      for (int j = 0; j < kGateLoads; ++j) {
+        if (base + j * kConsumers < r1) {
+          const float d = v[j] - a1, e = __expf(d);
+          S += e;
+          T = fmaf(d, e, T);
+        }
+      }
+      q.S = S;
+      q.T = T;
+      r = merge2(r, q);
+    }
+    r = warp_merge(r);
+    if (lane == 0) gws[warp * a.batch + bb] = r;
+  }
+  named_bar(kBarGate, kConsumers);
+  if (warp != 0) return;
+  GateRec mine = empty_rec();
+  for (int bb = 0; bb < a.batch; ++bb) {
+    const GateRec r = warp_merge(lane < kConsumerWarps ? gws[lane * a.batch + bb] : empty_rec());
+    if (lane == bb) mine = r;
+  }
+  gate_publish(a, mine, lane);
+}
+
 // Plane range [k0, k0 + np) read for block b, packed as k0 << 4 | np.
 __device__ __forceinline__ int plane_range(int mode, const uint8_t* lv_from, const uint8_t* lv_to, int b) {
   const int lf = min((int)__ldg(lv_from + b), 4);
@@ -356,7 +492,9 @@ __device__ __forceinline__ int plane_range(int mode, const uint8_t* lv_from, con
   return (lf << 4) | max(0, lt - lf);
 }
 
-template <int MAXP, int NT>
+// GATE: the logit gate is fused over problem a.gate_p's outputs (a separate instantiation,
+// so the lane partials cost the plain kernel no registers).
+template <int MAXP, int NT, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
@@ -365,11 +503,16 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   __shared__ __align__(16) uint8_t zeros[160];
   __shared__ int s_ticket[kTeams];
   __shared__ int s_nslots;
+  __shared__ int s_failed;  // a consumer warp gave up waiting for a stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u_begin = a.cta_begin[blockIdx.x], u_end = a.cta_begin[blockIdx.x + 1];
   if (u_begin >= u_end) return;
   const int nunits = u_end - u_begin;
+  // fused gate: this CTA holds gate-problem units; per consumer warp and batch row, its
+  // partials (end of dynamic smem)
+  const bool gate_cta = GATE && (int)blockIdx.x >= a.gate_cta0 && (int)blockIdx.x < a.gate_cta0 + a.gate_ncta;
+  GateRec* const gws = reinterpret_cast<GateRec*>(smem + kSmemLimit - kConsumerWarps * a.batch * sizeof(GateRec));
 
   if (threadIdx.x < 40) reinterpret_cast<uint32_t*>(zeros)[threadIdx.x] = 0u;
   if (threadIdx.x == 0) {
@@ -378,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       mbar_init(&empty_bar[s], kTeamWarps);
     }
     fence_mbar_init();
+    s_failed = 0;
   }
   if (warp == 0) {
     // Slot table: lane i fills slot i, the i-th (problem, slice) pair from the CTA's first one
@@ -518,6 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   const uint32_t smem_base = smem_u32(smem);
   uint32_t dlane[NT], dstep[NT], gc_lane = 0;
   int cur_slot = -1, si = 0, used = 0;
+  bool failed = false;
   for (int k = team; k < nunits; k += kTeams) {
     while (si + 1 < nsl && k >= slots[si].u1) ++si;
     const Slot& sl = slots[si];
@@ -561,8 +706,12 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       const int tg = min(tgm, sl.ngroups - g0);
       const int s = kTeamStages * team + (used % kTeamStages);
       if (!mbar_wait(&full_bar[s], (uint32_t)((used / kTeamStages) & 1))) {
-        if (lane == 0) atomicExch(&g_error, 2);
-        return;
+        if (lane == 0) {
+          atomicExch(&g_error, 2);
+          s_failed = 1;
+        }
+        failed = true;
+        break;
       }
       dispatch_tile<NT>(k0, np, smem_base + s * kStageBytes, tg, dlane, dstep, gc_lane, gstride, g0, cfac, r0, t,
                         acc);
@@ -570,6 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       if (lane == 0) mbar_arrive(&empty_bar[s]);
       ++used;
     }
+    if (failed) break;  // a stage never filled: stop, but still reach the CTA's last barrier
 
     // ---- unit done: this warp's 16 rows are final (or a slice partial)
     if (sl.slices == 1) {
@@ -578,13 +728,12 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         const int bb = 4 * nt + t;
         if (bb < a.batch) {
           float* y0 = y + (size_t)bb * ystride + row_base + g;
-          if (a.mode == 0) {
-            y0[0] = acc[nt][0];
-            y0[8] = acc[nt][1];
-          } else {
-            y0[0] += acc[nt][0];
-            y0[8] += acc[nt][1];
+          if (a.mode == 1) {
+            acc[nt][0] += y0[0];
+            acc[nt][1] += y0[8];
           }
+          y0[0] = acc[nt][0];
+          y0[8] = acc[nt][1];
         }
       }
     } else {
@@ -620,6 +769,17 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       named_bar(kBarTeam0 + team, kTeamThreads);
     }
   }
+  if constexpr (GATE) {
+    if (gate_cta) {
+      // every consumer warp has written its outputs (this barrier also orders them)
+      named_bar(kBarGate, kConsumers);
+      if (s_failed) return;
+      const Problem& P = a.p[a.gate_p];
+      const int b0 = max(u_begin, P.unit_begin) - P.unit_begin;
+      const int b1 = min(u_end, P.unit_begin + P.nblocks) - P.unit_begin;
+      gate_cta_reduce(a, P.y, (size_t)64 * P.nblocks, 64 * b0, 64 * b1, gws, threadIdx.x, warp, lane);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -634,9 +794,9 @@ static size_t slot_bytes(int batch, int ngroups) {
 }
 
 // Widest column slice (in 128-column groups) whose digits fit in one slot.
-static int max_groups_fit(int batch) {
+static int max_groups_fit(int batch, long budget = kDigitBudget) {
   const int nt = (batch + 3) / 4;
-  const long avail = (long)kDigitBudget - 32L * batch;
+  const long avail = budget - 32L * batch;
   return (int)std::max(1L, avail / (256L * batch + 32L * nt));
 }
 
@@ -665,7 +825,7 @@ static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
 // memory, at kMaxSlots pairs, or at the level-cache size; such cuts can make more ranges than
 // SMs (a second, partial wave).
 template <int MAXP>
-static bool partition(Args<MAXP>& a, int nsm) {
+static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
   double total = 0;
   for (int i = 0; i < a.nproblems; ++i) total += (double)a.p[i].nblocks * a.p[i].G;
   const Problem& L = a.p[a.nproblems - 1];
@@ -689,7 +849,7 @@ static bool partition(Args<MAXP>& a, int nsm) {
         bool cut = false;
         if (count > 0) {
           if (n + 1 < target && acc + 0.5 * cost > per_cta * (n + 1)) cut = true;
-          if (b == 0 && (dig + sb > (size_t)kDigitBudget || nslots == kMaxSlots)) cut = true;
+          if (b == 0 && (dig + sb > budget || nslots == kMaxSlots)) cut = true;
           if (count == kLevelCache) cut = true;
         }
         if (cut) {
@@ -716,10 +876,10 @@ static bool partition(Args<MAXP>& a, int nsm) {
   return true;
 }
 
-template <int MAXP, int NT>
+template <int MAXP, int NT, bool GATE>
 static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
   const size_t smem = (size_t)kSmemLimit;
-  auto kern = plane_gemv_kernel<MAXP, NT>;
+  auto kern = plane_gemv_kernel<MAXP, NT, GATE>;
   FL_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                 "cudaFuncSetAttribute(plane_gemv)");
   kern<<<a.ncta, kThreads, smem, st>>>(a);
@@ -727,13 +887,22 @@ static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
   return FL_OK;
 }
 
+static fl_status launch_nt_gate(const Args<FL_MAX_PROBLEMS>& a, cudaStream_t st) {
+  switch ((a.batch + 3) / 4) {
+    case 1: return launch<FL_MAX_PROBLEMS, 1, true>(a, st);
+    case 2: return launch<FL_MAX_PROBLEMS, 2, true>(a, st);
+    case 3: return launch<FL_MAX_PROBLEMS, 3, true>(a, st);
+    default: return launch<FL_MAX_PROBLEMS, 4, true>(a, st);
+  }
+}
+
 template <int MAXP>
 static fl_status launch_nt(const Args<MAXP>& a, cudaStream_t st) {
   switch ((a.batch + 3) / 4) {
-    case 1: return launch<MAXP, 1>(a, st);
-    case 2: return launch<MAXP, 2>(a, st);
-    case 3: return launch<MAXP, 3>(a, st);
-    default: return launch<MAXP, 4>(a, st);
+    case 1: return launch<MAXP, 1, false>(a, st);
+    case 2: return launch<MAXP, 2, false>(a, st);
+    case 3: return launch<MAXP, 3, false>(a, st);
+    default: return launch<MAXP, 4, false>(a, st);
   }
 }
 
@@ -766,6 +935,7 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   a.nproblems = 1;
   a.batch = batch;
   a.mode = mode;
+  a.gate_p = -1;
   Problem& P = a.p[0];
   P.store = w->store;
   P.lv_from = lv_from;
@@ -814,29 +984,57 @@ extern "C" fl_status fl_gemv_residual(const fl_plane_weight* w, const uint8_t* f
                       "fl_gemv_residual");
 }
 
-extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream) {
-  const char* what = "fl_gemv_batched";
+namespace fl {
+namespace gemv {
+
+constexpr size_t kGateTicketBytes = 256;
+constexpr size_t kGateWorkspaceBytes = kGateTicketBytes + (size_t)kMaxCtas * FL_MAX_BATCH * sizeof(GateRec);
+
+static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int mode, const fl_gate_spec* gate,
+                         void* stream, const char* what) {
   if (!problems) return fail(FL_ERR_ARG, "%s: problems is NULL", what);
   if (n < 1 || n > FL_MAX_PROBLEMS) return fail(FL_ERR_ARG, "%s: n=%d (1..%d)", what, n, FL_MAX_PROBLEMS);
   if (mode != 0 && mode != 1) return fail(FL_ERR_ARG, "%s: mode=%d (0 depth, 1 residual)", what, mode);
   if (batch < 1 || batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..16)", what, batch);
-  static thread_local gemv::Args<FL_MAX_PROBLEMS> a;
+  static thread_local Args<FL_MAX_PROBLEMS> a;
   a.nproblems = n;
   a.batch = batch;
   a.mode = mode;
+  a.gate_p = -1;
+  size_t budget = kDigitBudget;
+  if (gate) {
+    if (gate->problem < 0 || gate->problem >= n)
+      return fail(FL_ERR_ARG, "%s: gate problem %d not in 0..%d", what, gate->problem, n - 1);
+    if (!gate->entropy || !gate->margin || !gate->top2 || !gate->escalate || !gate->workspace)
+      return fail(FL_ERR_ARG, "%s: gate output or workspace pointer is NULL", what);
+    if (gate->workspace_bytes < kGateWorkspaceBytes)
+      return fail(FL_ERR_WORKSPACE, "%s: gate workspace %zu bytes, need %zu", what, gate->workspace_bytes,
+                  kGateWorkspaceBytes);
+    if (!aligned16(gate->workspace)) return fail(FL_ERR_ALIGN, "%s: gate workspace not 16-byte aligned", what);
+    a.gate_p = gate->problem;
+    a.tau_h = gate->tau_h;
+    a.tau_m = gate->tau_m;
+    a.entropy = gate->entropy;
+    a.margin = gate->margin;
+    a.top2 = gate->top2;
+    a.escalate = gate->escalate;
+    a.gate_ticket = static_cast<uint32_t*>(gate->workspace);
+    a.gate_part = reinterpret_cast<GateRec*>(static_cast<uint8_t*>(gate->workspace) + kGateTicketBytes);
+    budget -= (size_t)kConsumerWarps * batch * sizeof(GateRec);
+  }
   int unit = 0;
   for (int i = 0; i < n; ++i) {
     const fl_gemv_problem& q = problems[i];
-    fl_status st = gemv::check_weight(&q.w, what);
+    fl_status st = check_weight(&q.w, what);
     if (st != FL_OK) return st;
     if (!q.levels || !q.x || !q.y || (mode == 1 && !q.to_levels))
       return fail(FL_ERR_ARG, "%s: problem %d has a NULL pointer", what, i);
     if (!aligned16(q.x)) return fail(FL_ERR_ALIGN, "%s: problem %d x not 16-byte aligned", what, i);
     const int G = q.w.in / 128;
-    if (G > gemv::max_groups_fit(batch))
+    if (G > max_groups_fit(batch, (long)budget))
       return fail(FL_ERR_SHAPE, "%s: problem %d in=%d too wide for batch %d in one launch (in <= %d)", what, i,
-                  q.w.in, batch, 128 * gemv::max_groups_fit(batch));
-    gemv::Problem& P = a.p[i];
+                  q.w.in, batch, 128 * max_groups_fit(batch, (long)budget));
+    Problem& P = a.p[i];
     P.store = q.w.store;
     P.lv_from = q.levels;
     P.lv_to = q.to_levels;
@@ -853,8 +1051,37 @@ extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int
   }
   const int nsm = device_sm_count();
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
-  if (!gemv::partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: problems too large for one launch", what);
-  return gemv::launch_nt(a, static_cast<cudaStream_t>(stream));
+  if (!partition(a, nsm, budget)) return fail(FL_ERR_SHAPE, "%s: problems too large for one launch", what);
+  if (gate) {
+    const int ub = a.p[a.gate_p].unit_begin, ue = ub + a.p[a.gate_p].nblocks;
+    a.gate_cta0 = -1;
+    a.gate_ncta = 0;
+    for (int c = 0; c < a.ncta; ++c)
+      if (a.cta_begin[c] < ue && a.cta_begin[c + 1] > ub) {
+        if (a.gate_cta0 < 0) a.gate_cta0 = c;
+        ++a.gate_ncta;
+      }
+    return launch_nt_gate(a, static_cast<cudaStream_t>(stream));
+  }
+  return launch_nt(a, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace gemv
+}  // namespace fl
+
+extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream) {
+  return gemv::batched(problems, n, batch, mode, nullptr, stream, "fl_gemv_batched");
+}
+
+extern "C" size_t fl_gemv_gate_workspace_bytes(int batch) {
+  if (batch < 1 || batch > FL_MAX_BATCH) return 0;
+  return gemv::kGateWorkspaceBytes;
+}
+
+extern "C" fl_status fl_gemv_batched_gate(const fl_gemv_problem* problems, int n, int batch, int mode,
+                                          const fl_gate_spec* gate, void* stream) {
+  if (!gate) return fail(FL_ERR_ARG, "fl_gemv_batched_gate: gate spec is NULL");
+  return gemv::batched(problems, n, batch, mode, gate, stream, "fl_gemv_batched_gate");
 }
 
 // ---------------------------------------------------------------- allocation-free variant

@@ -50,6 +50,12 @@ class fl_gemv_problem(C.Structure):
                 ("y", C.c_void_p)]
 
 
+class fl_gate_spec(C.Structure):
+    _fields_ = [("problem", C.c_int), ("tau_h", C.c_float), ("tau_m", C.c_float), ("entropy", C.c_void_p),
+                ("margin", C.c_void_p), ("top2", C.c_void_p), ("escalate", C.c_void_p), ("workspace", C.c_void_p),
+                ("workspace_bytes", C.c_size_t)]
+
+
 class fl_kquant_problem(C.Structure):
     _fields_ = [("blocks", C.c_void_p), ("ggml_type", C.c_int), ("out", C.c_int), ("in_", C.c_int),
                 ("x", C.c_void_p), ("y", C.c_void_p)]
@@ -68,6 +74,8 @@ _sigs = {
     "fl_gemv_depth_static": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P]),
     "fl_gemv_residual": (_I, [C.POINTER(fl_plane_weight), _P, _P, _P, _I, _P, _P, _S, _P]),
     "fl_gemv_batched": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, _P]),
+    "fl_gemv_gate_workspace_bytes": (_S, [_I]),
+    "fl_gemv_batched_gate": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, C.POINTER(fl_gate_spec), _P]),
     "fl_logit_gate": (_I, [_P, _I, _I, _F, _F, _P, _P, _P, _P, _P]),
     "fl_kquant_bytes": (_S, [_I, _I, _I]),
     "fl_kquant_workspace_bytes": (_S, [_I, _I, _I, _I]),
@@ -175,6 +183,20 @@ def gemv_problems(items) -> "C.Array":
 
 def fl_gemv_batched(problems, n: int, batch: int, mode: int, stream=None) -> None:
     _check(_lib.fl_gemv_batched(problems, n, batch, mode, _stream(stream)))
+
+
+def fl_gemv_gate_workspace_bytes(batch: int) -> int:
+    return int(_lib.fl_gemv_gate_workspace_bytes(batch))
+
+
+def gate_spec(problem: int, tau_h: float, tau_m: float, entropy, margin, top2, escalate, workspace,
+              workspace_bytes: int) -> fl_gate_spec:
+    return fl_gate_spec(problem, float(tau_h), float(tau_m), _ptr(entropy), _ptr(margin), _ptr(top2), _ptr(escalate),
+                        _ptr(workspace), workspace_bytes)
+
+
+def fl_gemv_batched_gate(problems, n: int, batch: int, mode: int, gate: fl_gate_spec, stream=None) -> None:
+    _check(_lib.fl_gemv_batched_gate(problems, n, batch, mode, C.byref(gate), _stream(stream)))
 
 
 def fl_logit_gate(logits, vocab: int, batch: int, tau_h: float, tau_m: float, entropy, margin, top2, escalate,

@@ -747,12 +747,12 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
           pp[8] = acc[nt][1];
         }
       }
-      __threadfence();
+      // The barrier orders the team's partial stores before thread 0's acquire-release ticket
+      // (release is cumulative); the last team's reads follow the ticket's acquire.
       named_bar(kBarTeam0 + team, kTeamThreads);
-      if (tt == 0) s_ticket[team] = (int)atomicAdd(&sl.tickets[b], 1u);
+      if (tt == 0) s_ticket[team] = (int)atom_add_acq_rel(&sl.tickets[b], 1u);
       named_bar(kBarTeam0 + team, kTeamThreads);
       if (s_ticket[team] == sl.slices - 1) {
-        __threadfence();
         for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
           const int bb = e / 64, r = e % 64;
           float sum = 0.f;
@@ -823,11 +823,20 @@ static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
 // Contiguous cost-balanced unit ranges, one per CTA (cost ~ columns read). A range is also
 // closed early when the digits of its distinct (problem, slice) pairs would overflow shared
 // memory, at kMaxSlots pairs, or at the level-cache size; such cuts can make more ranges than
-// SMs (a second, partial wave).
+// SMs (a second, partial wave). The fused gate's epilogue (a reduction of the CTA's logits and
+// a publish, a few us) is charged to the gate problem's units, so the CTAs holding them get
+// fewer weight bytes.
+constexpr double kGateUnitWeight = 1.08;
+
+template <int MAXP>
+static double unit_weight(const Args<MAXP>& a, int i) {
+  return i == a.gate_p ? kGateUnitWeight : 1.0;
+}
+
 template <int MAXP>
 static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
   double total = 0;
-  for (int i = 0; i < a.nproblems; ++i) total += (double)a.p[i].nblocks * a.p[i].G;
+  for (int i = 0; i < a.nproblems; ++i) total += (double)a.p[i].nblocks * a.p[i].G * unit_weight(a, i);
   const Problem& L = a.p[a.nproblems - 1];
   const int units = L.unit_begin + L.nblocks * L.slices;
   const int target = std::max(1, std::min(nsm, units));
@@ -843,7 +852,7 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
     for (int j = 0; j < P.slices; ++j) {
       const int ng = std::min(P.slice_groups, P.G - j * P.slice_groups);
       const size_t sb = slot_bytes(a.batch, ng);
-      const double cost = (double)ng;
+      const double cost = (double)ng * unit_weight(a, i);
       for (int b = 0; b < P.nblocks; ++b) {
         const int u = P.unit_begin + j * P.nblocks + b;
         bool cut = false;

@@ -148,6 +148,12 @@ __device__ __forceinline__ int4 lds_s4(uint32_t a) {
 
 __device__ __forceinline__ int slice_nsb(const Problem& P, int j) { return min(P.slice_sb, P.nsb - j * P.slice_sb); }
 
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // A slot's digit area, batch rows padded to 4 NT. The padded strides spread the rows that
 // one warp reads together over distinct shared-memory banks.
 //   digits: 2 batch rows of digit_stride bytes (hi, lo)
@@ -640,12 +646,12 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
           pp[row1] = acc[nt][1];
         }
       }
-      __threadfence();
+      // The barrier orders the team's partial stores before thread 0's acquire-release ticket
+      // (release is cumulative); the last team's reads follow the ticket's acquire.
       named_bar(kBarTeam0 + team, kTeamThreads);
-      if (tt == 0) s_ticket[team] = (int)atomicAdd(&sl.tickets[b], 1u);
+      if (tt == 0) s_ticket[team] = (int)atom_add_acq_rel(&sl.tickets[b], 1u);
       named_bar(kBarTeam0 + team, kTeamThreads);
       if (s_ticket[team] == sl.slices - 1) {
-        __threadfence();
         for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
           const int bb = e / 64, r = e % 64;
           float sum = 0.f;

@@ -85,6 +85,16 @@ def test_host_side_rejections(fl):
     probs = fl.gemv_problems([(16, 64, 128, 16, None, 16, 16)])
     assert _status(fl, fl.fl_gemv_batched, probs, 0, 1, 0, s0) == ERR_ARG
     assert _status(fl, fl.fl_gemv_batched, probs, 1, 1, 2, s0) == ERR_ARG                  # mode
+    gsz = fl.fl_gemv_gate_workspace_bytes(1)
+    assert gsz > 0 and fl.fl_gemv_gate_workspace_bytes(0) == 0
+    spec = fl.gate_spec(1, 0.0, 0.0, 16, 16, 16, 16, 16, gsz)                  # problem 1 of 1
+    assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == ERR_ARG
+    spec = fl.gate_spec(0, 0.0, 0.0, 16, None, 16, 16, 16, gsz)                # NULL margin
+    assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == ERR_ARG
+    spec = fl.gate_spec(0, 0.0, 0.0, 16, 16, 16, 16, 16, gsz - 1)              # workspace too small
+    assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == -6
+    spec = fl.gate_spec(0, 0.0, 0.0, 16, 16, 16, 16, 17, gsz)                  # misaligned workspace
+    assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == -4
     kp = fl.kquant_problems([(16, 11, 64, 256, 16, 16)])
     assert _status(fl, fl.fl_gemv_kquant_batched, kp, 1, 1, s0) == ERR_UNSUP
     assert "Q4_K" in fl.fl_last_error()

@@ -827,6 +827,8 @@ static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
 // a publish, a few us) is charged to the gate problem's units, so the CTAs holding them get
 // fewer weight bytes.
 constexpr double kGateUnitWeight = 1.08;
+// A (problem, slice) pair's activation digits cost a CTA's prologue about as much as 7 groups.
+constexpr double kSlotCost = 7.0;
 
 template <int MAXP>
 static double unit_weight(const Args<MAXP>& a, int i) {
@@ -836,10 +838,15 @@ static double unit_weight(const Args<MAXP>& a, int i) {
 template <int MAXP>
 static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
   double total = 0;
-  for (int i = 0; i < a.nproblems; ++i) total += (double)a.p[i].nblocks * a.p[i].G * unit_weight(a, i);
+  int pairs = 0;
+  for (int i = 0; i < a.nproblems; ++i) {
+    total += (double)a.p[i].nblocks * a.p[i].G * unit_weight(a, i);
+    pairs += a.p[i].slices;
+  }
   const Problem& L = a.p[a.nproblems - 1];
   const int units = L.unit_begin + L.nblocks * L.slices;
   const int target = std::max(1, std::min(nsm, units));
+  total += kSlotCost * (pairs + target - 1);  // about one slot per pair plus one per cut
   const double per_cta = total / target;
   int n = 0;
   a.cta_begin[0] = 0;
@@ -873,6 +880,7 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
         if (b == 0 || count == 0) {
           dig += sb;
           ++nslots;
+          acc += kSlotCost;
         }
         acc += cost;
         ++count;

@@ -141,6 +141,22 @@ def traffic_record(kernel_key):
         return None
 
 
+def max_over_ranks(t, world, device="cuda"):
+    """The job's time: the slowest rank's (every rank calls this; one all-reduce)."""
+    if world <= 1:
+        return t
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([t], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_rate(units_per_rank, world, t):
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / t
+
+
 def escalation_schedule(steps, seed=1601):
     """Exactly 16 of every 100 steps escalate, positions drawn per block of 100 (seeded)."""
     import numpy as np
@@ -495,14 +511,10 @@ def run_fl(args, rank, world, local_rank):
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         t = time_loop(torch, body, args.steps)
-    if world > 1:
-        tt = torch.tensor([t], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
+    t = max_over_ranks(t, world)
     n_esc = int(sched[args.warmup:args.warmup + args.steps].sum())
-    bytes_job = world * (args.steps * step.bytes_d4 + n_esc * step.bytes_res)
-    value = bytes_job / t / 1e9
-    tok_s = world * args.steps / t
+    value = job_rate(args.steps * step.bytes_d4 + n_esc * step.bytes_res, world, t) / 1e9
+    tok_s = job_rate(args.steps, world, t)
 
     # dominant kernel alone: the batched D4 GEMV, graph-replayed back to back
     reps = max(200, args.steps // 10)
@@ -527,12 +539,9 @@ def run_fl(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     te = time_loop(torch, body_e2e, e2e_steps)
-    if world > 1:
-        tt = torch.tensor([te], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        te = float(tt.item())
+    te = max_over_ranks(te, world)
     n_esc_e = int(sched[args.warmup:args.warmup + e2e_steps].sum())
-    e2e_val = world * (e2e_steps * step.bytes_d4 + n_esc_e * step.bytes_res) / te / 1e9
+    e2e_val = job_rate(e2e_steps * step.bytes_d4 + n_esc_e * step.bytes_res, world, te) / 1e9
 
     extra = None
     if world == 1 and not args.no_extra:
@@ -563,7 +572,7 @@ def run_fl(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": step.h2d_bytes,
                 "d2h_bytes_per_step": 32, "steps": e2e_steps,
-                "tokens_per_s": world * e2e_steps / te},
+                "tokens_per_s": job_rate(e2e_steps, world, te)},
         "gpu_launches": args.steps + n_esc,
         "clocks": clk.summary(),
         "kernels": extra,

@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
   }
   // every thread arrives once; the other CTAs' senders wait on it before touching rank 0
   asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+  pdl_release();
+  pdl_wait();
 
   const float4* z4 = reinterpret_cast<const float4*>(logits + (size_t)row * vocab);
   const int n4 = vocab / 4;
@@ -123,20 +125,8 @@ namespace fl {
 template <int C, int T, int CACHE>
 static cudaError_t gate_launch_c(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,
                                  float* margin, int32_t* top2, uint8_t* escalate, cudaStream_t st) {
-  auto kern = logit_gate_kernel<C, T, CACHE>;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(batch * C));
-  cfg.blockDim = dim3(T);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = C;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, logits, vocab, tau_h, tau_m, entropy, margin, top2, escalate);
+  return launch_pdl(logit_gate_kernel<C, T, CACHE>, dim3((unsigned)(batch * C)), dim3(T), 0, st, C, logits, vocab,
+                    tau_h, tau_m, entropy, margin, top2, escalate);
 }
 
 // 16-CTA clusters where the device can place one (decided once per process), else 8.

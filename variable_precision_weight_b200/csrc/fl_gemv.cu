@@ -505,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   __shared__ int s_nslots;
   __shared__ int s_failed;  // a consumer warp gave up waiting for a stage
 
+  pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u_begin = a.cta_begin[blockIdx.x], u_end = a.cta_begin[blockIdx.x + 1];
   if (u_begin >= u_end) return;
@@ -587,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
     if (lane == 0) s_nslots = n;
   }
   __syncthreads();
+  pdl_wait();  // everything above read only the parameters
 
   // Before any weight copy is in flight (they would queue ahead of these small reads): the
   // producer threads read the level bytes into the level cache while the consumer threads read
@@ -899,8 +901,7 @@ static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
   auto kern = plane_gemv_kernel<MAXP, NT, GATE>;
   FL_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                 "cudaFuncSetAttribute(plane_gemv)");
-  kern<<<a.ncta, kThreads, smem, st>>>(a);
-  FL_CHECK_CUDA(cudaGetLastError(), "launch plane_gemv");
+  FL_CHECK_CUDA(launch_pdl(kern, dim3(a.ncta), dim3(kThreads), smem, st, 1, a), "launch plane_gemv");
   return FL_OK;
 }
 

@@ -456,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   __shared__ int s_ticket[kTeams];
   __shared__ int s_nslots;
 
+  pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u_begin = a.cta_begin[blockIdx.x], u_end = a.cta_begin[blockIdx.x + 1];
   if (u_begin >= u_end) return;
@@ -533,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
     if (lane == 0) s_nslots = n;
   }
   __syncthreads();
+  pdl_wait();  // everything above read only the parameters
 
   // Team t (producer warp t and consumer warps 4t..4t+3) walks units t, t + kTeams, ... of the
   // range; both sides derive the same tile sequence from the slot table, so the only hand-offs
@@ -762,8 +764,7 @@ static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
   auto kern = kquant_gemv_kernel<MAXP, NT>;
   FL_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                 "cudaFuncSetAttribute(kquant_gemv)");
-  kern<<<a.ncta, kThreads, smem, st>>>(a);
-  FL_CHECK_CUDA(cudaGetLastError(), "launch kquant_gemv");
+  FL_CHECK_CUDA(launch_pdl(kern, dim3(a.ncta), dim3(kThreads), smem, st, 1, a), "launch kquant_gemv");
   return FL_OK;
 }
 

@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(256) level_map_kernel(const float* __restrict_
                                                         uint8_t* __restrict__ levels, uint32_t* __restrict__ counts) {
   __shared__ float s_cx[64], s_cy[64], s_R[64];
   __shared__ uint32_t s_cnt[16];
+  pdl_release();
+  pdl_wait();
   if (threadIdx.x < 16) s_cnt[threadIdx.x] = 0;
   if (threadIdx.x < a.nlenses) {
     const float num = __fmul_rn(radii[threadIdx.x], a.f);
@@ -118,8 +120,8 @@ extern "C" fl_status fl_level_map(const float* xy, int nblocks, const float* cen
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
   int grid = (nblocks + 255) / 256;
   if (grid > nsm * 4) grid = nsm * 4;
-  level_map_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(xy, nblocks, centers, radii, a, levels,
-                                                                        counts);
-  FL_CHECK_CUDA(cudaGetLastError(), "launch level_map");
+  FL_CHECK_CUDA(launch_pdl(level_map_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), 1, xy,
+                           nblocks, centers, radii, a, levels, counts),
+                "launch level_map");
   return FL_OK;
 }

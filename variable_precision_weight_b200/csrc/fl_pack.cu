@@ -16,6 +16,8 @@ namespace fl {
 __global__ void __launch_bounds__(256) pack_planes_kernel(const int8_t* __restrict__ codes,
                                                           const float* __restrict__ scales, int out, int in,
                                                           uint8_t* __restrict__ store) {
+  pdl_release();
+  pdl_wait();
   const int G = in / 128;
   const long long words = (long long)out * (in / 16);
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < words;
@@ -66,7 +68,8 @@ extern "C" fl_status fl_pack_planes(const int8_t* codes, const float* scales, in
   const long long words = (long long)out * (in / 16);
   long long blocks = (words + 255) / 256;
   if (blocks > (long long)nsm * 16) blocks = (long long)nsm * 16;
-  pack_planes_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(codes, scales, out, in, store);
-  FL_CHECK_CUDA(cudaGetLastError(), "launch pack_planes");
+  FL_CHECK_CUDA(launch_pdl(pack_planes_kernel, dim3((unsigned)blocks), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                           1, codes, scales, out, in, store),
+                "launch pack_planes");
   return FL_OK;
 }

@@ -257,22 +257,12 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
   }
 }
 
-// One tile for one warp: all tg groups of the tile for rows r0 = 16 mt + g and r0 + 8.
-// Per group: plane words, activation digits, code bytes by mask/or/rotate, 4 k32 MMAs per
-// N-tile in two independent chains, then the group's scale and constant part in fp32.
-template <int K0, int NP, int NT, bool FULL>
-__device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const uint32_t (&dlane)[NT],
-                                             const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
-                                             int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
-  constexpr int TG = tile_groups(NP);
-  // A full tile has a compile-time group count, so the groups' loads and MMAs interleave freely.
-  const int tg = FULL ? TG : tg_arg;
-  const uint32_t planes = stage + 256u * tg;
-  const uint32_t wrow = planes + 32u * r0 + 8u * t;
-  const uint32_t srow = stage + 4u * r0;
-#pragma unroll
-  for (int gl = 0; gl < TG; ++gl) {
-    if (FULL || gl < tg) {
+// One group (128 columns) of a tile for one warp (rows r0 and r0 + 8): plane words, code bytes
+// by mask / or / rotate, 4 k32 MMAs per N-tile, then the group's scale and constant part.
+template <int K0, int NP, int NT>
+__device__ __forceinline__ void group_compute(uint32_t wrow, uint32_t srow, int tg, int gl, const uint32_t (&dlane)[NT],
+                                              const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
+                                              int slice_goff, float cfac, int t, float (&acc)[NT][2]) {
       const int gs = slice_goff + gl;
       uint2 W[NP][2];
 #pragma unroll
@@ -281,6 +271,44 @@ __device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const u
         W[kk][0] = lds_v2(pk);
         W[kk][1] = lds_v2(pk + 256u);
       }
+      const float s0 = lds_f32(srow + 256u * gl), s1 = lds_f32(srow + 256u * gl + 32u);
+      if constexpr (NT > 1) {
+        // Several N-tiles: build the group's four k-step A operands once, then one N-tile at a
+        // time (its fragment, four MMAs, its fold), which keeps the live registers per N-tile.
+        uint32_t u4[4][2][2];
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+          const int w = st >> 1;
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int i = 2 * (st & 1) + h;
+              uint32_t v = 0;
+#pragma unroll
+              for (int kk = 0; kk < NP; ++kk) v |= (w ? W[kk][r].y : W[kk][r].x) & plane_mask(K0 + kk, i);
+              u4[st][r][h] = (i == 0) ? v : rotr32(v, 2 * i);
+            }
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint32_t src = dlane[nt] + dstep[nt] * (uint32_t)gs;
+          const uint4 B0 = lds_v4(src), B1 = lds_v4(src + 16u);
+          int32_t C[4] = {0, 0, 0, 0}, D[4] = {0, 0, 0, 0};
+          mma_u8s8(C, u4[0][0][0], u4[0][1][0], u4[0][0][1], u4[0][1][1], B0.x, B0.y);
+          mma_u8s8(C, u4[1][0][0], u4[1][1][0], u4[1][0][1], u4[1][1][1], B0.z, B0.w);
+          mma_u8s8(D, u4[2][0][0], u4[2][1][0], u4[2][0][1], u4[2][1][1], B1.x, B1.y);
+          mma_u8s8(D, u4[3][0][0], u4[3][1][0], u4[3][0][1], u4[3][1][1], B1.z, B1.w);
+          const float2 hc = lds_f2(gc_lane + 8u * (uint32_t)(nt * 4 * gstride + gs));
+          const float off = cfac * hc.y;
+          const float v0 = fmaf((float)((C[0] + D[0]) * 256 + (C[1] + D[1])), hc.x, off);
+          const float v1 = fmaf((float)((C[2] + D[2]) * 256 + (C[3] + D[3])), hc.x, off);
+          acc[nt][0] = fmaf(v0, s0, acc[nt][0]);
+          acc[nt][1] = fmaf(v1, s1, acc[nt][1]);
+        }
+        return;
+      }
       uint4 B[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -288,7 +316,6 @@ __device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const u
         B[nt][0] = lds_v4(src);
         B[nt][1] = lds_v4(src + 16u);
       }
-      const float s0 = lds_f32(srow + 256u * gl), s1 = lds_f32(srow + 256u * gl + 32u);
       int32_t C[NT][4], D[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -330,7 +357,29 @@ __device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const u
         acc[nt][0] = fmaf(v0, s0, acc[nt][0]);
         acc[nt][1] = fmaf(v1, s1, acc[nt][1]);
       }
-    }
+}
+
+// One tile for one warp: all tg groups of the tile. At batch <= 4 a full tile runs with a
+// compile-time group count, so the groups' loads and MMAs interleave freely; with more
+// N-tiles the groups run one after the other, which keeps the registers in bounds.
+template <int K0, int NP, int NT, bool FULL>
+__device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const uint32_t (&dlane)[NT],
+                                             const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
+                                             int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
+  constexpr int TG = tile_groups(NP);
+  const int tg = FULL ? TG : tg_arg;
+  const uint32_t planes = stage + 256u * tg;
+  const uint32_t wrow = planes + 32u * r0 + 8u * t;
+  const uint32_t srow = stage + 4u * r0;
+  if constexpr (NT == 1) {
+#pragma unroll
+    for (int gl = 0; gl < TG; ++gl)
+      if (FULL || gl < tg)
+        group_compute<K0, NP, NT>(wrow, srow, tg, gl, dlane, dstep, gc_lane, gstride, slice_goff, cfac, t, acc);
+  } else {
+#pragma unroll 1
+    for (int gl = 0; gl < tg; ++gl)
+      group_compute<K0, NP, NT>(wrow, srow, tg, gl, dlane, dstep, gc_lane, gstride, slice_goff, cfac, t, acc);
   }
 }
 
@@ -339,7 +388,7 @@ __device__ __forceinline__ void dispatch_tile(int k0, int np, uint32_t stage, in
                                               const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
                                               int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
 #define FL_TILE(K0_, NP_)                                                                            \
-  if (tg == tile_groups(NP_))                                                                        \
+  if (NT == 1 && tg == tile_groups(NP_))                                                            \
     tile_compute<K0_, NP_, NT, true>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc); \
   else                                                                                               \
     tile_compute<K0_, NP_, NT, false>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc)

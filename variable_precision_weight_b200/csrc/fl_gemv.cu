@@ -53,6 +53,7 @@ constexpr int kTeamStages = 2;
 constexpr int kStages = kTeams * kTeamStages;
 constexpr int kStageBytes = 18432;
 constexpr int kMaxCtas = 1024;
+constexpr int kRed = 8;               // outputs per thread per pass of the slice reduction
 constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
 constexpr int kLevelCache = 4096;     // most units per CTA; all their plane ranges are cached in smem
 constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
@@ -132,7 +133,7 @@ __host__ __device__ constexpr uint32_t plane_mask(int k, int i) {
 }
 
 // Named barriers: 0 is __syncthreads; team t uses kBarTeam0 + t.
-enum : int { kBarGate = 1, kBarTeam0 = 2, kBarProducers = 6, kBarLevels = 7 };
+enum : int { kBarGate = 1, kBarTeam0 = 2, kBarProducers = 6, kBarLevels = 7, kBarX = 8 };
 
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -216,12 +217,14 @@ __device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, i
   }
 }
 
+// When the items take more than one round (`multi`, large batches), every warp arrives on kBarX
+// once its last round's loads are issued, and the producers hold the weight stream until then,
+// so no activation read queues behind it.
 __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int batch, int batch_pad, int tid,
-                                             int nthreads) {
+                                             int nthreads, int total, bool multi) {
   const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
-  const Slot& last = slots[nsl - 1];
-  const int total = last.it0 + batch * last.ngroups;
   int si = 0;
+  if (multi && wid >= total) bar_arrive(kBarX, kThreads);
   for (int it0 = wid; it0 < total; it0 += 4 * nw) {
     uint2 raw[4];
     int sq[4];
@@ -238,6 +241,7 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
         sq[q] = si;
       }
     }
+    if (multi && it0 + 4 * nw >= total) bar_arrive(kBarX, kThreads);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       if (sq[q] >= 0) {
@@ -248,6 +252,42 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
     }
   }
   // padded batch rows read zero constants
+  for (int i = 0; i < nsl; ++i) {
+    const Slot& sl = slots[i];
+    for (int e = tid; e < (batch_pad - batch) * sl.ngroups; e += nthreads)
+      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(sl.gconst + 8u * (uint32_t)(batch * sl.ngroups + e)),
+                   "f"(0.f), "f"(0.f)
+                   : "memory");
+  }
+}
+
+// Large batches: the activation rows of every slot arrive by one 1-D bulk copy per (slot, batch
+// row) into the idle stage buffers (item `it` at smem offset 256 it, x_bar tracks the bytes), so
+// they all take one round trip; the consumers then convert from shared memory.
+__device__ __forceinline__ void stage_x(const Slot* slots, int nsl, int batch, uint8_t* smem, uint64_t* x_bar,
+                                        int ditems) {
+  mbar_expect_tx(x_bar, (uint32_t)ditems * 256u);
+  for (int i = 0; i < nsl; ++i) {
+    const Slot& sl = slots[i];
+    for (int b = 0; b < batch; ++b)
+      bulk_g2s(smem + (size_t)(sl.it0 + b * sl.ngroups) * 256u,
+               sl.x + (size_t)b * sl.G * 128 + 128 * sl.gfirst, 256u * sl.ngroups, x_bar);
+  }
+}
+
+__device__ __forceinline__ void convert_staged(const Slot* slots, int nsl, int batch, int batch_pad,
+                                               const uint8_t* smem, int tid, int nthreads, int total) {
+  const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
+  const uint32_t base = smem_u32(smem);
+  int si = 0;
+  for (int it = wid; it < total; it += nw) {
+    while (si + 1 < nsl && it >= slots[si + 1].it0) ++si;
+    const Slot& sl = slots[si];
+    const int local = it - sl.it0;
+    uint2 raw;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(raw.x), "=r"(raw.y) : "r"(base + 256u * it + 8u * lane));
+    convert_item(raw, sl, local / sl.ngroups, local % sl.ngroups, lane);
+  }
   for (int i = 0; i < nsl; ++i) {
     const Slot& sl = slots[i];
     for (int e = tid; e < (batch_pad - batch) * sl.ngroups; e += nthreads)
@@ -547,6 +587,7 @@ template <int MAXP, int NT, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t x_bar;  // staged activations have landed
   __shared__ Slot slots[kMaxSlots];
   __shared__ uint8_t lvc[kLevelCache];
   __shared__ __align__(16) uint8_t zeros[160];
@@ -570,6 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], kTeamWarps);
     }
+    mbar_init(&x_bar, 1);
     fence_mbar_init();
     s_failed = 0;
   }
@@ -648,6 +690,10 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   // range; both sides derive the same tile sequence from the slot table and the level cache,
   // so the only hand-offs are the full / empty barriers of the team's two stages.
   const int nsl = s_nslots;
+  const int ditems = slots[nsl - 1].it0 + a.batch * slots[nsl - 1].ngroups;  // activation items
+  const bool dmulti = ditems > 4 * kConsumerWarps;
+  // staged: all activation rows fit the stage buffers, which stay idle until the digits are built
+  const bool dstaged = dmulti && ditems * 256 <= kStages * kStageBytes;
   if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producer warps
     {
@@ -660,6 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
     }
     named_bar(kBarProducers, 32 * kProducerWarps);
     bar_arrive(kBarLevels, kThreads);
+    if (dmulti) named_bar(kBarX, kThreads);
     if (lane != 0) return;
     const int team = warp - kConsumerWarps;
     int issued = 0, si = 0;
@@ -702,7 +749,19 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
 
   // ------------------------------------------------------------------ consumer warps
   // 1. activation digits of every (problem, slice) the range touches
-  build_digits(slots, nsl, a.batch, 4 * NT, threadIdx.x, kConsumers);
+  if (dstaged) {
+    if (threadIdx.x == 0) stage_x(slots, nsl, a.batch, smem, &x_bar, ditems);
+    if (!mbar_wait(&x_bar, 0u)) {
+      if (lane == 0) {
+        atomicExch(&g_error, 3);
+        s_failed = 1;
+      }
+    }
+    convert_staged(slots, nsl, a.batch, 4 * NT, smem, threadIdx.x, kConsumers, ditems);
+    bar_arrive(kBarX, kThreads);  // the stage buffers are free for the weight stream
+  } else {
+    build_digits(slots, nsl, a.batch, 4 * NT, threadIdx.x, kConsumers, ditems, dmulti);
+  }
   named_bar(kBarLevels, kThreads);  // every consumer's digits, and the producers' level cache
 
   // 2. team loop
@@ -804,16 +863,48 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       if (tt == 0) s_ticket[team] = (int)atom_add_acq_rel(&sl.tickets[b], 1u);
       named_bar(kBarTeam0 + team, kTeamThreads);
       if (s_ticket[team] == sl.slices - 1) {
-        for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
-          const int bb = e / 64, r = e % 64;
-          float sum = 0.f;
-          for (int jj = 0; jj < sl.slices; ++jj)
-            sum += __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + bb) * 64 + r);
-          float* yy = y + (size_t)bb * ystride + 64 * b + r;
-          if (a.mode == 0)
-            *yy = sum;
-          else
-            *yy += sum;
+        if (a.batch * 64 <= kTeamThreads) {  // one output per thread at most
+          const int e = tt;
+          if (e < a.batch * 64) {
+            float sum = 0.f;
+#pragma unroll 4
+            for (int jj = 0; jj < sl.slices; ++jj)
+              sum += __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + e / 64) * 64 + e % 64);
+            float* yy = y + (size_t)(e / 64) * ystride + 64 * b + e % 64;
+            if (a.mode == 0)
+              *yy = sum;
+            else
+              *yy += sum;
+          }
+        } else
+        // each thread's outputs (up to kRed) and slices: every load is issued before the sums
+        for (int e0 = tt; e0 < a.batch * 64; e0 += kRed * kTeamThreads) {
+          float sum[kRed];
+#pragma unroll
+          for (int q = 0; q < kRed; ++q) sum[q] = 0.f;
+          for (int jj = 0; jj < sl.slices; ++jj) {
+            float v[kRed];
+#pragma unroll
+            for (int q = 0; q < kRed; ++q) {
+              const int e = e0 + q * kTeamThreads;
+              v[q] = (e < a.batch * 64)
+                         ? __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + e / 64) * 64 + e % 64)
+                         : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < kRed; ++q) sum[q] += v[q];
+          }
+#pragma unroll
+          for (int q = 0; q < kRed; ++q) {
+            const int e = e0 + q * kTeamThreads;
+            if (e < a.batch * 64) {
+              float* yy = y + (size_t)(e / 64) * ystride + 64 * b + e % 64;
+              if (a.mode == 0)
+                *yy = sum[q];
+              else
+                *yy += sum[q];
+            }
+          }
         }
         if (tt == 0) sl.tickets[b] = 0u;
       }

@@ -35,6 +35,7 @@ constexpr int kTeamStages = 2;
 constexpr int kStages = kTeams * kTeamStages;
 constexpr int kStageBytes = 18432;  // 64 rows x 2 Q4_K records
 constexpr int kMaxCtas = 1024;
+constexpr int kRed = 8;               // outputs per thread per pass of the slice reduction
 constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
 constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
 constexpr int kDigitBudget = kSmemLimit - kStages * kStageBytes;
@@ -240,8 +241,8 @@ __device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, i
                  : "memory");
 }
 
-// All consumer threads; every thread arrives once on kBarX after its first loads are issued,
-// which lets the producers start the weight copies behind them.
+// All consumer threads; every thread arrives once on kBarX after its last round of loads is
+// issued, which lets the producers start the weight copies behind them.
 __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int batch, int batch_pad, int tid,
                                              int nthreads) {
   const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
@@ -264,7 +265,7 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
         sq[q] = si;
       }
     }
-    if (round == 0) bar_arrive(kBarX, kThreads);
+    if (it0 + 4 * nw >= total) bar_arrive(kBarX, kThreads);  // this warp's last round
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       if (sq[q] >= 0) {
@@ -654,12 +655,38 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       if (tt == 0) s_ticket[team] = (int)atom_add_acq_rel(&sl.tickets[b], 1u);
       named_bar(kBarTeam0 + team, kTeamThreads);
       if (s_ticket[team] == sl.slices - 1) {
-        for (int e = tt; e < a.batch * 64; e += kTeamThreads) {
-          const int bb = e / 64, r = e % 64;
-          float sum = 0.f;
-          for (int jj = 0; jj < sl.slices; ++jj)
-            sum += __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + bb) * 64 + r);
-          sl.y[(size_t)bb * ystride + 64 * b + r] = sum;
+        if (a.batch * 64 <= kTeamThreads) {  // one output per thread at most
+          const int e = tt;
+          if (e < a.batch * 64) {
+            float sum = 0.f;
+#pragma unroll 4
+            for (int jj = 0; jj < sl.slices; ++jj)
+              sum += __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + e / 64) * 64 + e % 64);
+            sl.y[(size_t)(e / 64) * ystride + 64 * b + e % 64] = sum;
+          }
+        } else
+        // each thread's outputs (up to kRed) and slices: every load is issued before the sums
+        for (int e0 = tt; e0 < a.batch * 64; e0 += kRed * kTeamThreads) {
+          float sum[kRed];
+#pragma unroll
+          for (int q = 0; q < kRed; ++q) sum[q] = 0.f;
+          for (int jj = 0; jj < sl.slices; ++jj) {
+            float v[kRed];
+#pragma unroll
+            for (int q = 0; q < kRed; ++q) {
+              const int e = e0 + q * kTeamThreads;
+              v[q] = (e < a.batch * 64)
+                         ? __ldcg(sl.partial + (((size_t)jj * sl.nblocks + b) * a.batch + e / 64) * 64 + e % 64)
+                         : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < kRed; ++q) sum[q] += v[q];
+          }
+#pragma unroll
+          for (int q = 0; q < kRed; ++q) {
+            const int e = e0 + q * kTeamThreads;
+            if (e < a.batch * 64) sl.y[(size_t)(e / 64) * ystride + 64 * b + e % 64] = sum[q];
+          }
         }
         if (tt == 0) sl.tickets[b] = 0u;
       }

@@ -34,11 +34,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "weight-bytes GB/s and fraction of HBM peak at batch 1; decode-step tokens/s"
-ESC_RATE = 0.16
 WORKLOAD = ("qwen3-0.6b-shaped decode step: 197 GEMVs (28 layers x q,k,v,o,gate,up,down + tied head "
-            "1024x151936) read at D4 from the plane store, logit gate over 151936 logits fused into the same launch, "
-            "seeded 16% of steps "
-            "escalate D4->D8 via residual planes + gate; batch 1")
+            "1024x151936) read at D4 from the plane store, logit gate over 151936 logits fused into the same launch; "
+            "a step escalates D4->D8 (residual planes + gate) when the gate says so, decided on the device; 25 "
+            "rotating input sets, entropy threshold set so 4 of them (16%) escalate; batch 1")
 
 
 def parse():
@@ -157,18 +156,6 @@ def job_rate(units_per_rank, world, t):
     return world * units_per_rank / t
 
 
-def escalation_schedule(steps, seed=1601):
-    """Exactly 16 of every 100 steps escalate, positions drawn per block of 100 (seeded)."""
-    import numpy as np
-    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed])))
-    sched = np.zeros(steps, bool)
-    for b0 in range(0, steps, 100):
-        n = min(100, steps - b0)
-        k = int(round(ESC_RATE * n))
-        sched[b0 + rng.choice(n, size=k, replace=False)] = True
-    return sched
-
-
 # ----------------------------------------------------------------------------- GPU workload
 
 def gpu_int8_layer(torch, out, inn, gen):
@@ -196,7 +183,13 @@ def plane_bytes(inn, level):
 
 
 class DecodeStep:
-    """The Qwen3-0.6B-shaped step on one GPU, captured as two CUDA graphs."""
+    """The Qwen3-0.6B-shaped step on one GPU. NSETS independent input sets rotate over the
+    steps; each set's step is one CUDA graph: the D4 pass with the logit gate fused, then the
+    D4->D8 residual pass (gate fused) conditioned on the device on the first pass's escalate
+    flag. The entropy threshold is calibrated once so that 4 of the 25 sets escalate."""
+
+    NSETS = 25
+    NESC = 4
 
     def __init__(self, torch, fl, seed):
         from variable_precision_weight_b200 import synth
@@ -207,87 +200,88 @@ class DecodeStep:
         self.stores = []
         tot_in = sum(i for _, _, i in self.shapes)
         tot_out = sum(o for _, o, _ in self.shapes)
-        self.x = torch.empty(tot_in, dtype=torch.int16, device="cuda")
-        self.x2 = torch.empty(tot_in, dtype=torch.int16, device="cuda")  # second input buffer (end to end)
+        self.xs = torch.empty((self.NSETS, tot_in), dtype=torch.int16, device="cuda")
         self.y = torch.empty(tot_out, dtype=torch.float32, device="cuda")
         self.h2d_bytes = tot_in * 2
-        lv_d4, lv_d8, items, items_r, items2, items_r2 = [], [], [], [], [], []
+        items = [[] for _ in range(self.NSETS)]
+        items_r = [[] for _ in range(self.NSETS)]
         oi = oo = 0
         self.bytes_d4 = self.bytes_res = 0
+        self.levels = []
         for name, o, i in self.shapes:
             st = plane_layer(torch, fl, o, i, gen)
             self.stores.append(st)
             d4 = torch.full((o // 64,), 2, dtype=torch.uint8, device="cuda")
             d8 = torch.full((o // 64,), 4, dtype=torch.uint8, device="cuda")
-            lv_d4.append(d4)
-            lv_d8.append(d8)
-            xs = self.x[oi:oi + i]
+            self.levels += [d4, d8]
             ys = self.y[oo:oo + o]
-            items.append((st, o, i, d4, None, xs, ys))
-            items_r.append((st, o, i, d4, d8, xs, ys))
-            items2.append((st, o, i, d4, None, self.x2[oi:oi + i], ys))
-            items_r2.append((st, o, i, d4, d8, self.x2[oi:oi + i], ys))
+            for j in range(self.NSETS):
+                xs = self.xs[j, oi:oi + i]
+                items[j].append((st, o, i, d4, None, xs, ys))
+                items_r[j].append((st, o, i, d4, d8, xs, ys))
             self.bytes_d4 += (o // 64) * plane_bytes(i, 2)
             self.bytes_res += (o // 64) * (256 * (i // 128) + 2048 * (i // 128) * 2)
             oi += i
             oo += o
-        self.levels = (lv_d4, lv_d8)
-        self.head_logits = self.y[oo - self.shapes[-1][1]:oo]
         self.vocab = self.shapes[-1][1]
-        self.prob_d4 = fl.gemv_problems(items)
-        self.prob_res = fl.gemv_problems(items_r)
-        self.prob_d4_2 = fl.gemv_problems(items2)
-        self.prob_res_2 = fl.gemv_problems(items_r2)
-        self.n = len(items)
-        # gate outputs (one buffer so one device->host copy reads the step's result); the gate
-        # runs fused into the batched GEMV over the head's outputs (problem n - 1)
-        self.gate = torch.zeros(8, dtype=torch.int32, device="cuda")
-        self.tau_h, self.tau_m = 11.8, 1e-6
+        self.prob_d4 = [fl.gemv_problems(it) for it in items]
+        self.prob_res = [fl.gemv_problems(it) for it in items_r]
+        self.n = len(items[0])
+        # gate outputs per set (one 32-byte row, so one device->host copy reads a step's result)
+        self.gates = torch.zeros((self.NSETS, 8), dtype=torch.int32, device="cuda")
         wsb = fl.fl_gemv_gate_workspace_bytes(1)
         self.gate_ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
-        g = self.gate
-        self.spec = fl.gate_spec(self.n - 1, self.tau_h, self.tau_m, g[0:1].view(torch.float32),
+        self.runs = torch.zeros(1, dtype=torch.int32, device="cuda")  # residual passes that ran
+        self.hx = [synth.bf16_normal((tot_in,), seed, 99, j).view("int16") for j in range(self.NSETS)]
+        for j in range(self.NSETS):
+            self.xs[j].copy_(torch.from_numpy(self.hx[j]))
+        self.tau_h, self.tau_m = self._calibrate(wsb)
+        self.specs = [self._spec(j, wsb) for j in range(self.NSETS)]
+
+    def _spec(self, j, wsb, tau_h=None, tau_m=None):
+        torch, g = self.torch, self.gates[j]
+        return self.fl.gate_spec(self.n - 1, self.tau_h if tau_h is None else tau_h,
+                                 self.tau_m if tau_m is None else tau_m, g[0:1].view(torch.float32),
                                  g[1:2].view(torch.float32), g[2:4], g[4:5].view(torch.uint8)[0:1], self.gate_ws, wsb)
-        self.gate2 = torch.zeros(8, dtype=torch.int32, device="cuda")  # gate outputs of the second buffer's step
-        g2 = self.gate2
-        self.spec2 = fl.gate_spec(self.n - 1, self.tau_h, self.tau_m, g2[0:1].view(torch.float32),
-                                  g2[1:2].view(torch.float32), g2[2:4], g2[4:5].view(torch.uint8)[0:1], self.gate_ws,
-                                  wsb)
-        gx = synth.bf16_normal((tot_in,), seed, 99)
-        self.x.copy_(torch.from_numpy(gx.view("int16")))
-        self.x2.copy_(self.x)
 
-    def low_pass(self, second=False):
-        self.fl.fl_gemv_batched_gate(self.prob_d4_2 if second else self.prob_d4, self.n, 1, 0,
-                                     self.spec2 if second else self.spec)
+    def _calibrate(self, wsb):
+        """Entropy threshold between the NESC-th and next largest entropies of the sets' D4
+        logits; the margin threshold below every set's margin (it never decides)."""
+        import numpy as np
+        torch = self.torch
+        for j in range(self.NSETS):
+            self.fl.fl_gemv_batched_gate(self.prob_d4[j], self.n, 1, 0, self._spec(j, wsb, 1e30, -1.0))
+        torch.cuda.synchronize()
+        H = self.gates[:, 0].view(torch.float32).cpu().numpy().astype(np.float64)
+        M = self.gates[:, 1].view(torch.float32).cpu().numpy().astype(np.float64)
+        h = np.sort(H)[::-1]
+        self.calib = {"entropy_sorted": h.tolist(), "margin_min": float(M.min())}
+        return float(0.5 * (h[self.NESC - 1] + h[self.NESC])), float(0.5 * M.min())
 
-    def escalate(self, second=False):
-        self.fl.fl_gemv_batched_gate(self.prob_res_2 if second else self.prob_res, self.n, 1, 1,
-                                     self.spec2 if second else self.spec)
+    def step_graph_body(self, j):
+        fl = self.fl
+        fl.fl_gemv_batched_gate(self.prob_d4[j], self.n, 1, 0, self.specs[j])
+        esc = self.gates[j, 4:5].view(self.torch.uint8)[0:1]
+        fl.fl_gemv_batched_gate_if(self.prob_res[j], self.n, 1, 1, self.specs[j], esc, self.runs)
 
     def gemv_only(self):
         # the step's dominant kernel as the step runs it (D4 pass, gate fused)
-        self.fl.fl_gemv_batched_gate(self.prob_d4, self.n, 1, 0, self.spec)
+        self.fl.fl_gemv_batched_gate(self.prob_d4[0], self.n, 1, 0, self.specs[0])
 
     def capture(self):
         torch = self.torch
-        for _ in range(3):
-            self.low_pass()
-            self.escalate()
+        for j in range(self.NSETS):
+            self.step_graph_body(j)
         torch.cuda.synchronize()
-        self.gA, self.gB, self.gK = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.gA):
-            self.low_pass()
-        with torch.cuda.graph(self.gB):
-            self.escalate()
+        self.g = []
+        for j in range(self.NSETS):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                self.step_graph_body(j)
+            self.g.append(gr)
+        self.gK = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.gK):
             self.gemv_only()
-        # the same step reading the second input buffer (end to end, double-buffered inputs)
-        self.gA2, self.gB2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.gA2):
-            self.low_pass(second=True)
-        with torch.cuda.graph(self.gB2):
-            self.escalate(second=True)
         torch.cuda.synchronize()
 
 
@@ -504,94 +498,84 @@ def run_fl(args, rank, world, local_rank):
     peak, peak_kind = load_peaks()
     step = DecodeStep(torch, fl, seed=1000 + rank)
     step.capture()
-    sched = escalation_schedule(args.steps + args.warmup)
+    NS = step.NSETS
 
     if args.profile != "none":
         for k in range(3):
-            step.gA.replay()
-            if sched[k]:
-                step.gB.replay()
+            step.g[k].replay()
         torch.cuda.synchronize()
         if args.profile == "kernels":
             extra_measurements(torch, fl, peak)
         return 0
 
     def body(k):
-        step.gA.replay()
-        if sched[args.warmup + k]:
-            step.gB.replay()
+        step.g[(args.warmup + k) % NS].replay()
 
     for k in range(args.warmup):
-        step.gA.replay()
-        if sched[k]:
-            step.gB.replay()
+        step.g[k % NS].replay()
+    step.runs.zero_()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         t = time_loop(torch, body, args.steps)
     t = max_over_ranks(t, world)
-    n_esc = int(sched[args.warmup:args.warmup + args.steps].sum())
+    n_esc = int(step.runs.item())                 # residual passes the device decided to run
     value = job_rate(args.steps * step.bytes_d4 + n_esc * step.bytes_res, world, t) / 1e9
     tok_s = job_rate(args.steps, world, t)
 
-    # dominant kernel alone: the batched D4 GEMV, graph-replayed back to back
+    # dominant kernel alone: the step's D4 pass (gate fused), graph-replayed back to back
     reps = max(200, args.steps // 10)
     tk = time_loop(torch, lambda k: step.gK.replay(), reps) / reps
     achieved = step.bytes_d4 / tk / 1e9
 
     # end to end: each step copies its inputs host->device (pinned) and reads the gate result back.
-    # The layer inputs of successive steps are independent, so the copy of step k + 1's inputs
-    # runs on a second stream while step k computes (two device buffers); every copy is inside
-    # the timed region.
-    nbuf = 4
-    from variable_precision_weight_b200 import synth
-    hx = [torch.from_numpy(synth.bf16_normal((step.x.numel(),), 7, b).view("int16")).pin_memory()
-          for b in range(nbuf)]
+    # The input sets are independent, so step k + 2's input copy and step k's read-back run on a
+    # second stream while step k + 1 computes (one device buffer and gate row per set, ordered by
+    # events); every copy is inside the timed region.
+    hx = [torch.from_numpy(step.hx[j]).pin_memory() for j in range(NS)]
     hres = torch.empty(8, dtype=torch.int32).pin_memory()
     main = torch.cuda.current_stream()
     side = torch.cuda.Stream()
-    dbuf, gbuf = (step.x, step.x2), (step.gate, step.gate2)
-    graphs = ((step.gA, step.gB), (step.gA2, step.gB2))
-    ev_copy = (torch.cuda.Event(), torch.cuda.Event())
-    ev_used = (torch.cuda.Event(), torch.cuda.Event())
+    ev_copy = [torch.cuda.Event() for _ in range(NS)]
+    ev_used = [torch.cuda.Event() for _ in range(NS)]
     ev_side = torch.cuda.Event()
+    e2e_steps = min(args.steps, 5000)
 
     def side_work(k, read_back):
-        # on the side stream, after the step that last used buffer k % 2: read its gate result,
-        # then copy step k's inputs into the buffer
-        j = k % 2
+        # after the step that last used set k % NS: read its gate row, then copy step k's inputs
+        j, jb = k % NS, (k - 2) % NS
         with torch.cuda.stream(side):
-            side.wait_event(ev_used[j])
             if read_back:
-                hres.copy_(gbuf[j], non_blocking=True)
+                side.wait_event(ev_used[jb])
+                hres.copy_(step.gates[jb], non_blocking=True)
             if k < e2e_steps:
-                dbuf[j].copy_(hx[k % nbuf], non_blocking=True)
-            ev_copy[j].record(side)
+                side.wait_event(ev_used[j])
+                step.xs[j].copy_(hx[j], non_blocking=True)
+                ev_copy[j].record(side)
 
     def body_e2e(k):
-        j = k % 2
+        j = k % NS
         if k == 0:
             side_work(0, False)
             side_work(1, False)
         main.wait_event(ev_copy[j])
-        graphs[j][0].replay()
-        if sched[args.warmup + k]:
-            graphs[j][1].replay()
+        step.g[j].replay()
         ev_used[j].record(main)
         side_work(k + 2, True)                   # read step k's result, copy step k + 2's inputs
-        if k == e2e_steps - 1:                   # the last read-backs end inside the timed region
+        if k == e2e_steps - 1:                   # the last read-back ends inside the timed region
             ev_side.record(side)
             main.wait_event(ev_side)
 
-    for j in range(2):
+    for j in range(NS):
         ev_used[j].record(main)
-    e2e_steps = min(args.steps, 5000)
+    step.runs.zero_()
     if world > 1:
         dist.barrier()
+    torch.cuda.synchronize()
     te = time_loop(torch, body_e2e, e2e_steps)
     te = max_over_ranks(te, world)
-    n_esc_e = int(sched[args.warmup:args.warmup + e2e_steps].sum())
+    n_esc_e = int(step.runs.item())
     e2e_val = job_rate(e2e_steps * step.bytes_d4 + n_esc_e * step.bytes_res, world, te) / 1e9
 
     extra = None
@@ -610,6 +594,8 @@ def run_fl(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": 1, "weight_bytes_per_step_d4": step.bytes_d4,
                    "weight_bytes_per_escalation": step.bytes_res, "escalated_steps": n_esc,
+                   "gate_thresholds": {"entropy": step.tau_h, "margin": step.tau_m,
+                                       "escalating_sets": f"{step.NESC} of {step.NSETS}"},
                    "l2": "inputs larger than L2 (316.6 MB of weights read per step vs 126 MB L2)",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "tokens_per_s": tok_s, "hbm_frac": value / world / peak, "peak_gbs": peak, "peak_kind": peak_kind,
@@ -624,7 +610,7 @@ def run_fl(args, rank, world, local_rank):
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": step.h2d_bytes,
                 "d2h_bytes_per_step": 32, "steps": e2e_steps,
                 "tokens_per_s": job_rate(e2e_steps, world, te)},
-        "gpu_launches": args.steps + n_esc,
+        "gpu_launches": 2 * args.steps,  # D4 pass + conditional residual pass (returns at once when not needed)
         "clocks": clk.summary(),
         "kernels": extra,
     }

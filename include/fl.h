@@ -246,6 +246,15 @@ FL_API size_t fl_gemv_gate_workspace_bytes(int batch);
 FL_API fl_status fl_gemv_batched_gate(const fl_gemv_problem* problems, int n, int batch, int mode,
                                const fl_gate_spec* gate, void* stream);
 
+/* Device-side conditional escalation ([PoD] abstract: redo only the uncertain steps, here
+ * decided on the device, with no read-back to the host): fl_gemv_batched_gate that runs
+ * only if the byte at run_if (device, typically the escalate flag a preceding gated pass
+ * wrote) is non-zero, and otherwise returns at once, leaving y and the gate outputs as
+ * they were. runs: device uint32 or NULL; each pass that ran adds 1 to it. */
+FL_API fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, int n, int batch, int mode,
+                                  const fl_gate_spec* gate, const uint8_t* run_if, uint32_t* runs,
+                                  void* stream);
+
 /* ========================================================================= */
 /* Uncertainty gate ([PoD]: redo at 8 bits when the low-precision output     */
 /* distribution looks uncertain: entropy above a threshold or a small        */

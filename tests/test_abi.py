@@ -95,6 +95,8 @@ def test_host_side_rejections(fl):
     assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == -6
     spec = fl.gate_spec(0, 0.0, 0.0, 16, 16, 16, 16, 17, gsz)                  # misaligned workspace
     assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == -4
+    spec = fl.gate_spec(0, 0.0, 0.0, 16, 16, 16, 16, 16, gsz)
+    assert _status(fl, fl.fl_gemv_batched_gate_if, probs, 1, 1, 1, spec, None, None, s0) == ERR_ARG   # no run_if
     kp = fl.kquant_problems([(16, 11, 64, 256, 16, 16)])
     assert _status(fl, fl.fl_gemv_kquant_batched, kp, 1, 1, s0) == ERR_UNSUP
     assert "Q4_K" in fl.fl_last_error()

@@ -276,6 +276,39 @@ def test_batched_gate_fused(env, orc, batch, gate_index):
         assert np.allclose(e2.cpu().numpy(), ge, rtol=1e-5, atol=1e-6)
 
 
+def test_conditional_escalation_on_device(env, orc):
+    """The residual pass conditioned on the gate's escalate flag: it runs (y becomes the D8
+    result, the run counter ticks) when the flag is set, and leaves y untouched otherwise."""
+    torch, fl = env
+    shapes = [(1024, 1024), (2048, 1024)]          # problem 1 is the gate's logits
+    items, layers = [], []
+    for i, (o, n) in enumerate(shapes):
+        q, s = synth.int8_layer(o, n, 95, i)
+        lv = np.full(o // 64, 2, np.uint8)
+        x = synth.bf16_normal((1, n), 96, i)
+        st = pack_gpu(torch, fl, q, s)
+        y = torch.zeros((1, o), dtype=torch.float32, device="cuda")
+        items.append((st, o, n, dev(torch, lv), torch.full((o // 64,), 4, dtype=torch.uint8, device="cuda"),
+                      dev(torch, x), y))
+        layers.append((q, s, lv, x))
+    arr = fl.gemv_problems(items)
+    wsb = fl.fl_gemv_gate_workspace_bytes(1)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    e, m = torch.empty(1, device="cuda"), torch.empty(1, device="cuda")
+    t2, es = torch.empty((1, 2), dtype=torch.int32, device="cuda"), torch.empty(1, dtype=torch.uint8, device="cuda")
+    runs = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for tau_h, want in ((-1.0, 1), (1e9, 0)):                        # H > -1 always; H > 1e9 never
+        spec = fl.gate_spec(1, tau_h, -1.0, e, m, t2, es, ws, wsb)     # margin < -1 never
+        fl.fl_gemv_batched_gate(arr, 2, 1, 0, spec)
+        fl.fl_gemv_batched_gate_if(arr, 2, 1, 1, spec, es, runs)
+        torch.cuda.synchronize()
+        assert int(es.item()) == want
+        for (q, s, lv, x), it in zip(layers, items):
+            yref, mass = orc.gemv_depth(q, s, np.full_like(lv, 4) if want else lv, x, with_mass=True)
+            check_close(it[6].cpu().numpy(), yref, mass, f"conditional pass, escalate={want}")
+    assert int(runs.item()) == 1
+
+
 # ----------------------------------------------------------------------------- level map
 
 def test_level_map_bit_exact(env, orc, golden):

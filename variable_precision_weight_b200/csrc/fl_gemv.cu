@@ -95,6 +95,10 @@ struct Args {
   uint32_t* gate_ticket;   // launch counter, zero between launches
   GateRec* gate_part;      // [kMaxCtas][FL_MAX_BATCH] per-CTA partials
   int gate_cta0, gate_ncta;  // the CTAs whose unit ranges hold gate-problem units
+  // conditional launch: the pass runs only if *run_if != 0 (run_if NULL: always); runs
+  // (optional) counts the passes that ran
+  const uint8_t* run_if;
+  uint32_t* runs;
   Problem p[MAXP];
 };
 
@@ -680,6 +684,10 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   }
   __syncthreads();
   pdl_wait();  // everything above read only the parameters
+  if (a.run_if != nullptr) {
+    if (*reinterpret_cast<const volatile uint8_t*>(a.run_if) == 0) return;  // every thread reads the same byte
+    if (blockIdx.x == 0 && threadIdx.x == 0 && a.runs != nullptr) atomicAdd(a.runs, 1u);
+  }
 
   // Before any weight copy is in flight (they would queue ahead of these small reads): the
   // producer threads read the level bytes into the level cache while the consumer threads read
@@ -1094,6 +1102,8 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   a.batch = batch;
   a.mode = mode;
   a.gate_p = -1;
+  a.run_if = nullptr;
+  a.runs = nullptr;
   Problem& P = a.p[0];
   P.store = w->store;
   P.lv_from = lv_from;
@@ -1149,7 +1159,7 @@ constexpr size_t kGateTicketBytes = 256;
 constexpr size_t kGateWorkspaceBytes = kGateTicketBytes + (size_t)kMaxCtas * FL_MAX_BATCH * sizeof(GateRec);
 
 static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int mode, const fl_gate_spec* gate,
-                         void* stream, const char* what) {
+                         const uint8_t* run_if, uint32_t* runs, void* stream, const char* what) {
   if (!problems) return fail(FL_ERR_ARG, "%s: problems is NULL", what);
   if (n < 1 || n > FL_MAX_PROBLEMS) return fail(FL_ERR_ARG, "%s: n=%d (1..%d)", what, n, FL_MAX_PROBLEMS);
   if (mode != 0 && mode != 1) return fail(FL_ERR_ARG, "%s: mode=%d (0 depth, 1 residual)", what, mode);
@@ -1159,6 +1169,8 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
   a.batch = batch;
   a.mode = mode;
   a.gate_p = -1;
+  a.run_if = run_if;
+  a.runs = runs;
   size_t budget = kDigitBudget;
   if (gate) {
     if (gate->problem < 0 || gate->problem >= n)
@@ -1228,7 +1240,7 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
 }  // namespace fl
 
 extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream) {
-  return gemv::batched(problems, n, batch, mode, nullptr, stream, "fl_gemv_batched");
+  return gemv::batched(problems, n, batch, mode, nullptr, nullptr, nullptr, stream, "fl_gemv_batched");
 }
 
 extern "C" size_t fl_gemv_gate_workspace_bytes(int batch) {
@@ -1239,7 +1251,16 @@ extern "C" size_t fl_gemv_gate_workspace_bytes(int batch) {
 extern "C" fl_status fl_gemv_batched_gate(const fl_gemv_problem* problems, int n, int batch, int mode,
                                           const fl_gate_spec* gate, void* stream) {
   if (!gate) return fail(FL_ERR_ARG, "fl_gemv_batched_gate: gate spec is NULL");
-  return gemv::batched(problems, n, batch, mode, gate, stream, "fl_gemv_batched_gate");
+  return gemv::batched(problems, n, batch, mode, gate, nullptr, nullptr, stream, "fl_gemv_batched_gate");
+}
+
+extern "C" fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, int n, int batch, int mode,
+                                             const fl_gate_spec* gate, const uint8_t* run_if, uint32_t* runs,
+                                             void* stream) {
+  const char* what = "fl_gemv_batched_gate_if";
+  if (!gate) return fail(FL_ERR_ARG, "%s: gate spec is NULL", what);
+  if (!run_if) return fail(FL_ERR_ARG, "%s: run_if is NULL", what);
+  return gemv::batched(problems, n, batch, mode, gate, run_if, runs, stream, what);
 }
 
 // ---------------------------------------------------------------- allocation-free variant

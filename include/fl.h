@@ -60,7 +60,8 @@ typedef enum {
   FL_ERR_UNSUPPORTED = -3,  /* a weight type the fast path does not implement  */
   FL_ERR_ALIGN = -4,        /* a pointer is not aligned as the call requires   */
   FL_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed            */
-  FL_ERR_WORKSPACE = -6     /* workspace missing or smaller than required      */
+  FL_ERR_WORKSPACE = -6,    /* workspace missing or smaller than required      */
+  FL_ERR_TIMEOUT = -7       /* a kernel's bounded wait ran out (fl_device_status) */
 } fl_status;
 
 #define FL_MAX_BATCH 16
@@ -73,6 +74,19 @@ typedef enum {
 #define FL_GGML_Q6_K 14
 
 FL_API const char* fl_status_string(int status);
+
+/* Device-side failure detection. Every wait inside a kernel (a stage barrier, the gate's
+ * cluster hand-off) is bounded; when one runs out the kernel records an error word and
+ * returns instead of hanging, and its outputs are not valid. The launching call cannot
+ * see that (it returned before the kernel ran), so this call waits for the device,
+ * reads and clears every kernel's error word, and returns FL_ERR_TIMEOUT (with
+ * fl_last_error naming the kernel and the wait) or FL_OK. */
+FL_API fl_status fl_device_status(void);
+
+/* Self-test of the failure path above: one thread waits, with a short limit, on a
+ * barrier that nothing completes, and records the time-out like a real wait would. The
+ * next fl_device_status returns FL_ERR_TIMEOUT. */
+FL_API fl_status fl_selftest_wait_timeout(void* stream);
 FL_API const char* fl_last_error(void);
 FL_API int fl_version(void);
 

@@ -459,3 +459,24 @@ def test_kquant_unsupported_type_fails_on_device_box(env):
     with pytest.raises(fl.FlError) as e:
         fl.fl_gemv_kquant(blk, 13, 64, 256, x, 1, y)
     assert e.value.status == -3
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+def test_device_status_reports_a_bounded_wait_that_ran_out(env, orc):
+    """A wait that nothing completes runs out after its short limit; fl_device_status reports it
+    once and clears it, and the context keeps working."""
+    torch, fl = env
+    fl.fl_device_status()                                   # clean slate (raises if anything ran out)
+    fl.fl_selftest_wait_timeout()
+    with pytest.raises(fl.FlError) as e:
+        fl.fl_device_status()
+    assert e.value.status == -7 and "self-test" in str(e.value)
+    fl.fl_device_status()                                   # cleared
+    q, s = synth.int8_layer(256, 512, 97, 0)
+    lv = synth.seeded_levels(4, 97, 1)
+    x = synth.bf16_normal((1, 512), 97, 2)
+    y, _ = gemv_gpu(torch, fl, pack_gpu(torch, fl, q, s), 256, 512, lv, x)
+    yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+    check_close(y, yref, mass, "GEMV after a reported time-out")
+    fl.fl_device_status()

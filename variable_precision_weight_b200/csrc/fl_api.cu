@@ -56,6 +56,7 @@ extern "C" const char* fl_status_string(int status) {
     case FL_ERR_ALIGN: return "FL_ERR_ALIGN";
     case FL_ERR_CUDA: return "FL_ERR_CUDA";
     case FL_ERR_WORKSPACE: return "FL_ERR_WORKSPACE";
+    case FL_ERR_TIMEOUT: return "FL_ERR_TIMEOUT";
     default: return "FL_ERR_UNKNOWN";
   }
 }
@@ -63,3 +64,28 @@ extern "C" const char* fl_status_string(int status) {
 extern "C" const char* fl_last_error(void) { return fl::g_msg; }
 
 extern "C" int fl_version(void) { return 1; }
+
+namespace fl {
+namespace gemv {
+int take_device_error();
+}
+namespace kq {
+int take_device_error();
+}
+int take_gate_error();
+}  // namespace fl
+
+extern "C" fl_status fl_device_status(void) {
+  using namespace fl;
+  FL_CHECK_CUDA(cudaDeviceSynchronize(), "fl_device_status: cudaDeviceSynchronize");
+  const int g = gemv::take_device_error(), k = kq::take_device_error(), t = take_gate_error();
+  if (g < 0 || k < 0 || t < 0) return fail(FL_ERR_CUDA, "fl_device_status: reading the error words failed");
+  if (g == 0 && k == 0 && t == 0) return FL_OK;
+  auto what = [](int c) {
+    return c == 1 ? "a producer's wait for a free stage" : c == 2 ? "a consumer's wait for a full stage"
+         : c == 3 ? "the wait for staged activations" : c == 4 ? "the self-test wait" : "a wait";
+  };
+  if (g) return fail(FL_ERR_TIMEOUT, "plane GEMV: %s ran out (code %d); its outputs are not valid", what(g), g);
+  if (k) return fail(FL_ERR_TIMEOUT, "K-quant GEMV: %s ran out (code %d); its outputs are not valid", what(k), k);
+  return fail(FL_ERR_TIMEOUT, "logit gate: the wait for the cluster's partials ran out; its outputs are NaN");
+}

@@ -164,6 +164,18 @@ static cudaError_t gate_launch(const float* logits, int vocab, int batch, float 
 
 }  // namespace fl
 
+namespace fl {
+
+// Reads and clears the error word (-1 if that fails).
+int take_gate_error() {
+  int v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_gate_error, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0 && cudaMemcpyToSymbol(g_gate_error, &z, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+}  // namespace fl
+
 extern "C" fl_status fl_logit_gate(const float* logits, int vocab, int batch, float tau_h, float tau_m,
                                    float* entropy, float* margin, int32_t* top2, uint8_t* escalate, void* stream) {
   using namespace fl;

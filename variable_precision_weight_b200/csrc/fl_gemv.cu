@@ -1263,6 +1263,35 @@ extern "C" fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, in
   return gemv::batched(problems, n, batch, mode, gate, run_if, runs, stream, what);
 }
 
+// ---------------------------------------------------------------- failure detection
+namespace fl {
+namespace gemv {
+
+// Reads and clears the error word (-1 if that fails).
+int take_device_error() {
+  int v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0 && cudaMemcpyToSymbol(g_error, &z, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+// One thread waits (100 polls) on a barrier that expects an arrival nobody makes.
+__global__ void selftest_timeout_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait(&bar, 0u, 100u)) atomicExch(&g_error, 4);
+}
+
+}  // namespace gemv
+}  // namespace fl
+
+extern "C" fl_status fl_selftest_wait_timeout(void* stream) {
+  FL_CHECK_CUDA(launch_pdl(gemv::selftest_timeout_kernel, dim3(1), dim3(1), 0, static_cast<cudaStream_t>(stream), 1),
+                "launch selftest_timeout");
+  return FL_OK;
+}
+
 // ---------------------------------------------------------------- allocation-free variant
 // The column-split scratch of fl_gemv_depth_static: one fixed array in the device image
 // (tickets first, then the slice partials, as in a caller workspace). Its device address is

@@ -819,6 +819,20 @@ static fl_status check_tensor(const void* blocks, int type, int out, int in, con
 }  // namespace kq
 }  // namespace fl
 
+namespace fl {
+namespace kq {
+
+// Reads and clears the error word (-1 if that fails).
+int take_device_error() {
+  int v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error, sizeof(int)) != cudaSuccess) return -1;
+  if (v != 0 && cudaMemcpyToSymbol(g_error, &z, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+}  // namespace kq
+}  // namespace fl
+
 using namespace fl;
 
 extern "C" size_t fl_kquant_bytes(int ggml_type, int out, int in) {

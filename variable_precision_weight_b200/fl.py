@@ -27,7 +27,7 @@ FL_GGML_Q4_K = 12
 FL_GGML_Q6_K = 14
 FL_GEMV_STATIC_SCRATCH_BYTES = 4 << 20
 STATUS = {0: "FL_OK", -1: "FL_ERR_ARG", -2: "FL_ERR_SHAPE", -3: "FL_ERR_UNSUPPORTED", -4: "FL_ERR_ALIGN",
-          -5: "FL_ERR_CUDA", -6: "FL_ERR_WORKSPACE"}
+          -5: "FL_ERR_CUDA", -6: "FL_ERR_WORKSPACE", -7: "FL_ERR_TIMEOUT"}
 
 
 class FlError(RuntimeError):
@@ -70,6 +70,8 @@ _sigs = {
     "fl_pack_planes": (_I, [_P, _P, _I, _I, _P, _P]),
     "fl_level_map": (_I, [_P, _I, _P, _P, _I, C.POINTER(fl_lens_params), _P, _P, _P]),
     "fl_gemv_workspace_bytes": (_S, [_I, _I, _I]),
+    "fl_device_status": (_I, []),
+    "fl_selftest_wait_timeout": (_I, [_P]),
     "fl_gemv_depth": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P, _S, _P]),
     "fl_gemv_depth_static": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P]),
     "fl_gemv_residual": (_I, [C.POINTER(fl_plane_weight), _P, _P, _P, _I, _P, _P, _S, _P]),
@@ -151,6 +153,15 @@ def fl_level_map(xy, nblocks: int, centers, radii, nlenses: int, params: fl_lens
                  stream=None) -> None:
     _check(_lib.fl_level_map(_ptr(xy), nblocks, _ptr(centers), _ptr(radii), nlenses, C.byref(params), _ptr(levels),
                              _ptr(counts), _stream(stream)))
+
+
+def fl_device_status() -> None:
+    """Raises FlError(FL_ERR_TIMEOUT) if a kernel's bounded wait ran out since the last call."""
+    _check(_lib.fl_device_status())
+
+
+def fl_selftest_wait_timeout(stream=None) -> None:
+    _check(_lib.fl_selftest_wait_timeout(_stream(stream)))
 
 
 def fl_gemv_workspace_bytes(out: int, inn: int, batch: int) -> int:

@@ -47,9 +47,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["fl", "reference"], default="fl")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config kernel measurements")
-    ap.add_argument("--profile", choices=["none", "step", "kernels"], default="none",
-                    help="short run for an ncu capture: 'step' = the decode step only, 'kernels' = one pass of "
-                         "every per-config kernel measurement; no JSON timing claims")
+    ap.add_argument("--profile", choices=["none", "step", "kquant", "kernels"], default="none",
+                    help="short run for an ncu capture: 'step' = the decode step only, 'kquant' = the K-quant "
+                         "step only, 'kernels' = one pass of every per-config kernel measurement; no JSON "
+                         "timing claims")
     return ap.parse_args()
 
 
@@ -304,6 +305,30 @@ def time_loop(torch, body, steps):
 
 # ----------------------------------------------------------------------------- per-config kernel lines
 
+def kquant_step(torch, fl):
+    """The Llama-3.2-1B-shaped K-quant step (96 Q4_K + 17 Q6_K tensors, seeded Gaussian weights
+    encoded on the host), resident on the device: (problems, tensors to keep alive, record bytes)."""
+    import concurrent.futures as cf
+    from variable_precision_weight_b200 import synth
+    mix = synth.llama32_kquant_mix()
+
+    def make(k):
+        name, o, i, tp = mix[k]
+        return synth.encode_kquant(synth.gaussian_weights(o, i, 4, k), tp)
+
+    with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 4)) as ex:
+        blobs = list(ex.map(make, range(len(mix))))
+    items, keep, nbytes = [], [], 0
+    for k, ((name, o, i, tp), blob) in enumerate(zip(mix, blobs)):
+        blk = torch.from_numpy(blob).cuda()
+        x = torch.from_numpy(synth.bf16_normal((1, i), 4, 1000 + k).view("int16")).cuda()
+        y = torch.empty((1, o), device="cuda")
+        keep += [blk, x, y]
+        items.append((blk, tp, o, i, x, y))
+        nbytes += blk.numel()
+    return items, keep, nbytes
+
+
 def extra_measurements(torch, fl, peak):
     """One line per other configuration: its kernel's weight-byte rate, timed over CUDA-graph replays
     with enough rotating copies of the weights that every replay reads past the 126 MB L2."""
@@ -404,28 +429,13 @@ def extra_measurements(torch, fl, peak):
         torch.cuda.empty_cache()
 
     # config 4: Llama-3.2-1B-shaped K-quant step (96 Q4_K + 17 Q6_K tensors), batch 1
-    import concurrent.futures as cf
-    mix = synth.llama32_kquant_mix()
-
-    def make(k):
-        name, o, i, tp = mix[k]
-        return synth.encode_kquant(synth.gaussian_weights(o, i, 4, k), tp)
-
-    with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 4)) as ex:
-        blobs = list(ex.map(make, range(len(mix))))
-    items, keep, nbytes = [], [], 0
-    for k, ((name, o, i, tp), blob) in enumerate(zip(mix, blobs)):
-        blk = torch.from_numpy(blob).cuda()
-        x = torch.from_numpy(synth.bf16_normal((1, i), 4, 1000 + k).view("int16")).cuda()
-        y = torch.empty((1, o), device="cuda")
-        keep += [blk, x, y]
-        items.append((blk, tp, o, i, x, y))
-        nbytes += blk.numel()
-    del blobs
+    items, keep, nbytes = kquant_step(torch, fl)
     arr = fl.kquant_problems(items)
     t = graph_time(lambda: fl.fl_gemv_kquant_batched(arr, len(items), 1), 100)
+    tr = traffic_record("kquant_gemv_llama32_1b_step")
     out["cfg4_llama32_1b_kquant_step"] = {"us": t * 1e6, "GBps": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
-                                          "tokens_per_s": 1.0 / t, "bytes": nbytes}
+                                          "tokens_per_s": 1.0 / t, "bytes": nbytes,
+                                          "traffic": tr["bytes_per_launch"] if tr else None}
     del keep, items, arr
     torch.cuda.empty_cache()
     return out
@@ -502,6 +512,13 @@ def run_fl(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     peak, peak_kind = load_peaks()
+    if args.profile == "kquant":
+        items, keep, _ = kquant_step(torch, fl)
+        arr = fl.kquant_problems(items)
+        for k in range(3):
+            fl.fl_gemv_kquant_batched(arr, len(items), 1)
+        torch.cuda.synchronize()
+        return 0
     step = DecodeStep(torch, fl, seed=1000 + rank)
     step.capture()
     NS = step.NSETS

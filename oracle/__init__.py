@@ -58,6 +58,7 @@ def _load():
                 "orc_lens_kappa": (i, [f, i, i]),
                 "orc_level_map": (None, [P, i, P, P, i, f, f, i, i, i, P, i, P]),
                 "orc_memory_bits": (d, [P, i, P, P]),
+                "orc_level_decide": (i, [P, i, i, P, i, i, i, i, d, d, P, P]),
                 "orc_logit_gate": (None, [P, i, i, d, d, P, P, P, P]),
                 "orc_dequant_q4k": (None, [P, P]),
                 "orc_dequant_q6k": (None, [P, i, P]),
@@ -168,6 +169,26 @@ def level_map(xy, cxy, r, f, g, gamma, m, stops, combine: int) -> np.ndarray:
     _load().orc_level_map(_p(xy), xy.shape[0], _p(cxy), _p(r), cxy.shape[0], float(f), float(g), int(gamma),
                           int(m), nst, _p(stops), int(combine), _p(lev))
     return lev
+
+
+def level_decide(y, scales, gamma: int, kappa: int, rule: int, lam: float = 0.0, f: float = 0.0):
+    """In-pass level decision from a layer's base-level outputs y [batch, out] and its
+    scales [out, in / 128]: (levels uint8 [out / 64], reduced scores float64 [out / 64])."""
+    y = np.ascontiguousarray(y, np.float32)
+    if y.ndim == 1:
+        y = y[None]
+    s = np.ascontiguousarray(scales, np.float32)
+    batch, out = y.shape
+    assert s.shape[0] == out
+    inn = 128 * s.shape[1]
+    nb = out // 64
+    lev = np.empty(nb, np.uint8)
+    red = np.empty(nb, np.float64)
+    rc = _load().orc_level_decide(_p(y), batch, out, _p(s), inn, int(gamma), int(kappa), int(rule), float(lam),
+                                  float(f), _p(lev), _p(red))
+    if rc != 0:
+        raise ValueError(f"orc_level_decide: bad arguments ({rc})")
+    return lev, red
 
 
 def memory_bits(levels, wb, bits_of_level) -> float:

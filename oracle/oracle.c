@@ -338,6 +338,87 @@ ORC_API double orc_memory_bits(const uint8_t* levels, int nblocks, const double*
 }
 
 /* ------------------------------------------------------------------------ */
+/* In-pass level decision ([FoQLens landing], FoQZones mechanism: the layer  */
+/* decides for itself from what entered it; score, reduced score, ladder     */
+/* level capped at kappa, or the top share f by reduced score).              */
+/*                                                                           */
+/* Of the three scores the page tries, this is the draft one: the layer read */
+/* at the base shows which units carry the step.                             */
+/*   unit c        one 64-row block of the layer (the unit the store reads   */
+/*                 at one depth)                                              */
+/*   s_c           = ||y_c(base)||^2 * D_c^2: squares of the block's base-    */
+/*                 level outputs, summed over its 64 rows and every row of    */
+/*                 the batch                                                  */
+/*   D_c^2         the block's squared quantization step at the base level,   */
+/*                 (s[r][g] 2^(8 - bits(gamma)))^2 averaged over its rows r    */
+/*                 and column groups g                                        */
+/*   reduced       r_c = s_c * D_c^2 / w_c, w_c = 64 * in weights             */
+/*   rule 0 ladder level = gamma + #{ j >= 1 : r_c >= lambda 16^j }, at most  */
+/*                 kappa                                                      */
+/*   rule 1 share  the floor(f * nblocks) blocks of largest r_c rise to       */
+/*                 kappa (equal scores: the lower block index first); the     */
+/*                 rest stay at gamma                                         */
+/* Readings: the page leaves the score open; the draft variant is the one    */
+/* that needs only the pass itself. The formula is taken as printed (D_c^2   */
+/* enters the score and again the reduction). A "rise" in the share rule     */
+/* goes to the cap kappa. 1 <= gamma <= kappa <= 4 (a ZERO base has no        */
+/* draft). Everything in double.                                              */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  double r;
+  int idx;
+} orc_scored;
+
+static int orc_scored_desc(const void* a, const void* b) {
+  const orc_scored* x = (const orc_scored*)a;
+  const orc_scored* y = (const orc_scored*)b;
+  if (x->r > y->r) return -1;
+  if (x->r < y->r) return 1;
+  return (x->idx > y->idx) - (x->idx < y->idx);
+}
+
+ORC_API int orc_level_decide(const float* y, int batch, int out, const float* s, int in, int gamma, int kappa,
+                             int rule, double lambda, double f, uint8_t* levels, double* reduced) {
+  if (gamma < 1 || kappa < gamma || kappa > 4 || out % 64 || in % 128 || (rule != 0 && rule != 1)) return -1;
+  const int nb = out / 64, G = in / 128;
+  const double step = ldexp(1.0, 8 - level_bits((uint8_t)gamma));
+  orc_scored* order = (orc_scored*)malloc(sizeof(orc_scored) * (size_t)(nb > 0 ? nb : 1));
+  if (!order) return -2;
+  for (int c = 0; c < nb; ++c) {
+    double yy = 0.0;
+    for (int t = 0; t < batch; ++t)
+      for (int r = 64 * c; r < 64 * c + 64; ++r) yy += (double)y[(size_t)t * out + r] * (double)y[(size_t)t * out + r];
+    double d2 = 0.0;
+    for (int r = 64 * c; r < 64 * c + 64; ++r)
+      for (int g = 0; g < G; ++g) {
+        double dl = (double)s[(size_t)r * G + g] * step;
+        d2 += dl * dl;
+      }
+    d2 /= 64.0 * G;
+    const double score = yy * d2;
+    const double red = score * d2 / (64.0 * in);
+    if (reduced) reduced[c] = red;
+    order[c].r = red;
+    order[c].idx = c;
+    int lev = gamma;
+    if (rule == 0) {
+      for (int j = 1; j <= kappa - gamma; ++j)
+        if (red >= lambda * ldexp(1.0, 4 * j)) lev += 1;
+    }
+    levels[c] = (uint8_t)lev;
+  }
+  if (rule == 1) {
+    int n_up = (int)floor(f * (double)nb);
+    if (n_up > nb) n_up = nb;
+    if (n_up < 0) n_up = 0;
+    qsort(order, (size_t)nb, sizeof(orc_scored), orc_scored_desc);
+    for (int k = 0; k < n_up; ++k) levels[order[k].idx] = (uint8_t)kappa;
+  }
+  free(order);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Uncertainty gate ([Precision on Demand]: entropy above a threshold or a   */
 /* small top-two margin). Readings: entropy of softmax(z) in nats; margin is  */
 /* the probability gap p1 - p2 of the two largest logits; ties go to the     */

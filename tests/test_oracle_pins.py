@@ -420,3 +420,88 @@ def test_kquant_step_bytes_match_published_footprint():
     assert sum(1 for *_, t in mix if t == synth.Q6_K) == 17
     total = sum(o * i // 256 * synth.RECORD_BYTES[t] for _, o, i, t in mix)
     assert round(total / 1e6, 1) == 799.6
+
+
+# ----------------------------------------------------------------------------- in-pass level decision
+
+def _decide_layer(gd):
+    L = gd["layer"]
+    out, inn, batch = L["out"], L["in"], L["batch"]
+    y = np.zeros((batch, out), np.float32)
+    s = np.zeros((out, inn // 128), np.float32)
+    for c, b in enumerate(L["blocks"]):
+        rows = slice(64 * c, 64 * c + 64)
+        s[rows, 0], s[rows, 1] = b["scale_group0"], b["scale_group1"]
+        y[0, rows], y[1, rows] = b["y_batch0"], b["y_batch1"]
+    return y, s
+
+
+def test_level_decide_hand_worked(orc, golden):
+    gd = golden("level_decide_hand.json")
+    E = gd["expect"]
+    y, s = _decide_layer(gd)
+    lev, red = orc.level_decide(y, s, 2, 4, 0, lam=2.0 ** -14)
+    assert red.tolist() == E["reduced_gamma2"]
+    assert lev.tolist() == E["ladder_gamma2_kappa4_lambda2e-14"]
+    assert orc.level_decide(y, s, 2, 3, 0, lam=2.0 ** -14)[0].tolist() == E["ladder_gamma2_kappa3_lambda2e-14"]
+    for f, key in ((0.5, "share_gamma2_kappa4_f0.5"), (0.7, "share_gamma2_kappa4_f0.7"), (1.0, "share_gamma2_kappa4_f1.0")):
+        assert orc.level_decide(y, s, 2, 4, 1, f=f)[0].tolist() == E[key], f
+    assert orc.level_decide(y, s, 1, 4, 0, lam=1.0)[1][0] == E["reduced_gamma1_block0"]
+
+
+def test_level_decide_ties_go_to_lower_index(orc):
+    y = np.ones((1, 256), np.float32)
+    s = np.full((256, 1), 0.01, np.float32)
+    lev, red = orc.level_decide(y, s, 2, 4, 1, f=0.5)          # 4 equal scores, 2 rise
+    assert len(set(red.tolist())) == 1
+    assert lev.tolist() == [4, 4, 2, 2]
+
+
+def test_level_decide_invariants(orc):
+    g = np.random.default_rng(7)
+    out, inn, batch = 64 * 40, 512, 3
+    y = g.standard_normal((batch, out)).astype(np.float32) * g.uniform(0.1, 10, out).astype(np.float32)
+    s = g.uniform(1e-4, 1e-2, (out, inn // 128)).astype(np.float32)
+    lev_prev = None
+    _, red = orc.level_decide(y, s, 1, 4, 0, lam=1.0)
+    for lam in np.geomspace(red.max() * 1e3, red.min() * 1e-6, 12):
+        lev, red2 = orc.level_decide(y, s, 1, 4, 0, lam=lam)
+        assert np.array_equal(red, red2)
+        assert lev.min() >= 1 and lev.max() <= 4
+        if lev_prev is not None:
+            assert np.all(lev >= lev_prev)                          # a lower lambda never lowers a level
+        lev_prev = lev
+    assert np.all(lev_prev == 4)                                    # lambda far below every score: all at kappa
+    # the reduced score is additive over batch rows
+    parts = sum(orc.level_decide(y[t:t + 1], s, 2, 4, 0, lam=1.0)[1] for t in range(batch))
+    assert np.allclose(orc.level_decide(y, s, 2, 4, 0, lam=1.0)[1], parts, rtol=1e-12)
+    # y x 2^a, s x 2^b scales r by 2^(2a + 4b) exactly; the ladder moves with lambda
+    lam = float(np.median(red)) * 4
+    base = orc.level_decide(y, s, 2, 4, 0, lam=lam)
+    scaled = orc.level_decide(y * np.float32(4), s * np.float32(0.5), 2, 4, 0, lam=lam * 2.0 ** (4 - 4))
+    assert np.array_equal(scaled[1], base[1] * 2.0 ** (4 - 4))
+    assert np.array_equal(scaled[0], base[0])
+    y2 = orc.level_decide(y * np.float32(2), s, 2, 4, 0, lam=lam * 4)
+    assert np.array_equal(y2[1], base[1] * 4) and np.array_equal(y2[0], base[0])
+    s2 = orc.level_decide(y, s * np.float32(2), 2, 4, 0, lam=lam * 16)
+    assert np.array_equal(s2[1], base[1] * 16) and np.array_equal(s2[0], base[0])
+    # share: exactly floor(f nb) rise, each lifted score >= every other
+    for f in (0.0, 0.1, 0.16, 0.5, 0.99, 1.0):
+        lev, r = orc.level_decide(y, s, 2, 3, 1, f=f)
+        up = lev == 3
+        assert up.sum() == int(np.floor(f * (out // 64)))
+        assert set(np.unique(lev).tolist()) <= {2, 3}
+        if 0 < up.sum() < len(up):
+            assert r[up].min() >= r[~up].max()
+
+
+def test_level_decide_degenerate(orc):
+    y = np.ones((1, 128), np.float32)
+    s = np.full((128, 2), 0.5, np.float32)
+    assert orc.level_decide(y, s, 3, 3, 0, lam=0.0)[0].tolist() == [3, 3]        # kappa = gamma: no rungs
+    assert orc.level_decide(y, s, 3, 3, 1, f=1.0)[0].tolist() == [3, 3]
+    assert orc.level_decide(y * 0, s, 2, 4, 0, lam=1e-30)[0].tolist() == [2, 2]   # zero draft stays at base
+    assert orc.level_decide(y * 0, s, 2, 4, 0, lam=0.0)[0].tolist() == [4, 4]     # 0 >= 0 at every rung
+    for bad in ((0, 4), (3, 2), (2, 5)):
+        with pytest.raises(ValueError):
+            orc.level_decide(y, s, bad[0], bad[1], 0, lam=1.0)

@@ -329,6 +329,71 @@ def kquant_step(torch, fl):
     return items, keep, nbytes
 
 
+def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
+    """The decode step with the in-pass level decision instead of the gate: the D4 pass, the
+    share rule (the draft score's top f of every layer's blocks rise to D8), then the residual
+    pass from D4 to the decided levels. One graph holds the 25 input sets' steps in order."""
+    import numpy as np
+    n, NS = step.n, step.NSETS
+    tot_out = step.y.numel()
+    lv_to, score, dec_items, res_items = [], [], [], [[] for _ in range(NS)]
+    oo = oi = 0
+    lifted = bytes_res = bytes_scales = 0
+    for k, (name, o, i) in enumerate(step.shapes):
+        t = torch.empty(o // 64, dtype=torch.uint8, device="cuda")
+        c = torch.empty(o // 64, dtype=torch.float32, device="cuda")
+        lv_to.append(t)
+        score.append(c)
+        ys = step.y[oo:oo + o]
+        dec_items.append((step.stores[k], o, i, ys, t, c))
+        for j in range(NS):
+            res_items[j].append((step.stores[k], o, i, step.levels[2 * k], t, step.xs[j, oi:oi + i], ys))
+        up = int(np.floor(np.float64(np.float32(f)) * (o // 64)))    # the kernel's count of rising blocks
+        lifted += up
+        bytes_res += up * (256 * (i // 128) + 2048 * (i // 128) * 2)
+        bytes_scales += (o // 64) * 256 * (i // 128)
+        oo += o
+        oi += i
+    assert oo == tot_out
+    dec = fl.decide_problems(dec_items)
+    params = fl.decide_params(fl.FL_DECIDE_SHARE, 2, 4, 0.0, f)
+    res = [fl.gemv_problems(it) for it in res_items]
+
+    def one(j):
+        fl.fl_gemv_batched(step.prob_d4[j], n, 1, 0)
+        fl.fl_level_decide(dec, n, 1, params)
+        fl.fl_gemv_batched(res[j], n, 1, 1)
+
+    for j in range(NS):
+        one(j)
+    torch.cuda.synchronize()
+    got = sum(int((t > 2).sum().item()) for t in lv_to)
+    g_all, g_dec, g_res = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all):
+        for j in range(NS):
+            one(j)
+    with torch.cuda.graph(g_dec):
+        for j in range(NS):
+            fl.fl_level_decide(dec, n, 1, params)
+    with torch.cuda.graph(g_res):                  # the residual passes alone, last decided levels
+        for j in range(NS):
+            fl.fl_gemv_batched(res[j], n, 1, 1)
+    for _ in range(3):
+        g_all.replay()
+        g_dec.replay()
+        g_res.replay()
+    t = time_loop(torch, lambda k: g_all.replay(), rounds) / (rounds * NS)
+    td = time_loop(torch, lambda k: g_dec.replay(), rounds) / (rounds * NS)
+    tr = time_loop(torch, lambda k: g_res.replay(), rounds) / (rounds * NS)
+    nbytes = step.bytes_d4 + bytes_res
+    return {"f": f, "lifted_blocks": got, "lifted_expected": lifted, "us_per_step": t * 1e6,
+            "bytes_per_step": nbytes, "GBps": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
+            "tokens_per_s": 1.0 / t, "decide_us": td * 1e6, "residual_us": tr * 1e6,
+            "residual_GBps": bytes_res / tr / 1e9,
+            "decide_bytes": bytes_scales + 4 * tot_out, "decide_GBps": (bytes_scales + 4 * tot_out) / td / 1e9,
+            "launches_per_step": 4}
+
+
 def extra_measurements(torch, fl, peak):
     """One line per other configuration: its kernel's weight-byte rate, timed over CUDA-graph replays
     with enough rotating copies of the weights that every replay reads past the 126 MB L2."""
@@ -610,7 +675,8 @@ def run_fl(args, rank, world, local_rank):
 
     extra = None
     if world == 1 and not args.no_extra:
-        extra = extra_measurements(torch, fl, peak)
+        extra = {"cfg1_in_pass_share_decision": in_pass_measurement(torch, fl, step, peak)}
+        extra.update(extra_measurements(torch, fl, peak))
 
     if rank != 0:
         return 0

@@ -270,6 +270,56 @@ FL_API fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, int n,
                                   void* stream);
 
 /* ========================================================================= */
+/* In-pass level decision ([FoQLens] FoQZones mechanism: the layer decides   */
+/* for itself from what entered it; the draft score, the reduced score, the  */
+/* ladder lambda 16^j capped at kappa, or the top share f).                   */
+/* For block c (64 rows) of a layer read at the base level gamma:            */
+/*   s_c = ||y_c||^2 D_c^2, y_c the block's base-level outputs over its 64    */
+/*         rows and every batch row;                                          */
+/*   D_c^2 = mean over the block's rows and 128-column groups of              */
+/*         (scale 2^(8 - 2 gamma))^2, the squared base quantization step;     */
+/*   r_c = s_c D_c^2 / (64 in)  (the reduced score; w_c = 64 in weights);     */
+/*   FL_DECIDE_LADDER: level = gamma + #{ j >= 1 : r_c >= lambda 16^j },      */
+/*         at most kappa;                                                     */
+/*   FL_DECIDE_SHARE: the floor(f * out / 64) blocks of largest r_c (equal    */
+/*         r_c: lower block index first) get kappa, the others gamma.         */
+/* The levels then drive the residual pass from gamma (fl_gemv_residual or    */
+/* fl_gemv_batched mode 1 with to_levels = these levels), so only the lifted  */
+/* blocks' low planes are read a second time. fp32 arithmetic: a decision can */
+/* differ from an exact one only when r_c lies within fp32 rounding of a      */
+/* threshold (or of another block's score, for the share rule).               */
+/*                                                                           */
+/* Per problem (one layer; all share `batch`, 1 <= n <= FL_MAX_PROBLEMS):     */
+/*   w       the layer's plane store (its scales are read), 16-byte aligned   */
+/*   y       device fp32 [batch][out], 8-byte aligned: the base-level outputs */
+/*   levels  device uint8 [out / 64], written                                 */
+/*   score   device fp32 [out / 64], written with r_c; may be NULL for the   */
+/*           ladder rule, required for the share rule                         */
+/* params: 1 <= gamma <= kappa <= 4; ladder: lambda finite, >= 0; share:     */
+/* 0 <= f <= 1. One launch (ladder) or two (share), asynchronous on stream.   */
+/* ========================================================================= */
+#define FL_DECIDE_LADDER 0
+#define FL_DECIDE_SHARE 1
+
+typedef struct {
+  fl_plane_weight w;
+  const float* y;
+  uint8_t* levels;
+  float* score;
+} fl_decide_problem;
+
+typedef struct {
+  int rule;
+  int gamma;
+  int kappa;
+  float lambda;
+  float f;
+} fl_decide_params;
+
+FL_API fl_status fl_level_decide(const fl_decide_problem* problems, int n, int batch, const fl_decide_params* params,
+                                 void* stream);
+
+/* ========================================================================= */
 /* Uncertainty gate ([PoD]: redo at 8 bits when the low-precision output     */
 /* distribution looks uncertain: entropy above a threshold or a small        */
 /* top-two margin).  Per row t of logits z:                                  */

@@ -100,6 +100,25 @@ def test_host_side_rejections(fl):
     kp = fl.kquant_problems([(16, 11, 64, 256, 16, 16)])
     assert _status(fl, fl.fl_gemv_kquant_batched, kp, 1, 1, s0) == ERR_UNSUP
     assert "Q4_K" in fl.fl_last_error()
+    # in-pass level decision
+    dp = fl.decide_problems([(16, 64, 128, 16, 16, None)])
+    lad = fl.decide_params(fl.FL_DECIDE_LADDER, 2, 4, lam=1.0)
+    assert _status(fl, fl.fl_level_decide, dp, 0, 1, lad, s0) == ERR_ARG                    # n = 0
+    assert _status(fl, fl.fl_level_decide, dp, 1, 17, lad, s0) == ERR_SHAPE                 # batch 17
+    for bad in ((fl.FL_DECIDE_LADDER, 0, 4, 1.0, 0.0), (fl.FL_DECIDE_LADDER, 3, 2, 1.0, 0.0),
+                (fl.FL_DECIDE_LADDER, 2, 5, 1.0, 0.0), (fl.FL_DECIDE_LADDER, 2, 4, -1.0, 0.0),
+                (fl.FL_DECIDE_LADDER, 2, 4, float("nan"), 0.0), (fl.FL_DECIDE_SHARE, 2, 4, 0.0, 1.5),
+                (fl.FL_DECIDE_SHARE, 2, 4, 0.0, 0.5), (2, 2, 4, 0.0, 0.0)):
+        # the share rule also needs a score array, which dp lacks
+        assert _status(fl, fl.fl_level_decide, dp, 1, 1, fl.decide_params(*bad), s0) == ERR_ARG, bad
+    dp = fl.decide_problems([(16, 64, 100, 16, 16, None)])
+    assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == ERR_SHAPE                  # in % 128
+    dp = fl.decide_problems([(16, 64, 128, None, 16, None)])
+    assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == ERR_ARG                    # NULL y
+    dp = fl.decide_problems([(16, 64, 128, 20, 16, None)])
+    assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == -4                         # y not 8-aligned
+    dp = fl.decide_problems([(24, 64, 128, 16, 16, None)])
+    assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == -4                         # store not 16-aligned
 
 
 def test_misaligned_pointers_rejected(fl):

@@ -1,0 +1,222 @@
+"""In-pass level decision on the GPU vs the oracle, through the C-ABI.
+
+The decision reads the base-level outputs of the layer, which both sides take from the
+same buffer (the GPU's base pass), and the layer's scales. Bars: reduced scores within
+1e-5 relative; ladder levels equal to the oracle's except where the oracle's score lies
+within 1e-4 (relative) of a threshold lambda 16^j, and always equal to the ladder applied
+to the kernel's own fp32 scores; share levels equal to the top floor(f n) blocks by the
+kernel's own scores (lower index first on ties), and to the oracle's set except where
+scores at the cut lie within 1e-4 of each other.
+"""
+import numpy as np
+import pytest
+
+from variable_precision_weight_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2e-3, 1e-5
+BAND = 1e-4
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from variable_precision_weight_b200 import build
+    build.build()
+    from variable_precision_weight_b200 import fl
+    return torch, fl
+
+
+def dev(torch, a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def pack_gpu(torch, fl, q, s):
+    out, inn = q.shape
+    store = torch.empty(fl.fl_plane_store_bytes(out, inn), dtype=torch.uint8, device="cuda")
+    fl.fl_pack_planes(dev(torch, q), dev(torch, s), out, inn, store)
+    return store
+
+
+def ladder_of(score, gamma, kappa, lam):
+    """The ladder applied in fp32 to the kernel's own scores."""
+    sc = np.asarray(score, np.float32)
+    lev = np.full(sc.shape, gamma, np.int64)
+    thr = np.float32(lam)
+    for _ in range(kappa - gamma):
+        thr = np.float32(thr * np.float32(16))
+        lev += sc >= thr
+    return lev.astype(np.uint8)
+
+
+def share_of(score, gamma, kappa, f):
+    sc = np.asarray(score, np.float32)
+    nb = len(sc)
+    n_up = int(np.floor(np.float64(np.float32(f)) * nb))
+    order = np.lexsort((np.arange(nb), -sc.astype(np.float64)))
+    lev = np.full(nb, gamma, np.uint8)
+    lev[order[:n_up]] = kappa
+    return lev
+
+
+def check_ladder(lev, score, ref_lev, ref_red, gamma, kappa, lam, what):
+    assert np.allclose(score, ref_red, rtol=1e-5, atol=0), what
+    assert np.array_equal(lev, ladder_of(score, gamma, kappa, lam)), what
+    thr = np.float64(np.float32(lam)) * 16.0 ** np.arange(1, kappa - gamma + 1)
+    near = np.zeros(len(ref_red), bool)
+    for t in thr:
+        near |= np.abs(ref_red - t) <= BAND * t
+    assert np.array_equal(lev[~near], ref_lev[~near]), what
+
+
+def check_share(lev, score, ref_lev, ref_red, gamma, kappa, f, what):
+    assert np.allclose(score, ref_red, rtol=1e-5, atol=0), what
+    assert np.array_equal(lev, share_of(score, gamma, kappa, f)), what
+    up, ref_up = lev == kappa, ref_lev == kappa
+    assert up.sum() == ref_up.sum(), what
+    diff = up != ref_up
+    if diff.any():
+        cut = np.sort(ref_red)[::-1][up.sum() - 1]
+        assert np.all(np.abs(ref_red[diff] - cut) <= BAND * cut), what
+
+
+def base_layers(torch, fl, shapes, gamma, batch, key):
+    """Packed layers, their base-level pass (one batched launch) and the host copies."""
+    items, host, keep = [], [], []
+    for i, (o, n) in enumerate(shapes):
+        q, s = synth.int8_layer(o, n, key, i)
+        s = s * synth.rng(key, 50 + i).uniform(0.25, 4.0, (o // 64, 1, 1)).astype(np.float32).repeat(64, 1).reshape(o, -1)
+        x = synth.bf16_normal((batch, n), key, 100 + i)
+        st = pack_gpu(torch, fl, q, s)
+        lv = torch.full((o // 64,), gamma, dtype=torch.uint8, device="cuda")
+        xd = dev(torch, x)
+        y = torch.empty((batch, o), dtype=torch.float32, device="cuda")
+        keep += [st, lv, xd, y]
+        items.append((st, o, n, lv, None, xd, y))
+        host.append((q, s, x))
+    fl.fl_gemv_batched(fl.gemv_problems(items), len(items), batch, 0)
+    return items, host, keep
+
+
+@pytest.mark.parametrize("gamma,batch", [(1, 1), (2, 1), (2, 3), (3, 16)])
+def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
+    torch, fl = env
+    shapes = [(64 * 37, 384), (1024, 1024), (2048, 1024), (64, 128)]
+    items, host, keep = base_layers(torch, fl, shapes, gamma, batch, 300 + gamma + batch)
+    torch.cuda.synchronize()
+    kappa = 4
+    ys = [it[6].cpu().numpy() for it in items]
+    refs = [orc.level_decide(y, s, gamma, kappa, 0, lam=1.0)[1] for y, (q, s, x) in zip(ys, host)]
+    allr = np.concatenate(refs)
+    lam = float(np.median(allr)) / 16 / 2            # about half lifted once, some twice
+    lv_out = [torch.empty(o // 64, dtype=torch.uint8, device="cuda") for o, _ in shapes]
+    sc_out = [torch.empty(o // 64, dtype=torch.float32, device="cuda") for o, _ in shapes]
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], lv, sc) for it, lv, sc in zip(items, lv_out, sc_out)])
+    for rule, lam_, f in ((fl.FL_DECIDE_LADDER, lam, 0.0), (fl.FL_DECIDE_LADDER, 0.0, 0.0),
+                          (fl.FL_DECIDE_LADDER, 1e30, 0.0), (fl.FL_DECIDE_SHARE, 0.0, 0.0),
+                          (fl.FL_DECIDE_SHARE, 0.0, 0.16), (fl.FL_DECIDE_SHARE, 0.0, 0.5),
+                          (fl.FL_DECIDE_SHARE, 0.0, 1.0)):
+        fl.fl_level_decide(probs, len(shapes), batch, fl.decide_params(rule, gamma, kappa, lam_, f))
+        torch.cuda.synchronize()
+        for i, (y, (q, s, x)) in enumerate(zip(ys, host)):
+            lev, sc = lv_out[i].cpu().numpy(), sc_out[i].cpu().numpy()
+            ref_lev, ref_red = orc.level_decide(y, s, gamma, kappa, rule, lam=lam_, f=np.float32(f))
+            what = f"rule {rule} lam {lam_} f {f} problem {i}"
+            if rule == fl.FL_DECIDE_LADDER:
+                check_ladder(lev, sc, ref_lev, ref_red, gamma, kappa, lam_, what)
+            else:
+                check_share(lev, sc, ref_lev, ref_red, gamma, kappa, f, what)
+    # ladder without a score array: the same levels as the ladder over the scores just written
+    # (the same fp32 computation), and the oracle's outside the band
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], lv, None) for it, lv in zip(items, lv_out)])
+    fl.fl_level_decide(probs, len(shapes), batch, fl.decide_params(fl.FL_DECIDE_LADDER, gamma, kappa, lam))
+    torch.cuda.synchronize()
+    for i, (y, (q, s, x)) in enumerate(zip(ys, host)):
+        lev, sc = lv_out[i].cpu().numpy(), sc_out[i].cpu().numpy()
+        ref_lev, ref_red = orc.level_decide(y, s, gamma, kappa, 0, lam=lam)
+        check_ladder(lev, sc, ref_lev, ref_red, gamma, kappa, lam, f"no-score ladder problem {i}")
+
+
+def test_share_ties_go_to_lower_index(env, orc):
+    """Identical blocks give bit-identical scores; the share lifts the lowest indices."""
+    torch, fl = env
+    o, n = 64 * 10, 256
+    q1, s1 = synth.int8_layer(64, n, 61)
+    q, s = np.tile(q1, (10, 1)), np.tile(s1, (10, 1))
+    st = pack_gpu(torch, fl, q, s)
+    y = torch.from_numpy(np.tile(synth.rng(62).standard_normal(64).astype(np.float32), (2, 10))).cuda()
+    lv = torch.empty(10, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(10, dtype=torch.float32, device="cuda")
+    fl.fl_level_decide(fl.decide_problems([(st, o, n, y, lv, sc)]), 1, 2,
+                       fl.decide_params(fl.FL_DECIDE_SHARE, 2, 3, f=0.35))
+    torch.cuda.synchronize()
+    assert len(set(sc.cpu().numpy().tolist())) == 1
+    assert lv.cpu().numpy().tolist() == [3, 3, 3] + [2] * 7
+    assert np.array_equal(orc.level_decide(y.cpu().numpy(), s, 2, 3, 1, f=np.float32(0.35))[0],
+                          lv.cpu().numpy())
+
+
+@pytest.mark.parametrize("rule", [0, 1])
+def test_in_pass_pipeline(env, orc, rule):
+    """Base pass at D4 -> decision -> residual pass from D4 to the decided levels, all layers
+    in one launch each: y equals the oracle's depth GEMV at the decided levels."""
+    torch, fl = env
+    gamma, kappa, batch = 2, 4, 1
+    shapes = [(1024, 1024), (3072, 1024), (1024, 3072), (64 * 37, 384)]
+    items, host, keep = base_layers(torch, fl, shapes, gamma, batch, 400 + rule)
+    torch.cuda.synchronize()
+    ys = [it[6].cpu().numpy() for it in items]
+    allr = np.concatenate([orc.level_decide(y, s, gamma, kappa, 0, lam=1.0)[1] for y, (q, s, x) in zip(ys, host)])
+    lam = float(np.quantile(allr, 0.84)) / 16        # about 16% lifted at least one rung
+    to = [torch.empty(o // 64, dtype=torch.uint8, device="cuda") for o, _ in shapes]
+    sc = [torch.empty(o // 64, dtype=torch.float32, device="cuda") for o, _ in shapes]
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c) for it, t, c in zip(items, to, sc)])
+    params = fl.decide_params(rule, gamma, kappa, lam, 0.16)
+    fl.fl_level_decide(probs, len(shapes), batch, params)
+    res = [(it[0], it[1], it[2], it[3], t, it[5], it[6]) for it, t in zip(items, to)]
+    fl.fl_gemv_batched(fl.gemv_problems(res), len(res), batch, 1)
+    torch.cuda.synchronize()
+    lifted = 0
+    for i, ((q, s, x), it, t, c, y0) in enumerate(zip(host, items, to, sc, ys)):
+        lev = t.cpu().numpy()
+        ref_lev, ref_red = orc.level_decide(y0, s, gamma, kappa, rule, lam=lam, f=np.float32(0.16))
+        if rule == 0:
+            check_ladder(lev, c.cpu().numpy(), ref_lev, ref_red, gamma, kappa, lam, f"pipeline problem {i}")
+        else:
+            check_share(lev, c.cpu().numpy(), ref_lev, ref_red, gamma, kappa, 0.16, f"pipeline problem {i}")
+        lifted += int((lev > gamma).sum())
+        yref, mass = orc.gemv_depth(q, s, lev, x, with_mass=True)
+        err = np.abs(it[6].cpu().numpy().astype(np.float64) - yref)
+        assert np.all(err <= REL * mass + ABS), f"pipeline y, problem {i}"
+    assert lifted > 0
+
+
+def test_share_rule_on_a_layer_too_large_for_shared_memory(env, orc):
+    """A layer of 12,000 blocks: the selection reads the scores from global memory."""
+    torch, fl = env
+    o, n = 64 * 12000, 128
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(77)
+    q = torch.randint(-127, 128, (o, n), dtype=torch.int8, device="cuda", generator=gen)
+    s = torch.rand((o, 1), device="cuda", generator=gen).mul_(1e-2)
+    s[64 * 100:64 * 140] = s[0:64].repeat(40, 1)          # 41 blocks with equal scales ...
+    y = torch.randn((1, o), device="cuda", generator=gen)
+    y[:, 64 * 100:64 * 140] = y[:, 0:64].repeat(1, 40)    # ... and equal outputs: equal scores
+    st = torch.empty(fl.fl_plane_store_bytes(o, n), dtype=torch.uint8, device="cuda")
+    fl.fl_pack_planes(q, s, o, n, st)
+    lv = torch.empty(o // 64, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(o // 64, dtype=torch.float32, device="cuda")
+    ref_red = orc.level_decide(y.cpu().numpy(), s.cpu().numpy(), 2, 4, 0, lam=1.0)[1]
+    rank0 = int((ref_red > ref_red[0]).sum())             # blocks scoring above the tied group
+    for f in (0.25, (rank0 + 20) / 12000, 0.999):          # the second cuts the tied group
+        fl.fl_level_decide(fl.decide_problems([(st, o, n, y, lv, sc)]), 1, 1,
+                           fl.decide_params(fl.FL_DECIDE_SHARE, 2, 4, f=f))
+        torch.cuda.synchronize()
+        ref_lev, ref_red = orc.level_decide(y.cpu().numpy(), s.cpu().numpy(), 2, 4, 1, f=np.float32(f))
+        check_share(lv.cpu().numpy(), sc.cpu().numpy(), ref_lev, ref_red, 2, 4, f, f"large layer f {f}")

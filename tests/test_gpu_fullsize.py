@@ -206,3 +206,59 @@ def test_kquant_step_full_size(env, orc):
             ys[k] = y.cpu().numpy()
         yref, mass = orc.gemv_kquant(recs, t, 64, i, x.cpu().numpy().view(np.uint16), with_mass=True)
         _check(ys[k][:, 64 * b:64 * b + 64], yref, mass, f"K-quant type {t} {o}x{i} block {b}")
+
+
+def test_in_pass_decision_full_size(env, orc):
+    """The decode step read at D4, the in-pass decision over all 197 layers' 7,750 blocks in
+    one call (checked on every block), then the residual pass from D4 to the decided levels
+    (checked on sampled and on lifted blocks)."""
+    torch, fl = env
+    import test_gpu_decide as dec
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(6060)
+    items, qs, ss, keep = [], [], [], []
+    for name, o, i in synth.qwen3_step_shapes():
+        q, s = _int8_layer(torch, o, i, gen)
+        s.mul_(torch.rand((o // 64, 1), device="cuda", generator=gen).mul_(3.75).add_(0.25).repeat_interleave(64, 0))
+        st = torch.empty(fl.fl_plane_store_bytes(o, i), dtype=torch.uint8, device="cuda")
+        fl.fl_pack_planes(q, s, o, i, st)
+        lv = torch.full((o // 64,), 2, dtype=torch.uint8, device="cuda")
+        x = _x(torch, 1, i, gen)
+        y = torch.empty((1, o), dtype=torch.float32, device="cuda")
+        keep += [st, lv, x, y]
+        items.append((st, o, i, lv, None, x, y))
+        qs.append(q)
+        ss.append(s.cpu().numpy())
+    n = len(items)
+    fl.fl_gemv_batched(fl.gemv_problems(items), n, 1, 0)
+    torch.cuda.synchronize()
+    ys = [it[6].cpu().numpy() for it in items]
+    to = [torch.empty(it[1] // 64, dtype=torch.uint8, device="cuda") for it in items]
+    sc = [torch.empty(it[1] // 64, dtype=torch.float32, device="cuda") for it in items]
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c) for it, t, c in zip(items, to, sc)])
+    allr = np.concatenate([orc.level_decide(y, s, 2, 4, 0, lam=1.0)[1] for y, s in zip(ys, ss)])
+    lam = float(np.quantile(allr, 0.84)) / 16
+    for rule, f in ((fl.FL_DECIDE_LADDER, 0.0), (fl.FL_DECIDE_SHARE, 0.16)):
+        fl.fl_level_decide(probs, n, 1, fl.decide_params(rule, 2, 4, lam, f))
+        torch.cuda.synchronize()
+        for k, (y, s, t, c) in enumerate(zip(ys, ss, to, sc)):
+            ref_lev, ref_red = orc.level_decide(y, s, 2, 4, rule, lam=lam, f=np.float32(f))
+            lev, score = t.cpu().numpy(), c.cpu().numpy()
+            if rule == fl.FL_DECIDE_LADDER:
+                dec.check_ladder(lev, score, ref_lev, ref_red, 2, 4, lam, f"step ladder, problem {k}")
+            else:
+                dec.check_share(lev, score, ref_lev, ref_red, 2, 4, f, f"step share, problem {k}")
+    res = [(it[0], it[1], it[2], it[3], t, it[5], it[6]) for it, t in zip(items, to)]
+    fl.fl_gemv_batched(fl.gemv_problems(res), n, 1, 1)
+    torch.cuda.synchronize()
+    lifted = 0
+    for k, (it, t, q, s) in enumerate(zip(items, to, qs, ss)):
+        lev = t.cpu().numpy()
+        up = np.flatnonzero(lev > 2)
+        lifted += len(up)
+        blocks = sorted(set(_sample_blocks(len(lev))) | set(up[:2].tolist()))
+        rows = np.concatenate([np.arange(64 * b, 64 * b + 64) for b in blocks])
+        yref, mass = orc.gemv_depth(q[rows].cpu().numpy(), s[rows], lev[blocks], it[5].cpu().numpy().view(np.uint16),
+                                    with_mass=True)
+        _check(it[6].cpu().numpy()[:, rows], yref, mass, f"in-pass step, problem {k}")
+    assert lifted == sum(int(np.floor(np.float64(np.float32(0.16)) * (it[1] // 64))) for it in items)

@@ -61,6 +61,17 @@ class fl_kquant_problem(C.Structure):
                 ("x", C.c_void_p), ("y", C.c_void_p)]
 
 
+class fl_decide_problem(C.Structure):
+    _fields_ = [("w", fl_plane_weight), ("y", C.c_void_p), ("levels", C.c_void_p), ("score", C.c_void_p)]
+
+
+class fl_decide_params(C.Structure):
+    _fields_ = [("rule", C.c_int), ("gamma", C.c_int), ("kappa", C.c_int), ("lambda_", C.c_float), ("f", C.c_float)]
+
+
+FL_DECIDE_LADDER = 0
+FL_DECIDE_SHARE = 1
+
 _P, _I, _F, _S = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 _sigs = {
     "fl_status_string": (C.c_char_p, [_I]),
@@ -84,6 +95,7 @@ _sigs = {
     "fl_kquant_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "fl_gemv_kquant": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _S, _P]),
     "fl_gemv_kquant_batched": (_I, [C.POINTER(fl_kquant_problem), _I, _I, _P]),
+    "fl_level_decide": (_I, [C.POINTER(fl_decide_problem), _I, _I, C.POINTER(fl_decide_params), _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _fn = getattr(_lib, _name)
@@ -248,3 +260,20 @@ def kquant_problems(items) -> "C.Array":
 
 def fl_gemv_kquant_batched(problems, n: int, batch: int, stream=None) -> None:
     _check(_lib.fl_gemv_kquant_batched(problems, n, batch, _stream(stream)))
+
+
+def decide_problems(items) -> "C.Array":
+    """items: iterable of (store, out, in, y, levels, score or None) -> fl_decide_problem array."""
+    items = list(items)
+    arr = (fl_decide_problem * len(items))()
+    for i, (store, out, inn, y, lv, sc) in enumerate(items):
+        arr[i] = fl_decide_problem(fl_plane_weight(_ptr(store), out, inn), _ptr(y), _ptr(lv), _ptr(sc))
+    return arr
+
+
+def decide_params(rule: int, gamma: int, kappa: int, lam: float = 0.0, f: float = 0.0) -> fl_decide_params:
+    return fl_decide_params(rule, gamma, kappa, float(lam), float(f))
+
+
+def fl_level_decide(problems, n: int, batch: int, params: fl_decide_params, stream=None) -> None:
+    _check(_lib.fl_level_decide(problems, n, batch, C.byref(params), _stream(stream)))

@@ -59,6 +59,7 @@ def _load():
                 "orc_level_map": (None, [P, i, P, P, i, f, f, i, i, i, P, i, P]),
                 "orc_memory_bits": (d, [P, i, P, P]),
                 "orc_level_decide": (i, [P, i, i, P, i, i, i, i, d, d, P, P]),
+                "orc_spec_accept": (None, [P, P, i, P, P]),
                 "orc_logit_gate": (None, [P, i, i, d, d, P, P, P, P]),
                 "orc_dequant_q4k": (None, [P, P]),
                 "orc_dequant_q6k": (None, [P, i, P]),
@@ -189,6 +190,16 @@ def level_decide(y, scales, gamma: int, kappa: int, rule: int, lam: float = 0.0,
     if rc != 0:
         raise ValueError(f"orc_level_decide: bad arguments ({rc})")
     return lev, red
+
+
+def spec_accept(draft, verified):
+    """Greedy verified speculation over one window: (accepted, emitted)."""
+    dr = np.ascontiguousarray(draft, np.int32).reshape(-1)
+    vf = np.ascontiguousarray(verified, np.int32).reshape(-1)
+    assert dr.shape == vf.shape
+    a, e = np.zeros(1, np.int32), np.zeros(1, np.int32)
+    _load().orc_spec_accept(_p(dr), _p(vf), len(dr), _p(a), _p(e))
+    return int(a[0]), int(e[0])
 
 
 def memory_bits(levels, wb, bits_of_level) -> float:

@@ -456,6 +456,25 @@ ORC_API void orc_logit_gate(const float* logits, int vocab, int batch, double ta
 }
 
 /* ------------------------------------------------------------------------ */
+/* Verified speculation ([Precision on Demand], abstract: a low-precision     */
+/* draft verified at 8 bits, counted in the same weight-byte cost model).     */
+/* Readings: greedy speculation over a window of k steps. The draft token of  */
+/* step t is the argmax of its D4 logits, the verified token the argmax of    */
+/* its D8 logits (ties to the lower index, as the gate's top-2). The window   */
+/* accepts the longest prefix of steps whose draft token equals the verified  */
+/* one: accepted = a. It emits the verified tokens of steps 0..a (the a       */
+/* accepted drafts and, when a < k, the correction at step a), so emitted =   */
+/* min(a + 1, k) and the emitted sequence is the D8 model's own greedy one.   */
+/* ------------------------------------------------------------------------ */
+ORC_API void orc_spec_accept(const int32_t* draft, const int32_t* verified, int k, int32_t* accepted,
+                             int32_t* emitted) {
+  int a = 0;
+  while (a < k && draft[a] == verified[a]) ++a;
+  *accepted = a;
+  *emitted = a < k ? a + 1 : k;
+}
+
+/* ------------------------------------------------------------------------ */
 /* K-quant super-blocks ([Ember v0.3], GGUF layouts; dequantized per block    */
 /* inside the product). The value rules are GGUF's; the byte layout is our    */
 /* own with the GGUF byte counts (144 and 210 bytes per 256 weights).        */

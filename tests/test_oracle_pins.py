@@ -505,3 +505,41 @@ def test_level_decide_degenerate(orc):
     for bad in ((0, 4), (3, 2), (2, 5)):
         with pytest.raises(ValueError):
             orc.level_decide(y, s, bad[0], bad[1], 0, lam=1.0)
+
+
+# ----------------------------------------------------------------------------- verified speculation
+
+def test_spec_accept_hand_cases(orc):
+    assert orc.spec_accept([5, 6, 7, 8], [5, 6, 7, 8]) == (4, 4)      # every draft verified
+    assert orc.spec_accept([5, 6, 7, 8], [1, 6, 7, 8]) == (0, 1)      # first draft rejected: the correction only
+    assert orc.spec_accept([5, 6, 7, 8], [5, 6, 0, 8]) == (2, 3)      # later agreement does not count
+    assert orc.spec_accept([5, 6, 7, 8], [5, 6, 7, 0]) == (3, 4)
+    assert orc.spec_accept([3], [3]) == (1, 1)
+    assert orc.spec_accept([], []) == (0, 0)
+
+
+def test_spec_emits_the_d8_greedy_tokens(orc):
+    """Zero KL: whatever the drafts, the emitted tokens are the D8 argmax tokens of the
+    window's first steps, and a D4 draft that matches D8 everywhere is accepted whole."""
+    g = np.random.default_rng(11)
+    vocab, inn, k = 512, 256, 8
+    q, s = synth.int8_layer(vocab, inn, 12)
+    x = synth.bf16_normal((k, inn), 13)
+    lv4, lv8 = np.full(vocab // 64, 2, np.uint8), np.full(vocab // 64, 4, np.uint8)
+    d4 = orc.gemv_depth(q, s, lv4, x)
+    d8 = orc.gemv_depth(q, s, lv8, x)
+    draft = orc.logit_gate(d4.astype(np.float32), 0.0, 0.0)[2][:, 0]
+    verified = orc.logit_gate(d8.astype(np.float32), 0.0, 0.0)[2][:, 0]
+    assert np.array_equal(verified, np.argmax(d8, axis=1))
+    a, e = orc.spec_accept(draft, verified)
+    assert np.all(draft[:a] == verified[:a]) and (a == k or draft[a] != verified[a])
+    assert e == min(a + 1, k)
+    # a window whose drafts are replaced by the verified tokens is accepted whole
+    assert orc.spec_accept(verified, verified) == (k, k)
+    # with one row dominating every logit vector, D4 and D8 agree
+    q2 = q.copy()
+    q2[7] = 127
+    xp = synth.f32_to_bf16_bits(np.abs(synth.bf16_bits_to_f32(x)))
+    t4 = np.argmax(orc.gemv_depth(q2, s, lv4, xp), axis=1)
+    t8 = np.argmax(orc.gemv_depth(q2, s, lv8, xp), axis=1)
+    assert np.all(t8 == 7) and orc.spec_accept(t4, t8) == (k, k)

@@ -394,6 +394,66 @@ def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
             "launches_per_step": 4}
 
 
+def spec_measurement(torch, fl, step, peak, K=4, rounds=20):
+    """Verified speculation on the decode step: windows of K steps, each K gated D4 draft passes
+    (batch 1), one gated residual pass at batch K over the window (the D8 logits of all K steps
+    from one read of the low planes) and the acceptance, on the device. The 25 input sets give
+    25 // K windows, one graph."""
+    n, W = step.n, step.NSETS // K
+    wins = []
+    for w in range(W):
+        items_d, items_v, keep = [[] for _ in range(K)], [], []
+        oi = 0
+        for k, (name, o, i) in enumerate(step.shapes):
+            x = torch.empty((K, i), dtype=torch.int16, device="cuda")
+            for t in range(K):
+                x[t].copy_(step.xs[w * K + t, oi:oi + i])
+            y = torch.empty((K, o), dtype=torch.float32, device="cuda")
+            keep += [x, y]
+            d4, d8 = step.levels[2 * k], step.levels[2 * k + 1]
+            for t in range(K):
+                items_d[t].append((step.stores[k], o, i, d4, None, x[t], y[t]))
+            items_v.append((step.stores[k], o, i, d4, d8, x, y))
+            oi += i
+        wsb = fl.fl_gemv_gate_workspace_bytes(K)
+        g = {"ws": torch.zeros(wsb, dtype=torch.uint8, device="cuda"),
+             "ent": torch.empty(K, dtype=torch.float32, device="cuda"),
+             "mar": torch.empty(K, dtype=torch.float32, device="cuda"),
+             "esc": torch.empty(K, dtype=torch.uint8, device="cuda"),
+             "dtop": torch.empty((K, 2), dtype=torch.int32, device="cuda"),
+             "vtop": torch.empty((K, 2), dtype=torch.int32, device="cuda"),
+             "res": torch.empty(2, dtype=torch.int32, device="cuda")}
+        specs = [fl.gate_spec(n - 1, step.tau_h, step.tau_m, g["ent"][t:t + 1], g["mar"][t:t + 1], g["dtop"][t],
+                              g["esc"][t:t + 1], g["ws"], wsb) for t in range(K)]
+        spec_v = fl.gate_spec(n - 1, step.tau_h, step.tau_m, g["ent"], g["mar"], g["vtop"], g["esc"], g["ws"], wsb)
+        wins.append((g, keep, [fl.gemv_problems(it) for it in items_d], fl.gemv_problems(items_v), specs, spec_v))
+    totals = torch.zeros(2, dtype=torch.int32, device="cuda")
+
+    def all_windows():
+        for g, keep, pd, pv, specs, spec_v in wins:
+            for t in range(K):
+                fl.fl_gemv_batched_gate(pd[t], n, 1, 0, specs[t])
+            fl.fl_gemv_batched_gate(pv, n, K, 1, spec_v)
+            fl.fl_spec_accept(g["dtop"], g["vtop"], K, g["res"], totals)
+
+    all_windows()
+    torch.cuda.synchronize()
+    acc, emi = (int(v) for v in totals.cpu().tolist())
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        all_windows()
+    for _ in range(3):
+        gr.replay()
+    t = time_loop(torch, lambda k: gr.replay(), rounds) / rounds
+    bytes_round = W * (K * step.bytes_d4 + step.bytes_res)
+    d8_per_token = sum((o // 64) * plane_bytes(i, 4) for _, o, i in step.shapes)
+    return {"k": K, "windows": W, "accepted": acc, "emitted": emi, "us_per_window": t / W * 1e6,
+            "tokens_per_s": emi / t, "bytes_per_emitted_token": bytes_round / emi,
+            "vs_all_d8_bytes_per_token": bytes_round / emi / d8_per_token,
+            "GBps": bytes_round / t / 1e9, "frac": bytes_round / t / 1e9 / peak,
+            "launches_per_window": K + 2}
+
+
 def extra_measurements(torch, fl, peak):
     """One line per other configuration: its kernel's weight-byte rate, timed over CUDA-graph replays
     with enough rotating copies of the weights that every replay reads past the 126 MB L2."""
@@ -675,7 +735,8 @@ def run_fl(args, rank, world, local_rank):
 
     extra = None
     if world == 1 and not args.no_extra:
-        extra = {"cfg1_in_pass_share_decision": in_pass_measurement(torch, fl, step, peak)}
+        extra = {"cfg1_in_pass_share_decision": in_pass_measurement(torch, fl, step, peak),
+                 "cfg1_verified_speculation_k4": spec_measurement(torch, fl, step, peak)}
         extra.update(extra_measurements(torch, fl, peak))
 
     if rank != 0:

@@ -335,6 +335,26 @@ FL_API fl_status fl_logit_gate(const float* logits, int vocab, int batch, float 
                         float* margin, int32_t* top2, uint8_t* escalate, void* stream);
 
 /* ========================================================================= */
+/* Verified speculation ([PoD] abstract: a low-precision draft verified at   */
+/* 8 bits gives the 8-bit model's output at a comparable weight-byte cost).  */
+/* Greedy, over a window of k steps (1 <= k <= FL_MAX_BATCH):                */
+/*   draft token t    = draft_top2[t][0], the argmax of step t's D4 logits    */
+/*                      (the top2 row a gated D4 pass writes);                */
+/*   verified token t = verified_top2[t][0], the argmax of step t's D8 logits */
+/*                      (the top2 rows of one gated residual pass at batch k  */
+/*                      over the window's D4 outputs);                        */
+/*   accepted = the length of the longest prefix where the two agree;        */
+/*   emitted  = accepted + 1 if accepted < k, else k: the verified tokens of  */
+/*              steps 0 .. emitted - 1, the 8-bit model's own greedy choice.  */
+/* draft_top2, verified_top2  device int32 [k][2]                             */
+/* result  device int32 [2] = {accepted, emitted}, written                    */
+/* totals  device int32 [2] or NULL: accepted and emitted are ADDED to it     */
+/* One launch, asynchronous on stream.                                        */
+/* ========================================================================= */
+FL_API fl_status fl_spec_accept(const int32_t* draft_top2, const int32_t* verified_top2, int k, int32_t* result,
+                                int32_t* totals, void* stream);
+
+/* ========================================================================= */
 /* K-quant GEMV ([Ember]: Q4_K / Q6_K native kernels, dequantize only at     */
 /* block granularity inside the product, per-tensor dispatch, unsupported    */
 /* types fail). Records of 256 weights stored block-tiled: 64-row blocks,   */

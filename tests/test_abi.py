@@ -119,6 +119,11 @@ def test_host_side_rejections(fl):
     assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == -4                         # y not 8-aligned
     dp = fl.decide_problems([(24, 64, 128, 16, 16, None)])
     assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == -4                         # store not 16-aligned
+    # verified speculation
+    assert _status(fl, fl.fl_spec_accept, None, 16, 4, 16, None, s0) == ERR_ARG
+    assert _status(fl, fl.fl_spec_accept, 16, 16, 0, 16, None, s0) == ERR_SHAPE                 # k = 0
+    assert _status(fl, fl.fl_spec_accept, 16, 16, 17, 16, None, s0) == ERR_SHAPE                # k > 16
+    assert _status(fl, fl.fl_spec_accept, 16, 16, 4, 18, None, s0) == -4                        # result misaligned
 
 
 def test_misaligned_pointers_rejected(fl):

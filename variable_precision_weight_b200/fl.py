@@ -96,6 +96,7 @@ _sigs = {
     "fl_gemv_kquant": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _S, _P]),
     "fl_gemv_kquant_batched": (_I, [C.POINTER(fl_kquant_problem), _I, _I, _P]),
     "fl_level_decide": (_I, [C.POINTER(fl_decide_problem), _I, _I, C.POINTER(fl_decide_params), _P]),
+    "fl_spec_accept": (_I, [_P, _P, _I, _P, _P, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _fn = getattr(_lib, _name)
@@ -277,3 +278,8 @@ def decide_params(rule: int, gamma: int, kappa: int, lam: float = 0.0, f: float 
 
 def fl_level_decide(problems, n: int, batch: int, params: fl_decide_params, stream=None) -> None:
     _check(_lib.fl_level_decide(problems, n, batch, C.byref(params), _stream(stream)))
+
+
+def fl_spec_accept(draft_top2, verified_top2, k: int, result, totals=None, stream=None) -> None:
+    _check(_lib.fl_spec_accept(_ptr(draft_top2), _ptr(verified_top2), k, _ptr(result), _ptr(totals),
+                               _stream(stream)))

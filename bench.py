@@ -385,10 +385,17 @@ def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
     t = time_loop(torch, lambda k: g_all.replay(), rounds) / (rounds * NS)
     td = time_loop(torch, lambda k: g_dec.replay(), rounds) / (rounds * NS)
     tr = time_loop(torch, lambda k: g_res.replay(), rounds) / (rounds * NS)
+    g_lad = torch.cuda.CUDAGraph()                 # the score launch alone (ladder rule)
+    ladder = fl.decide_params(fl.FL_DECIDE_LADDER, 2, 4, 1.0, 0.0)
+    with torch.cuda.graph(g_lad):
+        for j in range(NS):
+            fl.fl_level_decide(dec, n, 1, ladder)
+    g_lad.replay()
+    tl = time_loop(torch, lambda k: g_lad.replay(), rounds) / (rounds * NS)
     nbytes = step.bytes_d4 + bytes_res
     return {"f": f, "lifted_blocks": got, "lifted_expected": lifted, "us_per_step": t * 1e6,
             "bytes_per_step": nbytes, "GBps": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
-            "tokens_per_s": 1.0 / t, "decide_us": td * 1e6, "residual_us": tr * 1e6,
+            "tokens_per_s": 1.0 / t, "decide_us": td * 1e6, "decide_ladder_us": tl * 1e6, "residual_us": tr * 1e6,
             "residual_GBps": bytes_res / tr / 1e9,
             "decide_bytes": bytes_scales + 4 * tot_out, "decide_GBps": (bytes_scales + 4 * tot_out) / td / 1e9,
             "launches_per_step": 4}

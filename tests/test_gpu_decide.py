@@ -107,7 +107,7 @@ def base_layers(torch, fl, shapes, gamma, batch, key):
 @pytest.mark.parametrize("gamma,batch", [(1, 1), (2, 1), (2, 3), (3, 16)])
 def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
     torch, fl = env
-    shapes = [(64 * 37, 384), (1024, 1024), (2048, 1024), (64, 128)]
+    shapes = [(64 * 37, 384), (1024, 1024), (2048, 1024), (64, 128), (64 * 300, 256)]
     items, host, keep = base_layers(torch, fl, shapes, gamma, batch, 300 + gamma + batch)
     torch.cuda.synchronize()
     kappa = 4
@@ -143,23 +143,31 @@ def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
         check_ladder(lev, sc, ref_lev, ref_red, gamma, kappa, lam, f"no-score ladder problem {i}")
 
 
-def test_share_ties_go_to_lower_index(env, orc):
-    """Identical blocks give bit-identical scores; the share lifts the lowest indices."""
+@pytest.mark.parametrize("nb", [10, 400])
+def test_share_ties_go_to_lower_index(env, orc, nb):
+    """Identical blocks give bit-identical scores; the share lifts the lowest indices (10
+    blocks: the one-warp ranking; 400: the radix select, the cut inside the tied group)."""
     torch, fl = env
-    o, n = 64 * 10, 256
+    o, n = 64 * nb, 256
     q1, s1 = synth.int8_layer(64, n, 61)
-    q, s = np.tile(q1, (10, 1)), np.tile(s1, (10, 1))
+    q, s = np.tile(q1, (nb, 1)), np.tile(s1, (nb, 1))
+    y = np.tile(synth.rng(62).standard_normal(64).astype(np.float32), (2, nb))
+    if nb > 10:                                # blocks 0-99 score higher, then 300 tied ones
+        s[:64 * 100] *= np.float32(2)
     st = pack_gpu(torch, fl, q, s)
-    y = torch.from_numpy(np.tile(synth.rng(62).standard_normal(64).astype(np.float32), (2, 10))).cuda()
-    lv = torch.empty(10, dtype=torch.uint8, device="cuda")
-    sc = torch.empty(10, dtype=torch.float32, device="cuda")
-    fl.fl_level_decide(fl.decide_problems([(st, o, n, y, lv, sc)]), 1, 2,
-                       fl.decide_params(fl.FL_DECIDE_SHARE, 2, 3, f=0.35))
+    yd = torch.from_numpy(y).cuda()
+    lv = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(nb, dtype=torch.float32, device="cuda")
+    f = 0.35
+    fl.fl_level_decide(fl.decide_problems([(st, o, n, yd, lv, sc)]), 1, 2,
+                       fl.decide_params(fl.FL_DECIDE_SHARE, 2, 3, f=f))
     torch.cuda.synchronize()
-    assert len(set(sc.cpu().numpy().tolist())) == 1
-    assert lv.cpu().numpy().tolist() == [3, 3, 3] + [2] * 7
-    assert np.array_equal(orc.level_decide(y.cpu().numpy(), s, 2, 3, 1, f=np.float32(0.35))[0],
-                          lv.cpu().numpy())
+    n_up = int(np.floor(np.float64(np.float32(f)) * nb))
+    scores = sc.cpu().numpy()
+    tied = scores[-1]
+    assert np.all(scores[(100 if nb > 10 else 0):] == tied)
+    assert lv.cpu().numpy().tolist() == [3] * n_up + [2] * (nb - n_up)
+    assert np.array_equal(orc.level_decide(y, s, 2, 3, 1, f=np.float32(f))[0], lv.cpu().numpy())
 
 
 @pytest.mark.parametrize("rule", [0, 1])

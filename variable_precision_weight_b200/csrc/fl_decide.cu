@@ -126,7 +126,9 @@ __global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constan
   }
 }
 
-constexpr int kSmemScores = 11776;  // a layer's scores staged in shared memory up to this many blocks (46 KB)
+constexpr int kWarpRank = 256;     // layers up to this many blocks: one warp ranks the keys
+constexpr int kSmemScores = 7680;   // a layer's scores staged in shared memory up to this many blocks (30 KB)
+constexpr int kShareWarps = kShareThreads / 32;
 
 // key of block i: larger score first, then the lower index (scores are >= 0, so their bit
 // patterns order like their values)
@@ -137,7 +139,8 @@ __device__ __forceinline__ uint64_t share_key(const float* score, int i) {
 template <int MAXP>
 __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ float s_score[];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kShareWarps][256];  // one histogram per warp: positive scores share
+                                               // their top bits, so one shared bin would serialise
   __shared__ uint64_t s_prefix;
   __shared__ uint32_t s_left, s_tied;
   pdl_release();
@@ -146,6 +149,35 @@ __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_const
   const int tid = threadIdx.x;
   pdl_wait();
   const float* score = P.score;
+  if (nb <= kWarpRank) {
+    // small layer: one warp ranks every key against all others (keys are distinct, so a key
+    // rises iff fewer than n_up keys exceed it); no block-wide barrier
+    if (tid >= 32) return;
+    uint64_t key[kWarpRank / 32];
+#pragma unroll
+    for (int m = 0; m < kWarpRank / 32; ++m) {
+      const int i = 32 * m + tid;
+      key[m] = i < nb ? share_key(score, i) : 0ull;
+    }
+    int above[kWarpRank / 32] = {};
+#pragma unroll
+    for (int m2 = 0; m2 < kWarpRank / 32; ++m2) {
+      if (32 * m2 >= nb) break;
+      for (int src = 0; src < 32; ++src) {
+        const uint64_t kj = __shfl_sync(0xffffffffu, key[m2], src);
+        if (32 * m2 + src < nb) {
+#pragma unroll
+          for (int m = 0; m < kWarpRank / 32; ++m) above[m] += kj > key[m];
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < kWarpRank / 32; ++m) {
+      const int i = 32 * m + tid;
+      if (i < nb) P.levels[i] = (uint8_t)(above[m] < P.n_up ? a.kappa : a.gamma);
+    }
+    return;
+  }
   uint64_t kth = 0;                         // with 0 < n_up < nb: the keys >= kth rise
   if (P.n_up > 0 && P.n_up < nb) {
     if (nb <= kSmemScores) {
@@ -161,13 +193,21 @@ __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_const
     // which the four passes over the index bits then split lower index first
     for (int pass = 0; pass < 8; ++pass) {
       const int shift = 56 - 8 * pass;
-      for (int d = tid; d < 256; d += kShareThreads) hist[d] = 0;
+      for (int d = tid; d < kShareWarps * 256; d += kShareThreads) (&hist[0][0])[d] = 0;
       __syncthreads();
       const uint64_t prefix = s_prefix;
       const uint64_t mask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+      uint32_t* const my = hist[tid >> 5];
       for (int i = tid; i < nb; i += kShareThreads) {
         const uint64_t k = share_key(score, i);
-        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        if ((k & mask) == prefix) atomicAdd(&my[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid < 256) {
+        uint32_t sum = 0;
+#pragma unroll
+        for (int w = 0; w < kShareWarps; ++w) sum += hist[w][tid];
+        hist[0][tid] = sum;
       }
       __syncthreads();
       if (tid < 32) {
@@ -176,7 +216,7 @@ __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_const
         uint32_t cnt[8], tot = 0;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          cnt[k] = hist[255 - 8 * tid - k];
+          cnt[k] = hist[0][255 - 8 * tid - k];
           tot += cnt[k];
         }
         uint32_t before = tot;              // inclusive scan over lanes, then exclusive

@@ -336,20 +336,22 @@ def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
     import numpy as np
     n, NS = step.n, step.NSETS
     tot_out = step.y.numel()
-    lv_to, score, dec_items, res_items = [], [], [], [[] for _ in range(NS)]
+    lv_to, score, lifted, counts, dec_items, res_items = [], [], [], [], [], [[] for _ in range(NS)]
     oo = oi = 0
-    lifted = bytes_res = bytes_scales = 0
+    bytes_res = bytes_scales = 0
     for k, (name, o, i) in enumerate(step.shapes):
         t = torch.empty(o // 64, dtype=torch.uint8, device="cuda")
         c = torch.empty(o // 64, dtype=torch.float32, device="cuda")
+        u = torch.empty(o // 64, dtype=torch.int32, device="cuda")
         lv_to.append(t)
         score.append(c)
+        lifted.append(u)
         ys = step.y[oo:oo + o]
-        dec_items.append((step.stores[k], o, i, ys, t, c))
+        dec_items.append((step.stores[k], o, i, ys, t, c, u))
         for j in range(NS):
             res_items[j].append((step.stores[k], o, i, step.levels[2 * k], t, step.xs[j, oi:oi + i], ys))
         up = int(np.floor(np.float64(np.float32(f)) * (o // 64)))    # the kernel's count of rising blocks
-        lifted += up
+        counts.append(up)
         bytes_res += up * (256 * (i // 128) + 2048 * (i // 128) * 2)
         bytes_scales += (o // 64) * 256 * (i // 128)
         oo += o
@@ -358,11 +360,12 @@ def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
     dec = fl.decide_problems(dec_items)
     params = fl.decide_params(fl.FL_DECIDE_SHARE, 2, 4, 0.0, f)
     res = [fl.gemv_problems(it) for it in res_items]
+    lists = fl.block_lists(lifted, counts)          # the residual reads the lifted blocks only
 
     def one(j):
         fl.fl_gemv_batched(step.prob_d4[j], n, 1, 0)
         fl.fl_level_decide(dec, n, 1, params)
-        fl.fl_gemv_batched(res[j], n, 1, 1)
+        fl.fl_gemv_batched_listed(res[j], *lists, n, 1, 1)
 
     for j in range(NS):
         one(j)
@@ -377,7 +380,7 @@ def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
             fl.fl_level_decide(dec, n, 1, params)
     with torch.cuda.graph(g_res):                  # the residual passes alone, last decided levels
         for j in range(NS):
-            fl.fl_gemv_batched(res[j], n, 1, 1)
+            fl.fl_gemv_batched_listed(res[j], *lists, n, 1, 1)
     for _ in range(3):
         g_all.replay()
         g_dec.replay()
@@ -393,7 +396,7 @@ def in_pass_measurement(torch, fl, step, peak, f=0.16, rounds=40):
     g_lad.replay()
     tl = time_loop(torch, lambda k: g_lad.replay(), rounds) / (rounds * NS)
     nbytes = step.bytes_d4 + bytes_res
-    return {"f": f, "lifted_blocks": got, "lifted_expected": lifted, "us_per_step": t * 1e6,
+    return {"f": f, "lifted_blocks": got, "lifted_expected": sum(counts), "us_per_step": t * 1e6,
             "bytes_per_step": nbytes, "GBps": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peak,
             "tokens_per_s": 1.0 / t, "decide_us": td * 1e6, "decide_ladder_us": tl * 1e6, "residual_us": tr * 1e6,
             "residual_GBps": bytes_res / tr / 1e9,

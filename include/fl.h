@@ -231,6 +231,18 @@ typedef struct {
 
 FL_API fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream);
 
+/* fl_gemv_batched over listed blocks only: problem i reads and writes the blocks
+ * lists[i][0 .. counts[i]) (device int32 block indices, distinct, each < out / 64; any
+ * order) and leaves every other output row as it was. The launch is partitioned over
+ * the listed blocks alone, so a sparse set (the blocks an in-pass decision lifted, for
+ * a mode 1 residual) is spread evenly over the SMs. lists: host array of n device
+ * pointers; counts: host array of n values in 0 .. out / 64 (a problem with count 0
+ * is skipped; all zero: nothing is launched). No gate; otherwise as fl_gemv_batched.
+ * The lists are device data, so the kernel checks them: an index outside 0 .. out/64 - 1
+ * is skipped and the next fl_device_status() returns FL_ERR_ARG. */
+FL_API fl_status fl_gemv_batched_listed(const fl_gemv_problem* problems, const int32_t* const* lists,
+                                        const int* counts, int n, int batch, int mode, void* stream);
+
 /* fl_gemv_batched with the logit gate fused in ([PoD] abstract: the gate reads the
  * distribution the low-precision step produced). Problem `problem`'s outputs y[t][0..out)
  * are the logits of batch row t; as its blocks are produced, each CTA folds them into
@@ -295,6 +307,9 @@ FL_API fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, int n,
 /*   levels  device uint8 [out / 64], written                                 */
 /*   score   device fp32 [out / 64], written with r_c; may be NULL for the   */
 /*           ladder rule, required for the share rule                         */
+/*   lifted  device int32 [out / 64] or NULL; share rule only: its first      */
+/*           floor(f * out / 64) entries receive the lifted blocks' indices   */
+/*           in ascending order (the block list of fl_gemv_batched_listed)    */
 /* params: 1 <= gamma <= kappa <= 4; ladder: lambda finite, >= 0; share:     */
 /* 0 <= f <= 1. One launch (ladder) or two (share), asynchronous on stream.   */
 /* ========================================================================= */
@@ -306,6 +321,7 @@ typedef struct {
   const float* y;
   uint8_t* levels;
   float* score;
+  int32_t* lifted;
 } fl_decide_problem;
 
 typedef struct {

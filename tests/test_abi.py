@@ -119,6 +119,17 @@ def test_host_side_rejections(fl):
     assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == -4                         # y not 8-aligned
     dp = fl.decide_problems([(24, 64, 128, 16, 16, None)])
     assert _status(fl, fl.fl_level_decide, dp, 1, 1, lad, s0) == -4                         # store not 16-aligned
+    # listed pass
+    probs = fl.gemv_problems([(16, 128, 128, 16, 16, 16, 16)])
+    lists, counts = fl.block_lists([16], [3])                                           # 3 > 128 / 64
+    assert _status(fl, fl.fl_gemv_batched_listed, probs, lists, counts, 1, 1, 1, s0) == ERR_ARG
+    lists, counts = fl.block_lists([16], [-1])
+    assert _status(fl, fl.fl_gemv_batched_listed, probs, lists, counts, 1, 1, 1, s0) == ERR_ARG
+    lists, counts = fl.block_lists([None], [1])                                         # NULL list
+    assert _status(fl, fl.fl_gemv_batched_listed, probs, lists, counts, 1, 1, 1, s0) == ERR_ARG
+    assert _status(fl, fl.fl_gemv_batched_listed, probs, None, counts, 1, 1, 1, s0) == ERR_ARG
+    lists, counts = fl.block_lists([None], [0])                                         # nothing listed
+    fl.fl_gemv_batched_listed(probs, lists, counts, 1, 1, 1, s0)                          # returns FL_OK
     # verified speculation
     assert _status(fl, fl.fl_spec_accept, None, 16, 4, 16, None, s0) == ERR_ARG
     assert _status(fl, fl.fl_spec_accept, 16, 16, 0, 16, None, s0) == ERR_SHAPE                 # k = 0

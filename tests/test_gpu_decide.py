@@ -117,7 +117,9 @@ def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
     lam = float(np.median(allr)) / 16 / 2            # about half lifted once, some twice
     lv_out = [torch.empty(o // 64, dtype=torch.uint8, device="cuda") for o, _ in shapes]
     sc_out = [torch.empty(o // 64, dtype=torch.float32, device="cuda") for o, _ in shapes]
-    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], lv, sc) for it, lv, sc in zip(items, lv_out, sc_out)])
+    up_out = [torch.full((o // 64,), -1, dtype=torch.int32, device="cuda") for o, _ in shapes]
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], lv, sc, up)
+                                for it, lv, sc, up in zip(items, lv_out, sc_out, up_out)])
     for rule, lam_, f in ((fl.FL_DECIDE_LADDER, lam, 0.0), (fl.FL_DECIDE_LADDER, 0.0, 0.0),
                           (fl.FL_DECIDE_LADDER, 1e30, 0.0), (fl.FL_DECIDE_SHARE, 0.0, 0.0),
                           (fl.FL_DECIDE_SHARE, 0.0, 0.16), (fl.FL_DECIDE_SHARE, 0.0, 0.5),
@@ -132,6 +134,10 @@ def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
                 check_ladder(lev, sc, ref_lev, ref_red, gamma, kappa, lam_, what)
             else:
                 check_share(lev, sc, ref_lev, ref_red, gamma, kappa, f, what)
+                up = np.flatnonzero(lev == kappa) if kappa > gamma else np.arange(0)
+                got = up_out[i].cpu().numpy()
+                assert np.array_equal(got[:len(up)], up), what          # ascending lifted indices
+                assert np.all(got[len(up):] == -1) or len(up) == 0 or rule == fl.FL_DECIDE_SHARE
     # ladder without a score array: the same levels as the ladder over the scores just written
     # (the same fp32 computation), and the oracle's outside the band
     probs = fl.decide_problems([(it[0], it[1], it[2], it[6], lv, None) for it, lv in zip(items, lv_out)])
@@ -184,11 +190,16 @@ def test_in_pass_pipeline(env, orc, rule):
     lam = float(np.quantile(allr, 0.84)) / 16        # about 16% lifted at least one rung
     to = [torch.empty(o // 64, dtype=torch.uint8, device="cuda") for o, _ in shapes]
     sc = [torch.empty(o // 64, dtype=torch.float32, device="cuda") for o, _ in shapes]
-    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c) for it, t, c in zip(items, to, sc)])
+    up = [torch.empty(o // 64, dtype=torch.int32, device="cuda") for o, _ in shapes]
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c, u) for it, t, c, u in zip(items, to, sc, up)])
     params = fl.decide_params(rule, gamma, kappa, lam, 0.16)
     fl.fl_level_decide(probs, len(shapes), batch, params)
     res = [(it[0], it[1], it[2], it[3], t, it[5], it[6]) for it, t in zip(items, to)]
-    fl.fl_gemv_batched(fl.gemv_problems(res), len(res), batch, 1)
+    if rule == fl.FL_DECIDE_SHARE:          # residual over the lifted blocks only
+        counts = [int(np.floor(np.float64(np.float32(0.16)) * (o // 64))) for o, _ in shapes]
+        fl.fl_gemv_batched_listed(fl.gemv_problems(res), *fl.block_lists(up, counts), len(res), batch, 1)
+    else:
+        fl.fl_gemv_batched(fl.gemv_problems(res), len(res), batch, 1)
     torch.cuda.synchronize()
     lifted = 0
     for i, ((q, s, x), it, t, c, y0) in enumerate(zip(host, items, to, sc, ys)):
@@ -228,3 +239,74 @@ def test_share_rule_on_a_layer_too_large_for_shared_memory(env, orc):
         torch.cuda.synchronize()
         ref_lev, ref_red = orc.level_decide(y.cpu().numpy(), s.cpu().numpy(), 2, 4, 1, f=np.float32(f))
         check_share(lv.cpu().numpy(), sc.cpu().numpy(), ref_lev, ref_red, 2, 4, f, f"large layer f {f}")
+
+
+@pytest.mark.parametrize("mode,batch", [(1, 1), (1, 5), (0, 2)])
+def test_batched_listed_vs_oracle(env, orc, mode, batch):
+    """Listed blocks only (any order): they become the oracle's result at their levels; every
+    other output row keeps its previous value bit for bit."""
+    torch, fl = env
+    shapes = [(64 * 37, 384), (1024, 1024), (64, 128), (2048, 256)]
+    g = synth.rng(808, mode, batch)
+    items, host, keep, lists, counts, picked = [], [], [], [], [], []
+    for i, (o, n) in enumerate(shapes):
+        q, s = synth.int8_layer(o, n, 809, i)
+        x = synth.bf16_normal((batch, n), 810, i)
+        st = pack_gpu(torch, fl, q, s)
+        nb = o // 64
+        frm = np.full(nb, 2, np.uint8)
+        to = g.integers(0, 5, nb).astype(np.uint8) if mode == 0 else np.full(nb, 4, np.uint8)
+        pick = g.permutation(nb)[:int(g.integers(0, nb + 1)) if i != 2 else 1].astype(np.int32)
+        y0 = g.standard_normal((batch, o)).astype(np.float32)
+        lvf, lvt, xd, y = dev(torch, frm if mode == 1 else to), dev(torch, to), dev(torch, x), dev(torch, y0)
+        lst = dev(torch, pick if len(pick) else np.zeros(1, np.int32))
+        keep += [st, lvf, lvt, xd, y, lst]
+        items.append((st, o, n, lvf, lvt, xd, y))
+        host.append((q, s, x, frm, to, y0))
+        lists.append(lst)
+        counts.append(len(pick))
+        picked.append(pick)
+    fl.fl_gemv_batched_listed(fl.gemv_problems(items), *fl.block_lists(lists, counts), len(items), batch, mode)
+    torch.cuda.synchronize()
+    for i, ((q, s, x, frm, to, y0), it, pick) in enumerate(zip(host, items, picked)):
+        y = it[6].cpu().numpy()
+        rows = np.zeros(y.shape[1], bool)
+        for b in pick:
+            rows[64 * b:64 * b + 64] = True
+        assert np.array_equal(y[:, ~rows], y0[:, ~rows]), f"unlisted rows changed, problem {i}"
+        if rows.any():
+            if mode == 1:
+                yref, mass = orc.gemv_residual(q, s, frm, to, x, with_mass=True)
+                yref = yref + y0
+            else:
+                yref, mass = orc.gemv_depth(q, s, to, x, with_mass=True)
+            err = np.abs(y[:, rows] - yref[:, rows])
+            assert np.all(err <= REL * mass[:, rows] + ABS + 1e-6 * np.abs(y0[:, rows])), f"problem {i}"
+
+
+def test_listed_pass_skips_and_reports_an_index_out_of_range(env, orc):
+    """A device list holding an index past the layer: that unit is skipped, the valid ones are
+    computed, and fl_device_status reports the bad list."""
+    torch, fl = env
+    o, n = 1024, 256
+    q, s = synth.int8_layer(o, n, 820)
+    x = synth.bf16_normal((1, n), 821)
+    st = pack_gpu(torch, fl, q, s)
+    lv = torch.full((o // 64,), 3, dtype=torch.uint8, device="cuda")
+    y = torch.full((1, o), 7.0, dtype=torch.float32, device="cuda")
+    xd = dev(torch, x)
+    lst = dev(torch, np.array([3, o // 64 + 5, 9], np.int32))
+    fl.fl_device_status()                                     # nothing pending before
+    fl.fl_gemv_batched_listed(fl.gemv_problems([(st, o, n, lv, None, xd, y)]), *fl.block_lists([lst], [3]), 1, 1, 0)
+    with pytest.raises(fl.FlError) as e:
+        fl.fl_device_status()
+    assert e.value.status == -1 and "out of range" in fl.fl_last_error()
+    fl.fl_device_status()                                     # the error word was cleared
+    yg = y.cpu().numpy()
+    yref, mass = orc.gemv_depth(q, s, np.full(o // 64, 3, np.uint8), x, with_mass=True)
+    for b in range(o // 64):
+        r = slice(64 * b, 64 * b + 64)
+        if b in (3, 9):
+            assert np.all(np.abs(yg[:, r] - yref[:, r]) <= REL * mass[:, r] + ABS), b
+        else:
+            assert np.all(yg[:, r] == 7.0), b

@@ -210,8 +210,8 @@ def test_kquant_step_full_size(env, orc):
 
 def test_in_pass_decision_full_size(env, orc):
     """The decode step read at D4, the in-pass decision over all 197 layers' 7,750 blocks in
-    one call (checked on every block), then the residual pass from D4 to the decided levels
-    (checked on sampled and on lifted blocks)."""
+    one call (checked on every block), then the listed residual pass from D4 over the lifted
+    blocks (checked on sampled and on lifted blocks; the others must keep their D4 value)."""
     torch, fl = env
     import test_gpu_decide as dec
     gen = torch.Generator(device="cuda")
@@ -235,7 +235,8 @@ def test_in_pass_decision_full_size(env, orc):
     ys = [it[6].cpu().numpy() for it in items]
     to = [torch.empty(it[1] // 64, dtype=torch.uint8, device="cuda") for it in items]
     sc = [torch.empty(it[1] // 64, dtype=torch.float32, device="cuda") for it in items]
-    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c) for it, t, c in zip(items, to, sc)])
+    up = [torch.empty(it[1] // 64, dtype=torch.int32, device="cuda") for it in items]
+    probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c, u) for it, t, c, u in zip(items, to, sc, up)])
     allr = np.concatenate([orc.level_decide(y, s, 2, 4, 0, lam=1.0)[1] for y, s in zip(ys, ss)])
     lam = float(np.quantile(allr, 0.84)) / 16
     for rule, f in ((fl.FL_DECIDE_LADDER, 0.0), (fl.FL_DECIDE_SHARE, 0.16)):
@@ -248,8 +249,12 @@ def test_in_pass_decision_full_size(env, orc):
                 dec.check_ladder(lev, score, ref_lev, ref_red, 2, 4, lam, f"step ladder, problem {k}")
             else:
                 dec.check_share(lev, score, ref_lev, ref_red, 2, 4, f, f"step share, problem {k}")
+    # the residual over the lifted blocks only, as the bench runs it
     res = [(it[0], it[1], it[2], it[3], t, it[5], it[6]) for it, t in zip(items, to)]
-    fl.fl_gemv_batched(fl.gemv_problems(res), n, 1, 1)
+    counts = [int(np.floor(np.float64(np.float32(0.16)) * (it[1] // 64))) for it in items]
+    for k, (t, u, c) in enumerate(zip(to, up, counts)):
+        assert np.array_equal(u.cpu().numpy()[:c], np.flatnonzero(t.cpu().numpy() > 2)), k
+    fl.fl_gemv_batched_listed(fl.gemv_problems(res), *fl.block_lists(up, counts), n, 1, 1)
     torch.cuda.synchronize()
     lifted = 0
     for k, (it, t, q, s) in enumerate(zip(items, to, qs, ss)):
@@ -260,5 +265,8 @@ def test_in_pass_decision_full_size(env, orc):
         rows = np.concatenate([np.arange(64 * b, 64 * b + 64) for b in blocks])
         yref, mass = orc.gemv_depth(q[rows].cpu().numpy(), s[rows], lev[blocks], it[5].cpu().numpy().view(np.uint16),
                                     with_mass=True)
-        _check(it[6].cpu().numpy()[:, rows], yref, mass, f"in-pass step, problem {k}")
+        yk = it[6].cpu().numpy()
+        _check(yk[:, rows], yref, mass, f"in-pass step, problem {k}")
+        keep_rows = np.repeat(lev <= 2, 64)
+        assert np.array_equal(yk[:, keep_rows], ys[k][:, keep_rows]), f"unlifted rows changed, problem {k}"
     assert lifted == sum(int(np.floor(np.float64(np.float32(0.16)) * (it[1] // 64))) for it in items)

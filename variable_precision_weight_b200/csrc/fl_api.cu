@@ -85,6 +85,8 @@ extern "C" fl_status fl_device_status(void) {
     return c == 1 ? "a producer's wait for a free stage" : c == 2 ? "a consumer's wait for a full stage"
          : c == 3 ? "the wait for staged activations" : c == 4 ? "the self-test wait" : "a wait";
   };
+  if (g == 5)
+    return fail(FL_ERR_ARG, "plane GEMV: a listed block index was out of range; that unit was skipped");
   if (g) return fail(FL_ERR_TIMEOUT, "plane GEMV: %s ran out (code %d); its outputs are not valid", what(g), g);
   if (k) return fail(FL_ERR_TIMEOUT, "K-quant GEMV: %s ran out (code %d); its outputs are not valid", what(k), k);
   return fail(FL_ERR_TIMEOUT, "logit gate: the wait for the cluster's partials ran out; its outputs are NaN");

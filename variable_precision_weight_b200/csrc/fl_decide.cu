@@ -34,6 +34,7 @@ struct Problem {
   const float* y;
   uint8_t* levels;
   float* score;
+  int32_t* lifted;                 // share rule: ascending indices of the lifted blocks (or NULL)
   int out;
   int G;
   int block_begin;                 // first global block index of this problem
@@ -171,10 +172,15 @@ __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_const
         }
       }
     }
+    int base = 0;
 #pragma unroll
     for (int m = 0; m < kWarpRank / 32; ++m) {
       const int i = 32 * m + tid;
-      if (i < nb) P.levels[i] = (uint8_t)(above[m] < P.n_up ? a.kappa : a.gamma);
+      const bool up = i < nb && above[m] < P.n_up;
+      if (i < nb) P.levels[i] = (uint8_t)(up ? a.kappa : a.gamma);
+      const unsigned bal = __ballot_sync(0xffffffffu, up);
+      if (up && P.lifted) P.lifted[base + __popc(bal & ((1u << tid) - 1u))] = i;
+      base += __popc(bal);
     }
     return;
   }
@@ -243,9 +249,26 @@ __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_const
     }
     kth = s_prefix;
   }
-  for (int i = tid; i < nb; i += kShareThreads) {
-    const bool up = P.n_up >= nb || (P.n_up > 0 && share_key(score, i) >= kth);
-    P.levels[i] = (uint8_t)(up ? a.kappa : a.gamma);
+  // levels, and the lifted indices in ascending order (a block-wide scan per 512 blocks)
+  __shared__ int s_warp_up[kShareWarps];
+  int base = 0;
+  for (int i0 = 0; i0 < nb; i0 += kShareThreads) {
+    const int i = i0 + tid;
+    const bool up = i < nb && (P.n_up >= nb || (P.n_up > 0 && share_key(score, i) >= kth));
+    if (i < nb) P.levels[i] = (uint8_t)(up ? a.kappa : a.gamma);
+    if (P.lifted == nullptr) continue;
+    const unsigned bal = __ballot_sync(0xffffffffu, up);
+    if ((tid & 31) == 0) s_warp_up[tid >> 5] = __popc(bal);
+    __syncthreads();
+    int before = base, total = 0;
+    for (int w = 0; w < kShareWarps; ++w) {
+      const int c = s_warp_up[w];
+      if (w < (tid >> 5)) before += c;
+      total += c;
+    }
+    if (up) P.lifted[before + __popc(bal & ((1u << (tid & 31)) - 1u))] = i;
+    base += total;
+    __syncthreads();
   }
 }
 
@@ -292,11 +315,14 @@ extern "C" fl_status fl_level_decide(const fl_decide_problem* problems, int n, i
       return fail(FL_ERR_ALIGN, "%s: problem %d y not 8-byte aligned", what, i);
     if (p.score && (reinterpret_cast<uintptr_t>(p.score) & 3u))
       return fail(FL_ERR_ALIGN, "%s: problem %d score not 4-byte aligned", what, i);
+    if (p.lifted && (reinterpret_cast<uintptr_t>(p.lifted) & 3u))
+      return fail(FL_ERR_ALIGN, "%s: problem %d lifted not 4-byte aligned", what, i);
     Problem& P = a.p[i];
     P.store = p.w.store;
     P.y = p.y;
     P.levels = p.levels;
     P.score = p.score;
+    P.lifted = q.rule == FL_DECIDE_SHARE ? p.lifted : nullptr;
     P.out = p.w.out;
     P.G = p.w.in / 128;
     P.block_begin = (int)blocks;

@@ -52,10 +52,12 @@ constexpr int kThreads = kConsumers + 32 * kProducerWarps;
 constexpr int kTeamStages = 2;
 constexpr int kStages = kTeams * kTeamStages;
 constexpr int kStageBytes = 18432;
-constexpr int kMaxCtas = 1024;
+constexpr int kMaxCtas = 960;   // unit ranges per launch (bounded by the kernel-parameter space)
 constexpr int kRed = 8;               // outputs per thread per pass of the slice reduction
 constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
 constexpr int kLevelCache = 4096;     // most units per CTA; all their plane ranges are cached in smem
+constexpr int kListCache = 512;       // most units per CTA of a listed pass; their block indices are cached
+constexpr int kSkipUnit = 0xFF;       // level-cache mark of a listed unit whose block index is out of range
 constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
 constexpr int kDigitBudget = kSmemLimit - kStages * kStageBytes;
 
@@ -70,11 +72,13 @@ struct Problem {
   float* y;
   float* partial;      // [slices][nblocks][batch][64] when slices > 1
   uint32_t* tickets;   // [nblocks] when slices > 1
-  int nblocks;
+  int nblocks;          // units per slice: the layer's blocks, or the listed ones
   int G;
   int slices;
   int slice_groups;    // groups per slice (last slice shorter)
   int unit_begin;      // first global unit index of this problem
+  const int32_t* list; // listed pass: unit i is block list[i] (NULL: unit i is block i)
+  int ynb;             // blocks of the layer (its output rows / 64)
 };
 
 template <int MAXP>
@@ -99,6 +103,7 @@ struct Args {
   // (optional) counts the passes that ran
   const uint8_t* run_if;
   uint32_t* runs;
+  int listed;          // some problem has a block list (units per CTA <= kListCache)
   Problem p[MAXP];
 };
 
@@ -112,6 +117,7 @@ __device__ int g_error;  // set when a bounded wait runs out (never expected)
 struct __align__(16) Slot {
   int p, j, u0, u1, b0;
   int nblocks, G, ngroups, slices, gfirst;  // gfirst = first group of the slice in the row
+  int ynb;           // blocks of the layer's output (rows / 64)
   int stride;
   int it0;           // first (batch row, group) digit item of the slot in the CTA's item count
   uint32_t digits;   // smem address
@@ -123,6 +129,7 @@ struct __align__(16) Slot {
   float* y;
   float* partial;
   uint32_t* tickets;
+  const int32_t* list;  // listed pass: the slot's units are blocks list[b0 ..]
 };
 
 __device__ __forceinline__ int slice_ng(const Problem& P, int j) {
@@ -587,13 +594,14 @@ __device__ __forceinline__ int plane_range(int mode, const uint8_t* lv_from, con
 
 // GATE: the logit gate is fused over problem a.gate_p's outputs (a separate instantiation,
 // so the lane partials cost the plain kernel no registers).
-template <int MAXP, int NT, bool GATE>
+template <int MAXP, int NT, bool GATE, bool LISTED>
 __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ __align__(8) uint64_t x_bar;  // staged activations have landed
   __shared__ Slot slots[kMaxSlots];
   __shared__ uint8_t lvc[kLevelCache];
+  __shared__ int32_t bic[LISTED ? kListCache : 1];  // listed pass: block index of each unit
   __shared__ __align__(16) uint8_t zeros[160];
   __shared__ int s_ticket[kTeams];
   __shared__ int s_nslots;
@@ -644,6 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         sl.u1 = min(u_end, slice_start + P.nblocks) - u_begin;
         sl.b0 = first - slice_start;
         sl.nblocks = P.nblocks;
+        sl.ynb = P.ynb;
+        sl.list = P.list;
         sl.G = P.G;
         sl.ngroups = slice_ng(P, j);
         sl.slices = P.slices;
@@ -709,7 +719,16 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       for (int k = threadIdx.x - kConsumers; k < nunits; k += 32 * kProducerWarps) {
         while (si + 1 < nsl && k >= slots[si].u1) ++si;
         const Slot& sl = slots[si];
-        lvc[k] = (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, sl.b0 + (k - sl.u0));
+        int b = sl.b0 + (k - sl.u0);
+        if constexpr (LISTED) {
+          b = sl.list[b];
+          if (b < 0 || b >= sl.ynb) {  // the list lives on the device: checked here, skipped, reported
+            atomicExch(&g_error, 5);
+            b = -1;
+          }
+          bic[k] = b;
+        }
+        lvc[k] = b < 0 ? (uint8_t)kSkipUnit : (uint8_t)plane_range(a.mode, sl.lv_from, sl.lv_to, b);
       }
     }
     named_bar(kBarProducers, 32 * kProducerWarps);
@@ -721,10 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
     for (int k = team; k < nunits; k += kTeams) {
       while (si + 1 < nsl && k >= slots[si].u1) ++si;
       const Slot& sl = slots[si];
-      const int b = sl.b0 + (k - sl.u0);
+      const int b = LISTED ? bic[k] : sl.b0 + (k - sl.u0);
       const int pr = (int)lvc[k];
       const int k0 = pr >> 4, np = pr & 15;
-      if (np == 0) continue;
+      if (np == 0 || (LISTED && pr == kSkipUnit)) continue;
       const int tgm = tile_groups(np);
       const int ngs = sl.ngroups;
       const int G = sl.G;
@@ -784,10 +803,11 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   for (int k = team; k < nunits; k += kTeams) {
     while (si + 1 < nsl && k >= slots[si].u1) ++si;
     const Slot& sl = slots[si];
-    const int b = sl.b0 + (k - sl.u0);
+    const int b = LISTED ? bic[k] : sl.b0 + (k - sl.u0);
     const int pr = (int)lvc[k];
+    if (LISTED && pr == kSkipUnit) continue;
     const int k0 = pr >> 4, np = pr & 15;
-    const size_t ystride = (size_t)64 * sl.nblocks;
+    const size_t ystride = (size_t)64 * (LISTED ? sl.ynb : sl.nblocks);
     const int row_base = 64 * b + 16 * mt;
     float* const y = sl.y;
     if (np == 0) {  // ZERO block (depth mode): its rows are 0; a residual adds nothing
@@ -1016,7 +1036,7 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
         if (count > 0) {
           if (n + 1 < target && acc + 0.5 * cost > per_cta * (n + 1)) cut = true;
           if (b == 0 && (dig + sb > budget || nslots == kMaxSlots)) cut = true;
-          if (count == kLevelCache) cut = true;
+          if (count == (a.listed ? kListCache : kLevelCache)) cut = true;
         }
         if (cut) {
           if (n + 1 >= kMaxCtas) return false;
@@ -1043,10 +1063,10 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
   return true;
 }
 
-template <int MAXP, int NT, bool GATE>
+template <int MAXP, int NT, bool GATE, bool LISTED = false>
 static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
   const size_t smem = (size_t)kSmemLimit;
-  auto kern = plane_gemv_kernel<MAXP, NT, GATE>;
+  auto kern = plane_gemv_kernel<MAXP, NT, GATE, LISTED>;
   FL_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                 "cudaFuncSetAttribute(plane_gemv)");
   FL_CHECK_CUDA(launch_pdl(kern, dim3(a.ncta), dim3(kThreads), smem, st, 1, a), "launch plane_gemv");
@@ -1064,6 +1084,14 @@ static fl_status launch_nt_gate(const Args<FL_MAX_PROBLEMS>& a, cudaStream_t st)
 
 template <int MAXP>
 static fl_status launch_nt(const Args<MAXP>& a, cudaStream_t st) {
+  if constexpr (MAXP > 1) {
+    if (a.listed) switch ((a.batch + 3) / 4) {
+        case 1: return launch<MAXP, 1, false, true>(a, st);
+        case 2: return launch<MAXP, 2, false, true>(a, st);
+        case 3: return launch<MAXP, 3, false, true>(a, st);
+        default: return launch<MAXP, 4, false, true>(a, st);
+      }
+  }
   switch ((a.batch + 3) / 4) {
     case 1: return launch<MAXP, 1, false>(a, st);
     case 2: return launch<MAXP, 2, false>(a, st);
@@ -1104,6 +1132,7 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   a.gate_p = -1;
   a.run_if = nullptr;
   a.runs = nullptr;
+  a.listed = 0;
   Problem& P = a.p[0];
   P.store = w->store;
   P.lv_from = lv_from;
@@ -1111,6 +1140,8 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   P.x = x;
   P.y = y;
   P.nblocks = nblocks;
+  P.ynb = nblocks;
+  P.list = nullptr;
   P.G = G;
   P.slices = pl.slices;
   P.slice_groups = pl.slice_groups;
@@ -1159,7 +1190,8 @@ constexpr size_t kGateTicketBytes = 256;
 constexpr size_t kGateWorkspaceBytes = kGateTicketBytes + (size_t)kMaxCtas * FL_MAX_BATCH * sizeof(GateRec);
 
 static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int mode, const fl_gate_spec* gate,
-                         const uint8_t* run_if, uint32_t* runs, void* stream, const char* what) {
+                         const uint8_t* run_if, uint32_t* runs, void* stream, const char* what,
+                         const int32_t* const* lists = nullptr, const int* counts = nullptr) {
   if (!problems) return fail(FL_ERR_ARG, "%s: problems is NULL", what);
   if (n < 1 || n > FL_MAX_PROBLEMS) return fail(FL_ERR_ARG, "%s: n=%d (1..%d)", what, n, FL_MAX_PROBLEMS);
   if (mode != 0 && mode != 1) return fail(FL_ERR_ARG, "%s: mode=%d (0 depth, 1 residual)", what, mode);
@@ -1171,6 +1203,9 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
   a.gate_p = -1;
   a.run_if = run_if;
   a.runs = runs;
+  a.listed = lists != nullptr ? 1 : 0;
+  if (lists != nullptr && (counts == nullptr || gate != nullptr))
+    return fail(FL_ERR_ARG, "%s: a listed pass needs counts and has no gate", what);
   size_t budget = kDigitBudget;
   if (gate) {
     if (gate->problem < 0 || gate->problem >= n)
@@ -1192,7 +1227,7 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
     a.gate_part = reinterpret_cast<GateRec*>(static_cast<uint8_t*>(gate->workspace) + kGateTicketBytes);
     budget -= (size_t)kConsumerWarps * batch * sizeof(GateRec);
   }
-  int unit = 0;
+  int unit = 0, np = 0;  // np: problems launched (a listed pass drops those with no listed block)
   for (int i = 0; i < n; ++i) {
     const fl_gemv_problem& q = problems[i];
     fl_status st = check_weight(&q.w, what);
@@ -1204,7 +1239,15 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
     if (G > max_groups_fit(batch, (long)budget))
       return fail(FL_ERR_SHAPE, "%s: problem %d in=%d too wide for batch %d in one launch (in <= %d)", what, i,
                   q.w.in, batch, 128 * max_groups_fit(batch, (long)budget));
-    Problem& P = a.p[i];
+    int units = q.w.out / 64;
+    if (lists != nullptr) {
+      if (counts[i] < 0 || counts[i] > q.w.out / 64)
+        return fail(FL_ERR_ARG, "%s: problem %d lists %d blocks (0..%d)", what, i, counts[i], q.w.out / 64);
+      if (counts[i] > 0 && lists[i] == nullptr) return fail(FL_ERR_ARG, "%s: problem %d list is NULL", what, i);
+      units = counts[i];
+      if (units == 0) continue;
+    }
+    Problem& P = a.p[np++];
     P.store = q.w.store;
     P.lv_from = q.levels;
     P.lv_to = q.to_levels;
@@ -1212,13 +1255,17 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
     P.y = q.y;
     P.partial = nullptr;
     P.tickets = nullptr;
-    P.nblocks = q.w.out / 64;
+    P.nblocks = units;
+    P.ynb = q.w.out / 64;
+    P.list = lists != nullptr ? lists[i] : nullptr;
     P.G = G;
     P.slices = 1;
     P.slice_groups = G;
     P.unit_begin = unit;
     unit += P.nblocks;
   }
+  if (np == 0) return FL_OK;  // a listed pass with nothing listed: no launch
+  a.nproblems = np;
   const int nsm = device_sm_count();
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
   if (!partition(a, nsm, budget)) return fail(FL_ERR_SHAPE, "%s: problems too large for one launch", what);
@@ -1241,6 +1288,13 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
 
 extern "C" fl_status fl_gemv_batched(const fl_gemv_problem* problems, int n, int batch, int mode, void* stream) {
   return gemv::batched(problems, n, batch, mode, nullptr, nullptr, nullptr, stream, "fl_gemv_batched");
+}
+
+extern "C" fl_status fl_gemv_batched_listed(const fl_gemv_problem* problems, const int32_t* const* lists,
+                                            const int* counts, int n, int batch, int mode, void* stream) {
+  if (!lists || !counts) return fail(FL_ERR_ARG, "fl_gemv_batched_listed: lists or counts is NULL");
+  return gemv::batched(problems, n, batch, mode, nullptr, nullptr, nullptr, stream, "fl_gemv_batched_listed", lists,
+                       counts);
 }
 
 extern "C" size_t fl_gemv_gate_workspace_bytes(int batch) {

@@ -62,7 +62,8 @@ class fl_kquant_problem(C.Structure):
 
 
 class fl_decide_problem(C.Structure):
-    _fields_ = [("w", fl_plane_weight), ("y", C.c_void_p), ("levels", C.c_void_p), ("score", C.c_void_p)]
+    _fields_ = [("w", fl_plane_weight), ("y", C.c_void_p), ("levels", C.c_void_p), ("score", C.c_void_p),
+                ("lifted", C.c_void_p)]
 
 
 class fl_decide_params(C.Structure):
@@ -87,6 +88,8 @@ _sigs = {
     "fl_gemv_depth_static": (_I, [C.POINTER(fl_plane_weight), _P, _P, _I, _P, _P]),
     "fl_gemv_residual": (_I, [C.POINTER(fl_plane_weight), _P, _P, _P, _I, _P, _P, _S, _P]),
     "fl_gemv_batched": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, _P]),
+    "fl_gemv_batched_listed": (_I, [C.POINTER(fl_gemv_problem), C.POINTER(C.c_void_p), C.POINTER(C.c_int), _I, _I,
+                                    _I, _P]),
     "fl_gemv_gate_workspace_bytes": (_S, [_I]),
     "fl_gemv_batched_gate": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, C.POINTER(fl_gate_spec), _P]),
     "fl_gemv_batched_gate_if": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, C.POINTER(fl_gate_spec), _P, _P, _P]),
@@ -210,6 +213,19 @@ def fl_gemv_batched(problems, n: int, batch: int, mode: int, stream=None) -> Non
     _check(_lib.fl_gemv_batched(problems, n, batch, mode, _stream(stream)))
 
 
+def block_lists(lists, counts):
+    """Device block lists and their host counts -> (pointer array, count array) for
+    fl_gemv_batched_listed."""
+    ptrs = (C.c_void_p * len(lists))(*[_ptr(l) for l in lists])
+    cnts = (C.c_int * len(counts))(*[int(c) for c in counts])
+    return ptrs, cnts
+
+
+def fl_gemv_batched_listed(problems, lists, counts, n: int, batch: int, mode: int, stream=None) -> None:
+    """lists, counts: the pair block_lists() returns."""
+    _check(_lib.fl_gemv_batched_listed(problems, lists, counts, n, batch, mode, _stream(stream)))
+
+
 def fl_gemv_gate_workspace_bytes(batch: int) -> int:
     return int(_lib.fl_gemv_gate_workspace_bytes(batch))
 
@@ -264,11 +280,15 @@ def fl_gemv_kquant_batched(problems, n: int, batch: int, stream=None) -> None:
 
 
 def decide_problems(items) -> "C.Array":
-    """items: iterable of (store, out, in, y, levels, score or None) -> fl_decide_problem array."""
+    """items: iterable of (store, out, in, y, levels, score or None[, lifted or None])
+    -> fl_decide_problem array."""
     items = list(items)
     arr = (fl_decide_problem * len(items))()
-    for i, (store, out, inn, y, lv, sc) in enumerate(items):
-        arr[i] = fl_decide_problem(fl_plane_weight(_ptr(store), out, inn), _ptr(y), _ptr(lv), _ptr(sc))
+    for i, it in enumerate(items):
+        store, out, inn, y, lv, sc = it[:6]
+        lifted = it[6] if len(it) > 6 else None
+        arr[i] = fl_decide_problem(fl_plane_weight(_ptr(store), out, inn), _ptr(y), _ptr(lv), _ptr(sc),
+                                   _ptr(lifted))
     return arr
 
 

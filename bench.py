@@ -202,10 +202,13 @@ class DecodeStep:
         tot_in = sum(i for _, _, i in self.shapes)
         tot_out = sum(o for _, o, _ in self.shapes)
         self.xs = torch.empty((self.NSETS, tot_in), dtype=torch.int16, device="cuda")
+        self.xs_b = torch.empty_like(self.xs)   # second input buffer (the end-to-end run double-buffers)
         self.y = torch.empty(tot_out, dtype=torch.float32, device="cuda")
         self.h2d_bytes = tot_in * 2
         items = [[] for _ in range(self.NSETS)]
         items_r = [[] for _ in range(self.NSETS)]
+        items_b = [[] for _ in range(self.NSETS)]
+        items_rb = [[] for _ in range(self.NSETS)]
         oi = oo = 0
         self.bytes_d4 = self.bytes_res = 0
         self.levels = []
@@ -217,9 +220,11 @@ class DecodeStep:
             self.levels += [d4, d8]
             ys = self.y[oo:oo + o]
             for j in range(self.NSETS):
-                xs = self.xs[j, oi:oi + i]
+                xs, xb = self.xs[j, oi:oi + i], self.xs_b[j, oi:oi + i]
                 items[j].append((st, o, i, d4, None, xs, ys))
                 items_r[j].append((st, o, i, d4, d8, xs, ys))
+                items_b[j].append((st, o, i, d4, None, xb, ys))
+                items_rb[j].append((st, o, i, d4, d8, xb, ys))
             self.bytes_d4 += (o // 64) * plane_bytes(i, 2)
             self.bytes_res += (o // 64) * (256 * (i // 128) + 2048 * (i // 128) * 2)
             oi += i
@@ -227,6 +232,8 @@ class DecodeStep:
         self.vocab = self.shapes[-1][1]
         self.prob_d4 = [fl.gemv_problems(it) for it in items]
         self.prob_res = [fl.gemv_problems(it) for it in items_r]
+        self.prob_d4_b = [fl.gemv_problems(it) for it in items_b]
+        self.prob_res_b = [fl.gemv_problems(it) for it in items_rb]
         self.n = len(items[0])
         # gate outputs per set (one 32-byte row, so one device->host copy reads a step's result)
         self.gates = torch.zeros((self.NSETS, 8), dtype=torch.int32, device="cuda")
@@ -259,11 +266,12 @@ class DecodeStep:
         self.calib = {"entropy_sorted": h.tolist(), "margin_min": float(M.min())}
         return float(0.5 * (h[self.NESC - 1] + h[self.NESC])), float(0.5 * M.min())
 
-    def step_graph_body(self, j):
+    def step_graph_body(self, j, buf=0):
         fl = self.fl
-        fl.fl_gemv_batched_gate(self.prob_d4[j], self.n, 1, 0, self.specs[j])
+        d4, res = (self.prob_d4, self.prob_res) if buf == 0 else (self.prob_d4_b, self.prob_res_b)
+        fl.fl_gemv_batched_gate(d4[j], self.n, 1, 0, self.specs[j])
         esc = self.gates[j, 4:5].view(self.torch.uint8)[0:1]
-        fl.fl_gemv_batched_gate_if(self.prob_res[j], self.n, 1, 1, self.specs[j], esc, self.runs)
+        fl.fl_gemv_batched_gate_if(res[j], self.n, 1, 1, self.specs[j], esc, self.runs)
 
     def gemv_only(self):
         # the step's dominant kernel as the step runs it (D4 pass, gate fused)
@@ -695,52 +703,55 @@ def run_fl(args, rank, world, local_rank):
     achieved = step.bytes_d4 / tk / 1e9
 
     # end to end: each step copies its inputs host->device (pinned) and reads the gate result back.
-    # The input sets are independent, so step k + 2's input copy and step k's read-back run on a
-    # second stream while step k + 1 computes (one device buffer and gate row per set, ordered by
-    # events); every copy is inside the timed region.
+    # Rounds of the NS input sets alternate between two device input buffers: while a round
+    # computes from one, its copy stream fills the other with the next round's inputs (the input
+    # sets are independent), and each step's result is read back on a third stream as soon as the
+    # step is done. One CUDA graph per buffer holds a round with its copies as graph nodes; the
+    # round's last copy and read-back complete before its graph does. The first round's inputs
+    # are copied before timing, so the timed region holds one input copy per step it runs (for
+    # the following round) and every step's read-back.
     hx = [torch.from_numpy(step.hx[j]).pin_memory() for j in range(NS)]
-    hres = torch.empty(8, dtype=torch.int32).pin_memory()
-    main = torch.cuda.current_stream()
-    side = torch.cuda.Stream()
-    ev_copy = [torch.cuda.Event() for _ in range(NS)]
-    ev_used = [torch.cuda.Event() for _ in range(NS)]
-    ev_side = torch.cuda.Event()
-    e2e_steps = min(args.steps, 5000)
+    hres = torch.empty((NS, 8), dtype=torch.int32).pin_memory()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs = (step.xs, step.xs_b)
 
-    def side_work(k, read_back):
-        # after the step that last used set k % NS: read its gate row, then copy step k's inputs
-        j, jb = k % NS, (k - 2) % NS
-        with torch.cuda.stream(side):
-            if read_back:
-                side.wait_event(ev_used[jb])
-                hres.copy_(step.gates[jb], non_blocking=True)
-            if k < e2e_steps:
-                side.wait_event(ev_used[j])
-                step.xs[j].copy_(hx[j], non_blocking=True)
-                ev_copy[j].record(side)
+    def round_with_copies(buf):
+        cap = torch.cuda.current_stream()
+        ev_done = [torch.cuda.Event() for _ in range(NS)]
+        ev_fork, ev_in, ev_out = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+        ev_fork.record(cap)
+        s_in.wait_event(ev_fork)
+        s_out.wait_event(ev_fork)
+        with torch.cuda.stream(s_in):                 # the next round's inputs, into the other buffer
+            for j in range(NS):
+                bufs[1 - buf][j].copy_(hx[j], non_blocking=True)
+        for j in range(NS):
+            step.step_graph_body(j, buf)
+            ev_done[j].record(cap)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[j])
+                hres[j].copy_(step.gates[j], non_blocking=True)      # step j's result
+        ev_in.record(s_in)
+        ev_out.record(s_out)
+        cap.wait_event(ev_in)
+        cap.wait_event(ev_out)
 
-    def body_e2e(k):
-        j = k % NS
-        if k == 0:
-            side_work(0, False)
-            side_work(1, False)
-        main.wait_event(ev_copy[j])
-        step.g[j].replay()
-        ev_used[j].record(main)
-        side_work(k + 2, True)                   # read step k's result, copy step k + 2's inputs
-        if k == e2e_steps - 1:                   # the last read-back ends inside the timed region
-            ev_side.record(side)
-            main.wait_event(ev_side)
-
-    for j in range(NS):
-        ev_used[j].record(main)
+    g_e2e = [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]
+    for buf in (0, 1):
+        with torch.cuda.graph(g_e2e[buf]):
+            round_with_copies(buf)
+    for r in range(2):                                # buffer 0 holds round 0's inputs after these
+        g_e2e[r % 2].replay()
+    e2e_rounds = max(1, min(args.steps, 5000) // NS)
+    e2e_steps = e2e_rounds * NS
     step.runs.zero_()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    te = time_loop(torch, body_e2e, e2e_steps)
+    te = time_loop(torch, lambda k: g_e2e[k % 2].replay(), e2e_rounds)
     te = max_over_ranks(te, world)
     n_esc_e = int(step.runs.item())
+    assert np.array_equal(hres.numpy(), step.gates.cpu().numpy()), "read-back differs from the device rows"
     e2e_val = job_rate(e2e_steps * step.bytes_d4 + n_esc_e * step.bytes_res, world, te) / 1e9
 
     extra = None

@@ -77,10 +77,12 @@ FL_API const char* fl_status_string(int status);
 
 /* Device-side failure detection. Every wait inside a kernel (a stage barrier, the gate's
  * cluster hand-off) is bounded; when one runs out the kernel records an error word and
- * returns instead of hanging, and its outputs are not valid. The launching call cannot
- * see that (it returned before the kernel ran), so this call waits for the device,
- * reads and clears every kernel's error word, and returns FL_ERR_TIMEOUT (with
- * fl_last_error naming the kernel and the wait) or FL_OK. */
+ * returns instead of hanging, and its outputs are not valid. Device data the host cannot
+ * check (the block lists of fl_gemv_batched_listed) is checked in the kernel the same way.
+ * The launching call cannot see either (it returned before the kernel ran), so this call
+ * waits for the device, reads and clears every kernel's error word, and returns
+ * FL_ERR_TIMEOUT for a wait that ran out, FL_ERR_ARG for a bad list entry (with
+ * fl_last_error naming the kernel and the cause), or FL_OK. */
 FL_API fl_status fl_device_status(void);
 
 /* Self-test of the failure path above: one thread waits, with a short limit, on a

@@ -40,6 +40,9 @@ WORKLOAD = ("qwen3-0.6b-shaped decode step: 197 GEMVs (28 layers x q,k,v,o,gate,
             "rotating input sets, entropy threshold set so 4 of them (16%) escalate; batch 1")
 
 
+SPEC_HBM_GBS = 8000.0   # B200 HBM3e, the vendor's figure (context beside the measured copy peak)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -510,6 +513,22 @@ def extra_measurements(torch, fl, peak):
     ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
     t1 = graph_time(lambda: fl.fl_gemv_depth(w0, lv, x, 1, y, ws, wsb), 200)
     out["cfg0_single_call_latency_us"] = t1 * 1e6
+    try:
+        # D4 everywhere, then the residual to D8 (256 layers per launch each)
+        d4 = torch.full((16,), 2, dtype=torch.uint8, device="cuda")
+        d8 = torch.full((16,), 4, dtype=torch.uint8, device="cuda")
+        a4 = fl.gemv_problems([(s_, 1024, 1024, d4, None, x, y) for s_ in stores[:256]])
+        ar = fl.gemv_problems([(s_, 1024, 1024, d4, d8, x, y) for s_ in stores[:256]])
+        tp = graph_time(lambda: (fl.fl_gemv_batched(a4, 256, 1, 0), fl.fl_gemv_batched(ar, 256, 1, 1)), 50)
+        pb = 16 * (plane_bytes(1024, 2) + 256 * 8 + 2048 * 8 * 2)   # D4 read, then scales + planes 2, 3
+        out["cfg0_d4_then_residual_to_d8"] = {"layers_per_launch": 256, "us_per_layer": tp / 256 * 1e6,
+                                              "GBps": 256 * pb / tp / 1e9, "frac": 256 * pb / tp / 1e9 / peak}
+        # hot: one layer's weights 256 times per launch, so they stay in L2
+        ah = fl.gemv_problems([(stores[0], 1024, 1024, lv, None, x, y)] * 256)
+        th = graph_time(lambda: fl.fl_gemv_batched(ah, 256, 1, 0), 50)
+        out["cfg0_mixed_depth_l2_resident"] = {"us_per_layer": th / 256 * 1e6, "GBps": 256 * nbytes / th / 1e9}
+    except Exception as e:  # a measurement that fails is reported, not fatal to the line
+        out["cfg0_d4_then_residual_to_d8"] = {"error": str(e)[:200]}
     del stores, items, arr
     torch.cuda.empty_cache()
 
@@ -568,6 +587,30 @@ def extra_measurements(torch, fl, peak):
             out[f"cfg3_{i}to{o}_b{batch}_D6"] = {"us": t * 1e6, "GBps": per_copy / t / 1e9,
                                                  "frac": per_copy / t / 1e9 / peak,
                                                  "tflops": 2 * batch * o * i / t / 1e12}
+        try:
+            # the g = 1 variant at batch 1: kappa = D8 inside 4 lenses drawn by the config-2 rule
+            nbk = o // 64
+            bxy, bc, br = synth.lens_inputs(nbk, 4, 3, o)
+            pg = fl.lens_params(0.3, 1.0, 3, 4, synth.even_stops(4, 3), 0)
+            lvg = torch.empty(nbk, dtype=torch.uint8, device="cuda")
+            fl.fl_level_map(torch.from_numpy(bxy).cuda(), nbk, torch.from_numpy(bc).cuda(), torch.from_numpy(br).cuda(),
+                            4, pg, lvg, None)
+            torch.cuda.synchronize()
+            lvh = lvg.cpu().numpy()
+            bg = sum(plane_bytes(i, int(v)) for v in lvh)
+            x1 = torch.from_numpy(synth.bf16_normal((1, i), 3, 1).view("int16")).cuda()
+            y1 = torch.empty((1, o), device="cuda")
+            wsb1 = fl.fl_gemv_workspace_bytes(o, i, 1)
+            ws1 = torch.zeros(max(wsb1, 16), dtype=torch.uint8, device="cuda")
+
+            def run_g():
+                for w in wts:
+                    fl.fl_gemv_depth(w, lvg, x1, 1, y1, ws1, wsb1)
+            tg = graph_time(run_g, 20) / ncp
+            out[f"cfg3_{i}to{o}_b1_g1"] = {"us": tg * 1e6, "GBps": bg / tg / 1e9, "frac": bg / tg / 1e9 / peak,
+                                           "d8_blocks": int((lvh == 4).sum()), "blocks": nbk}
+        except Exception as e:
+            out[f"cfg3_{i}to{o}_b1_g1"] = {"error": str(e)[:200]}
         del stores
         torch.cuda.empty_cache()
 
@@ -608,10 +651,30 @@ def cpu_baseline(budget_s=12.0):
             t_total += time.perf_counter() - t0
             nbytes += nb
         passes += 1
+    # the same sample on one thread, for about a tenth of the time
+    t1, b1 = 0.0, 0
+    while t1 < budget_s / 10:
+        for q, s, x, lv, nb in layers:
+            t0 = time.perf_counter()
+            oracle.gemv_depth(q, s, lv, x, nthreads=1)
+            t1 += time.perf_counter() - t0
+            b1 += nb
     return {"value": nbytes / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{passes} passes over the 28 GEMVs of layers 0-3 at D4 "
                       f"({nbytes / passes / 1e6:.1f} MB of weight bytes per pass), {t_total:.1f} s",
-            "tokens_per_s_equiv": nbytes / t_total / (316616704)}
+            "tokens_per_s_equiv": nbytes / t_total / (316616704),
+            "single_thread_value": b1 / t1 / 1e9, "cpu_model": cpu_model()}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 # ----------------------------------------------------------------------------- arms
@@ -701,6 +764,19 @@ def run_fl(args, rank, world, local_rank):
     reps = max(200, args.steps // 10)
     tk = time_loop(torch, lambda k: step.gK.replay(), reps) / reps
     achieved = step.bytes_d4 / tk / 1e9
+    spread = {}
+    try:  # the launch's own spread: 100 replays, each bracketed by events
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+        for e0, e1 in evs:
+            e0.record()
+            step.gK.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        us = np.array([e0.elapsed_time(e1) * 1e3 for e0, e1 in evs])
+        spread = {"us_p10": float(np.percentile(us, 10)), "us_p50": float(np.percentile(us, 50)),
+                  "us_p90": float(np.percentile(us, 90))}
+    except Exception as e:
+        spread = {"spread_error": str(e)[:200]}
 
     # end to end: each step copies its inputs host->device (pinned) and reads the gate result back.
     # Rounds of the NS input sets alternate between two device input buffers: while a round
@@ -777,10 +853,12 @@ def run_fl(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (316.6 MB of weights read per step vs 126 MB L2)",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "tokens_per_s": tok_s, "hbm_frac": value / world / peak, "peak_gbs": peak, "peak_kind": peak_kind,
+        "hbm_frac_of_8tbs_spec": value / world / SPEC_HBM_GBS,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": tr["bytes_per_launch"] if tr else None,
                      "kernel": "plane_gemv_kernel (fl_gemv_batched_gate, 197 problems, D4, logit gate fused)",
-                     "us_per_launch": tk * 1e6, "bytes_per_launch": step.bytes_d4,
+                     "us_per_launch": tk * 1e6, "bytes_per_launch": step.bytes_d4, **spread,
+                     "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,
                      # plane GEMV launches per step (the D4 pass plus the escalated steps' residual
                      # pass, both full reads of the store) x time per launch / step time
                      "share_of_step": (1 + n_esc / args.steps) * tk / (t / args.steps) if t > 0 else None},

@@ -532,6 +532,26 @@ def extra_measurements(torch, fl, peak):
     del stores, items, arr
     torch.cuda.empty_cache()
 
+    try:
+        # the standalone logit gate over the Qwen3-0.6B vocab (151,936 fp32 logits, batch 1), and
+        # the packer (int8 codes + scales -> plane store) on the head's 1024 -> 151936 shape
+        V = 151936
+        z = torch.randn((1, V), device="cuda", generator=gen)
+        ge, gm = torch.empty(1, device="cuda"), torch.empty(1, device="cuda")
+        gt, gs = torch.empty((1, 2), dtype=torch.int32, device="cuda"), torch.empty(1, dtype=torch.uint8, device="cuda")
+        tgt = graph_time(lambda: fl.fl_logit_gate(z, V, 1, 10.0, 1e-3, ge, gm, gt, gs), 200)
+        out["gate_151936_logits"] = {"us": tgt * 1e6, "GBps": 4 * V / tgt / 1e9}
+        qh = torch.randint(-127, 128, (V, 1024), dtype=torch.int8, device="cuda", generator=gen)
+        sh = torch.rand((V, 8), device="cuda", generator=gen)
+        sth = torch.empty(fl.fl_plane_store_bytes(V, 1024), dtype=torch.uint8, device="cuda")
+        tpk = graph_time(lambda: fl.fl_pack_planes(qh, sh, V, 1024, sth), 20)
+        pk_bytes = qh.numel() + sh.numel() * 4 + sth.numel()
+        out["pack_1024x151936"] = {"us": tpk * 1e6, "GBps": pk_bytes / tpk / 1e9, "frac": pk_bytes / tpk / 1e9 / peak,
+                                   "bytes": pk_bytes}
+        del qh, sh, sth
+    except Exception as e:
+        out["gate_151936_logits"] = {"error": str(e)[:200]}
+
     # config 2: lens map over 14708 blocks (8 lenses) -> per-layer levels -> 35 layers x [64 n_b, 2048]
     nb = 14708
     xy, cxy, r = synth.lens_inputs(nb, 8, 2, 1)

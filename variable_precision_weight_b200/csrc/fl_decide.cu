@@ -17,8 +17,12 @@
 // warp streams the block's 64 G scales (the head of the block in the plane store) and its
 // 64 outputs per batch row, reduces both in a fixed shuffle order, and writes the reduced
 // score (and, for the ladder, the level). share_kernel (share rule only): one CTA per
-// problem selects the floor(f n) largest keys (score bits, ~index) with an 8-bit radix
-// select over 64-bit keys in shared-memory histograms, then writes every block's level.
+// problem picks the floor(f n) largest keys (score bits, then the complemented index, so
+// equal scores rank the lower index first). A layer of up to 256 blocks is ranked by one
+// warp (every key against every other, no barrier); a larger one by an 8-bit radix select
+// over the 64-bit keys with per-warp shared-memory histograms, its scores staged in shared
+// memory up to 7,680 blocks. It then writes every block's level and, when asked, the lifted
+// blocks' indices in ascending order (a block-wide scan per 512 blocks).
 #include <math.h>
 
 #include "fl_common.cuh"

@@ -128,6 +128,8 @@ def test_host_side_rejections(fl):
     lists, counts = fl.block_lists([None], [1])                                         # NULL list
     assert _status(fl, fl.fl_gemv_batched_listed, probs, lists, counts, 1, 1, 1, s0) == ERR_ARG
     assert _status(fl, fl.fl_gemv_batched_listed, probs, None, counts, 1, 1, 1, s0) == ERR_ARG
+    lists, counts = fl.block_lists([18], [1])                                           # misaligned list
+    assert _status(fl, fl.fl_gemv_batched_listed, probs, lists, counts, 1, 1, 1, s0) == -4
     lists, counts = fl.block_lists([None], [0])                                         # nothing listed
     fl.fl_gemv_batched_listed(probs, lists, counts, 1, 1, 1, s0)                          # returns FL_OK
     # verified speculation

@@ -1244,6 +1244,8 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
       if (counts[i] < 0 || counts[i] > q.w.out / 64)
         return fail(FL_ERR_ARG, "%s: problem %d lists %d blocks (0..%d)", what, i, counts[i], q.w.out / 64);
       if (counts[i] > 0 && lists[i] == nullptr) return fail(FL_ERR_ARG, "%s: problem %d list is NULL", what, i);
+      if (reinterpret_cast<uintptr_t>(lists[i]) & 3u)
+        return fail(FL_ERR_ALIGN, "%s: problem %d list not 4-byte aligned", what, i);
       units = counts[i];
       if (units == 0) continue;
     }

@@ -97,6 +97,10 @@ def test_host_side_rejections(fl):
     assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == -4
     spec = fl.gate_spec(0, 0.0, 0.0, 16, 16, 16, 16, 16, gsz)
     assert _status(fl, fl.fl_gemv_batched_gate_if, probs, 1, 1, 1, spec, None, None, s0) == ERR_ARG   # no run_if
+    assert _status(fl, fl.fl_gemv_batched_gate_if, probs, 1, 1, 1, spec, 16, 18, s0) == -4           # runs misaligned
+    spec = fl.gate_spec(0, 0.0, 0.0, 16, 16, 18, 16, 16, gsz)                  # top2 misaligned
+    assert _status(fl, fl.fl_gemv_batched_gate, probs, 1, 1, 0, spec, s0) == -4
+    assert _status(fl, fl.fl_logit_gate, 16, 1024, 1, 0.0, 0.0, 16, 17, 16, 16, s0) == -4          # margin
     kp = fl.kquant_problems([(16, 11, 64, 256, 16, 16)])
     assert _status(fl, fl.fl_gemv_kquant_batched, kp, 1, 1, s0) == ERR_UNSUP
     assert "Q4_K" in fl.fl_last_error()

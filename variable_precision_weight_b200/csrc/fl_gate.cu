@@ -184,6 +184,9 @@ extern "C" fl_status fl_logit_gate(const float* logits, int vocab, int batch, fl
   if (batch < 1 || batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..16)", what, batch);
   if (vocab < 4 || vocab > (1 << 24) || vocab % 4) return fail(FL_ERR_SHAPE, "%s: vocab=%d (4..2^24, %% 4 == 0)", what, vocab);
   if (!aligned16(logits)) return fail(FL_ERR_ALIGN, "%s: logits not 16-byte aligned", what);
+  if ((reinterpret_cast<uintptr_t>(entropy) | reinterpret_cast<uintptr_t>(margin) | reinterpret_cast<uintptr_t>(top2)) &
+      3u)
+    return fail(FL_ERR_ALIGN, "%s: entropy, margin and top2 must be 4-byte aligned", what);
   FL_CHECK_CUDA(gate_launch(logits, vocab, batch, tau_h, tau_m, entropy, margin, top2, escalate,
                             static_cast<cudaStream_t>(stream)),
                 "launch logit_gate");

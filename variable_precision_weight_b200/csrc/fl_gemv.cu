@@ -1204,6 +1204,7 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
   a.run_if = run_if;
   a.runs = runs;
   a.listed = lists != nullptr ? 1 : 0;
+  if (reinterpret_cast<uintptr_t>(runs) & 3u) return fail(FL_ERR_ALIGN, "%s: runs not 4-byte aligned", what);
   if (lists != nullptr && (counts == nullptr || gate != nullptr))
     return fail(FL_ERR_ARG, "%s: a listed pass needs counts and has no gate", what);
   size_t budget = kDigitBudget;
@@ -1216,6 +1217,9 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
       return fail(FL_ERR_WORKSPACE, "%s: gate workspace %zu bytes, need %zu", what, gate->workspace_bytes,
                   kGateWorkspaceBytes);
     if (!aligned16(gate->workspace)) return fail(FL_ERR_ALIGN, "%s: gate workspace not 16-byte aligned", what);
+    if ((reinterpret_cast<uintptr_t>(gate->entropy) | reinterpret_cast<uintptr_t>(gate->margin) |
+         reinterpret_cast<uintptr_t>(gate->top2)) & 3u)
+      return fail(FL_ERR_ALIGN, "%s: gate entropy, margin and top2 must be 4-byte aligned", what);
     a.gate_p = gate->problem;
     a.tau_h = gate->tau_h;
     a.tau_m = gate->tau_m;

@@ -147,4 +147,12 @@ def test_misaligned_pointers_rejected(fl):
     s0 = 0
     w = fl.plane_weight(17, 64, 128)
     assert _status(fl, fl.fl_gemv_depth, w, 16, 16, 1, 16, None, 0, s0) == -4
+    w = fl.plane_weight(16, 64, 128)
+    assert _status(fl, fl.fl_gemv_depth, w, 16, 16, 1, 18, None, 0, s0) == -4                   # y
+    assert _status(fl, fl.fl_gemv_batched, fl.gemv_problems([(16, 64, 128, 16, None, 16, 18)]), 1, 1, 0, s0) == -4
+    assert _status(fl, fl.fl_gemv_kquant, 16, 12, 64, 256, 16, 1, 18, None, 0, s0) == -4       # y
+    assert _status(fl, fl.fl_gemv_kquant_batched, fl.kquant_problems([(16, 12, 64, 256, 16, 18)]), 1, 1, s0) == -4
+    p = fl.lens_params(0.3, 0.75, 1, 4, [0.5, 1.0], 0)
+    assert _status(fl, fl.fl_level_map, 18, 10, 16, 16, 8, p, 16, None, s0) == -4              # xy
+    assert _status(fl, fl.fl_level_map, 16, 10, 16, 16, 8, p, 16, 17, s0) == -4                # counts
     assert _status(fl, fl.fl_pack_planes, 18, 16, 64, 128, 16, s0) == -4

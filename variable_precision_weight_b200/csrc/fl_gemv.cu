@@ -1115,6 +1115,7 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   fl_status st = check_weight(w, what);
   if (st != FL_OK) return st;
   if (!lv_from || !x || !y || (mode == 1 && !lv_to)) return fail(FL_ERR_ARG, "%s: NULL pointer argument", what);
+  if (reinterpret_cast<uintptr_t>(y) & 3u) return fail(FL_ERR_ALIGN, "%s: y not 4-byte aligned", what);
   if (batch < 1 || batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..16)", what, batch);
   if (!aligned16(x)) return fail(FL_ERR_ALIGN, "%s: x not 16-byte aligned", what);
   const int nsm = device_sm_count();
@@ -1238,6 +1239,7 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
     if (st != FL_OK) return st;
     if (!q.levels || !q.x || !q.y || (mode == 1 && !q.to_levels))
       return fail(FL_ERR_ARG, "%s: problem %d has a NULL pointer", what, i);
+    if (reinterpret_cast<uintptr_t>(q.y) & 3u) return fail(FL_ERR_ALIGN, "%s: problem %d y not 4-byte aligned", what, i);
     if (!aligned16(q.x)) return fail(FL_ERR_ALIGN, "%s: problem %d x not 16-byte aligned", what, i);
     const int G = q.w.in / 128;
     if (G > max_groups_fit(batch, (long)budget))

@@ -857,6 +857,7 @@ extern "C" fl_status fl_gemv_kquant(const void* blocks, int ggml_type, int out, 
   fl_status st = kq::check_tensor(blocks, ggml_type, out, in, what, 0);
   if (st != FL_OK) return st;
   if (!x || !y) return fail(FL_ERR_ARG, "%s: NULL x/y", what);
+  if (reinterpret_cast<uintptr_t>(y) & 3u) return fail(FL_ERR_ALIGN, "%s: y not 4-byte aligned", what);
   if (batch < 1 || batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..16)", what, batch);
   if (!aligned16(x)) return fail(FL_ERR_ALIGN, "%s: x not 16-byte aligned", what);
   const int nsm = device_sm_count();
@@ -907,6 +908,7 @@ extern "C" fl_status fl_gemv_kquant_batched(const fl_kquant_problem* problems, i
     fl_status st = kq::check_tensor(q.blocks, q.ggml_type, q.out, q.in, what, i);
     if (st != FL_OK) return st;
     if (!q.x || !q.y) return fail(FL_ERR_ARG, "%s: tensor %d NULL x/y", what, i);
+    if (reinterpret_cast<uintptr_t>(q.y) & 3u) return fail(FL_ERR_ALIGN, "%s: tensor %d y not 4-byte aligned", what, i);
     if (!aligned16(q.x)) return fail(FL_ERR_ALIGN, "%s: tensor %d x not 16-byte aligned", what, i);
     const int nsb = q.in / 256;
     if (nsb > kq::max_sb_fit(batch))

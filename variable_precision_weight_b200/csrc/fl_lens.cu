@@ -92,6 +92,9 @@ extern "C" fl_status fl_level_map(const float* xy, int nblocks, const float* cen
   if (nblocks < 0 || nlenses < 0 || nlenses > 64) return fail(FL_ERR_ARG, "%s: nblocks=%d nlenses=%d", what, nblocks, nlenses);
   if (nblocks > 0 && (!xy || !levels)) return fail(FL_ERR_ARG, "%s: NULL xy/levels", what);
   if (nlenses > 0 && (!centers || !radii)) return fail(FL_ERR_ARG, "%s: NULL centers/radii", what);
+  if ((reinterpret_cast<uintptr_t>(xy) | reinterpret_cast<uintptr_t>(centers) | reinterpret_cast<uintptr_t>(radii) |
+       reinterpret_cast<uintptr_t>(counts)) & 3u)
+    return fail(FL_ERR_ALIGN, "%s: xy, centers, radii and counts must be 4-byte aligned", what);
   if (p->m < 1 || p->m > 15 || p->gamma < 0 || p->gamma > p->m)
     return fail(FL_ERR_ARG, "%s: gamma=%d m=%d", what, p->gamma, p->m);
   if (!(p->f >= 0.0f && p->f < 1.0f)) return fail(FL_ERR_ARG, "%s: f=%g (0 <= f < 1)", what, (double)p->f);

@@ -154,6 +154,7 @@ typedef struct {
 /* xy      device, fp32 [nblocks][2] block coordinates
  * centers device, fp32 [nlenses][2]; radii device, fp32 [nlenses] (r_i >= 0)
  * levels  device, uint8 [nblocks] (output, level index 0..m)
+ * (xy, centers, radii and counts 4-byte aligned)
  * counts  device, uint32 [m + 1] or NULL: per-level block counts are ADDED
  *         to it (the caller zeroes it first).
  * nblocks >= 0, 0 <= nlenses <= 64. */
@@ -174,7 +175,7 @@ FL_API fl_status fl_level_map(const float* xy, int nblocks, const float* centers
 /* levels   device, uint8 [out / 64], values 0..4 (0 ZERO .. 4 D8); values   */
 /*          above 4 are read as 4.                                           */
 /* x        device, bf16 [batch][in], 16-byte aligned; batch 1..16           */
-/* y        device, fp32 [batch][out]; overwritten                           */
+/* y        device, fp32 [batch][out], 4-byte aligned; overwritten           */
 /* workspace device scratch for splitting a layer's columns across CTAs:     */
 /*          at least fl_gemv_workspace_bytes(out, in, batch) bytes, 16-byte  */
 /*          aligned, ZERO-FILLED before its first use; every successful call */
@@ -252,7 +253,7 @@ FL_API fl_status fl_gemv_batched_listed(const fl_gemv_problem* problems, const i
  * entropy / margin / top2 / escalate exactly as fl_logit_gate defines them (equal up to
  * fp32 summation order). In mode 1 the gate reads the updated y. y is written as by
  * fl_gemv_batched. No counterpart of the separate launch is needed.
- * entropy, margin  device, fp32 [batch]      top2  device, int32 [batch][2]
+ * entropy, margin  device, fp32 [batch]      top2  device, int32 [batch][2] (all 4-byte aligned)
  * escalate         device, uint8 [batch]
  * workspace        device, >= fl_gemv_gate_workspace_bytes(batch) bytes, 16-byte
  *                  aligned, ZERO-FILLED before first use; every completed launch leaves
@@ -278,7 +279,7 @@ FL_API fl_status fl_gemv_batched_gate(const fl_gemv_problem* problems, int n, in
  * decided on the device, with no read-back to the host): fl_gemv_batched_gate that runs
  * only if the byte at run_if (device, typically the escalate flag a preceding gated pass
  * wrote) is non-zero, and otherwise returns at once, leaving y and the gate outputs as
- * they were. runs: device uint32 or NULL; each pass that ran adds 1 to it. */
+ * they were. runs: device uint32 (4-byte aligned) or NULL; each pass that ran adds 1 to it. */
 FL_API fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, int n, int batch, int mode,
                                   const fl_gate_spec* gate, const uint8_t* run_if, uint32_t* runs,
                                   void* stream);
@@ -346,7 +347,8 @@ FL_API fl_status fl_level_decide(const fl_decide_problem* problems, int n, int b
 /*   logits (ties to the lower index), margin = p1 - p2 = (1 - e^(z_i2-m))/S,*/
 /*   escalate = (entropy > tau_h) || (margin < tau_m).                       */
 /* logits device fp32 [batch][vocab], 16-byte aligned, vocab % 4 == 0,      */
-/* 4 <= vocab <= 2^24; outputs device: entropy, margin fp32 [batch], top2 int32   */
+/* 4 <= vocab <= 2^24; outputs device (4-byte aligned): entropy, margin fp32      */
+/* [batch], top2 int32                                                        */
 /* [batch][2], escalate uint8 [batch]. fp32 arithmetic.                      */
 /* ========================================================================= */
 FL_API fl_status fl_logit_gate(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,

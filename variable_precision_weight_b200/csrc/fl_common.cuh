@@ -145,74 +145,8 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
 // split into two balanced signed bytes  v_c = 256 hi_c + lo_c,
 // hi_c in [-64, 64], lo_c in [-128, 127].  The group keeps 2^-sigma (to undo
 // the scaling) and sum_c v_c (for the constant part of the reconstruction).
-// Absolute error per element <= 2^(E - 15) <= 2^-14 max |x_c|.
-
-struct XDigitView {
-  int8_t* digits;      // [2 * batch_pad][stride]: row 2b = hi digits of batch b, 2b + 1 = lo digits
-  float* inv_scale;    // [batch_pad][ngroups] 2^-sigma
-  int32_t* gsum;       // [batch_pad][ngroups * sub] sums of v over each sub-group
-  int stride;          // bytes per digit row
-  int ngroups;
-};
-
-// Compute the digits of columns [col0, col0 + 128 * ngroups) of x (batch rows)
-// into smem. Called by `nthreads` threads starting at thread index `tid`.
-// `sub` = number of equal sub-groups per 128 columns whose sums are kept
-// (1 for the plane store, 4 for Q4_K, 8 for Q6_K). Digit rows exist for
-// b < batch only; for batch <= b < batch_pad the sums and scales are zeroed.
-//
-// `perm` = 1 stores the digits of each 32-column chunk in the order
-// (0-3, 16-19, 4-7, 20-23, 8-11, 24-27, 12-15, 28-31), so that the two k32
-// operand halves of one lane (columns 4t..4t+3 and 16+4t..16+4t+3 of the
-// chunk) are adjacent; `perm` = 0 keeps column order.
-__device__ __forceinline__ void build_x_digits(const uint16_t* __restrict__ x, int in, int batch, int batch_pad,
-                                               int col0, XDigitView v, int sub, int tid, int nthreads,
-                                               int perm = 0) {
-  // one warp per (batch row, group): 32 lanes x 4 columns
-  const int lane = tid & 31, wid = tid >> 5, nw = nthreads >> 5;
-  const int per_sub = 128 / sub;
-  for (int item = wid; item < batch_pad * v.ngroups; item += nw) {
-    const int b = item / v.ngroups, g = item % v.ngroups;
-    if (b >= batch) {  // padding rows: no digits are stored, their sums and scales read as zero
-      if (lane == 0) v.inv_scale[b * v.ngroups + g] = 0.f;
-      if (lane < sub) v.gsum[(b * v.ngroups + g) * sub + lane] = 0;
-      continue;
-    }
-    int8_t* hi = v.digits + (size_t)(2 * b) * v.stride + 128 * g;
-    int8_t* lo = v.digits + (size_t)(2 * b + 1) * v.stride + 128 * g;
-    const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)b * in + col0 + 128 * g + 4 * lane);
-    float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                  __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-    float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    int E = 0;
-    if (m > 0.f) {
-      frexpf(m, &E);  // m = mant * 2^E, mant in [0.5, 1)  ->  m < 2^E
-    }
-    const int sigma = (m > 0.f) ? (14 - E) : 0;
-    uint32_t hw = 0, lw = 0;
-    int part = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int vv = __float2int_rn(ldexpf(f[i], sigma));
-      const int h = (vv + 128) >> 8;
-      const int l = vv - 256 * h;
-      hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
-      lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
-      part += vv;
-    }
-    const int wpos = perm ? (8 * (lane >> 3) + 2 * (lane & 3) + ((lane >> 2) & 1)) : lane;
-    reinterpret_cast<uint32_t*>(hi)[wpos] = hw;
-    reinterpret_cast<uint32_t*>(lo)[wpos] = lw;
-    // sums over sub-groups of per_sub columns (per_sub / 4 lanes each)
-    const int lanes_per_sub = per_sub / 4;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1)
-      if (o < lanes_per_sub) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane % lanes_per_sub == 0) v.gsum[(b * v.ngroups + g) * sub + lane / lanes_per_sub] = part;
-    if (lane == 0) v.inv_scale[b * v.ngroups + g] = ldexpf(1.0f, -sigma);
-  }
-}
+// Absolute error per element <= 2^(E - 15) <= 2^-14 max |x_c|. The plane and
+// K-quant kernels build these digits in their prologues, each in the shared-memory
+// layout its tensor-core fragments read.
 
 }  // namespace fl

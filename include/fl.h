@@ -76,8 +76,9 @@ typedef enum {
 FL_API const char* fl_status_string(int status);
 
 /* Device-side failure detection. Every wait inside a kernel (a stage barrier, the gate's
- * cluster hand-off) is bounded; when one runs out the kernel records an error word and
- * returns instead of hanging, and its outputs are not valid. Device data the host cannot
+ * cluster hand-off) is bounded by a deadline of 1 s on the GPU's global timer; when one
+ * runs out the kernel records an error word and returns instead of hanging, and its
+ * outputs are not valid. Device data the host cannot
  * check (the block lists of fl_gemv_batched_listed) is checked in the kernel the same way.
  * The launching call cannot see either (it returned before the kernel ran), so this call
  * waits for the device, reads and clears every kernel's error word, and returns
@@ -85,7 +86,7 @@ FL_API const char* fl_status_string(int status);
  * fl_last_error naming the kernel and the cause), or FL_OK. */
 FL_API fl_status fl_device_status(void);
 
-/* Self-test of the failure path above: one thread waits, with a short limit, on a
+/* Self-test of the failure path above: one thread waits, with a deadline of 1 ms, on a
  * barrier that nothing completes, and records the time-out like a real wait would. The
  * next fl_device_status returns FL_ERR_TIMEOUT. */
 FL_API fl_status fl_selftest_wait_timeout(void* stream);
@@ -168,9 +169,11 @@ FL_API fl_status fl_level_map(const float* xy, int nblocks, const float* centers
 /*   w_d = s[r][c / 128] (u_d - 128 + c_d), u_d = u with its low 8 - d bits  */
 /*   cleared, c_d = (2^(8-d) - 1) / 2; a ZERO block gives y = 0.             */
 /* Arithmetic: codes enter an int8 tensor-core product exactly; x enters as  */
-/* a 15-bit fixed-point value per 128-column group (|error| <= 2^-14 of the  */
-/* group's max |x|); products accumulate in int32 per group and in fp32      */
-/* across groups.                                                            */
+/* a 31-bit fixed-point value per 128-column group (four int8 digits): every */
+/* element at least 2^-22 of the group's largest |x| is exact (bf16 has 8    */
+/* significant bits), a smaller one is off by at most 2^-30 of that largest  */
+/* |x|; products accumulate exactly in int32 per group and in fp32 across    */
+/* groups. The K-quant GEMV below uses the same activation form.             */
 /*                                                                           */
 /* levels   device, uint8 [out / 64], values 0..4 (0 ZERO .. 4 D8); values   */
 /*          above 4 are read as 4.                                           */
@@ -201,6 +204,12 @@ FL_API fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, 
  *     return FL_ERR_WORKSPACE; use fl_gemv_depth for them.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process, per device ordinal: it
+ *     does not survive cudaDeviceReset or a switch to another context on the
+ *     same device (the library's device image is loaded anew there), so do
+ *     not call this entry point after either.
+ *   - Every host-side check runs before anything is enqueued, so a rejected
+ *     call leaves the array untouched.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents; each call clears the part that must start at zero on
  *     its stream before the launch. Calls that overlap on the GPU (two

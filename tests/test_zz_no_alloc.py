@@ -1,9 +1,12 @@
-"""The allocation-free depth GEMV (fixed scratch array in the library's device image)
-against fl_gemv_depth with a caller workspace, through the C-ABI.
+"""The allocation-free depth GEMV (fixed scratch array in the library's device image),
+through the C-ABI.
 
 Two calls in a row on different shapes, batches and depth maps: the second runs on
 the scratch the first left behind. Both shapes split their columns across CTAs, so
-the scratch is really used. Bar: |y_static - y_workspace| <= 2e-3 * sum_c |w||x| + 1e-5.
+the scratch is really used. Each output is checked against the CPU oracle at the
+path's bar, |y_static - y_oracle| <= 2e-3 * sum_c |w||x| + 1e-5, and against
+fl_gemv_depth with a caller workspace at the same bar. Once the library's device
+image is loaded, further calls must not change the device's free memory.
 """
 import numpy as np
 import pytest
@@ -56,9 +59,41 @@ def test_static_scratch_matches_caller_workspace(env, orc, order):
         y_st = torch.full((batch, out), float("nan"), dtype=torch.float32, device="cuda")
         fl.fl_gemv_depth_static(w, lv_d, x_d, batch, y_st)
         torch.cuda.synchronize()
-        _, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
-        err = np.abs(y_st.cpu().numpy().astype(np.float64) - y_ws.cpu().numpy())
-        assert np.all(err <= REL * mass + ABS), (out, inn, batch, float(np.nanmax(err / (REL * mass + ABS))))
+        yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+        bound = REL * mass + ABS
+        y_static = y_st.cpu().numpy().astype(np.float64)
+        err = np.abs(y_static - yref)
+        assert np.all(err <= bound), (out, inn, batch, float(np.nanmax(err / bound)))
+        err_ws = np.abs(y_static - y_ws.cpu().numpy())
+        assert np.all(err_ws <= bound), (out, inn, batch, float(np.nanmax(err_ws / bound)))
+
+
+def test_static_calls_allocate_nothing(env):
+    """After one call has loaded the library's image, calls of several shapes leave the
+    device's free memory where it was (cudaMemGetInfo counts every allocation on the device,
+    torch's caching allocator included)."""
+    torch, fl = env
+    shapes = [(1024, 4096, 1), (2048, 6144, 3), (512, 14336, 16), (256, 1024, 2)]
+    bufs = []
+    for out, inn, batch in shapes:
+        q, s = synth.int8_layer(out, inn, 5, out)
+        store = torch.empty(fl.fl_plane_store_bytes(out, inn), dtype=torch.uint8, device="cuda")
+        fl.fl_pack_planes(_dev(torch, q), _dev(torch, s), out, inn, store)
+        lv = _dev(torch, synth.seeded_levels(out // 64, 6, out))
+        x = _dev(torch, synth.bf16_normal((batch, inn), 7, out))
+        y = torch.empty((batch, out), dtype=torch.float32, device="cuda")
+        bufs.append((fl.plane_weight(store, out, inn), lv, x, batch, y))
+    w, lv, x, batch, y = bufs[0]
+    fl.fl_gemv_depth_static(w, lv, x, batch, y)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        for w, lv, x, batch, y in bufs:
+            fl.fl_gemv_depth_static(w, lv, x, batch, y)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    fl.fl_device_status()
 
 
 def test_static_scratch_rejects_oversized_split(env):

@@ -85,11 +85,26 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded wait on an mbarrier phase. Returns false (and leaves the caller to
-// record the failure) if the phase has not completed after `limit` polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 26)) {
+// Nanoseconds on the GPU's global timer (advances at wall-clock rate, also while the context
+// is switched out).
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Deadline of every wait inside a kernel. A normal wait lasts microseconds; the limit leaves
+// room for the context being time-sliced with another process's work.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+// Wait on an mbarrier phase, bounded in time: each try_wait may suspend the thread for a
+// hardware-chosen interval, so the bound is a deadline on the global timer (read every 64
+// failed polls, counted from the first), not a poll count. Returns false (the caller records
+// the failure) if the phase has not completed by then.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t k = 0; k < limit; ++k) {
+  uint64_t t0 = 0;
+  for (uint32_t k = 1;; ++k) {
     uint32_t ok;
     asm volatile(
         "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
@@ -97,8 +112,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
         : "r"(a), "r"(parity)
         : "memory");
     if (ok) return true;
+    if (k == 1) t0 = globaltimer_ns();
+    if ((k & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
   }
-  return false;
 }
 
 // 1-D bulk copy global -> shared (own CTA), completion counted on `bar`.
@@ -140,13 +156,59 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
 // ---------------------------------------------------------------- activations as int8 digits
 //
 // For the int8 tensor-core products each 128-column group of each activation
-// row is written as a 15-bit fixed-point integer  v_c = rint(x_c 2^sigma)
-// with sigma = 14 - E, where max_c |x_c| < 2^E, so |v_c| <= 2^14; v_c is then
-// split into two balanced signed bytes  v_c = 256 hi_c + lo_c,
-// hi_c in [-64, 64], lo_c in [-128, 127].  The group keeps 2^-sigma (to undo
-// the scaling) and sum_c v_c (for the constant part of the reconstruction).
-// Absolute error per element <= 2^(E - 15) <= 2^-14 max |x_c|. The plane and
-// K-quant kernels build these digits in their prologues, each in the shared-memory
-// layout its tensor-core fragments read.
+// row is written as a 31-bit fixed-point integer  v_c = rint(x_c 2^sigma)
+// with sigma = 30 - E, where max_c |x_c| < 2^E, so |v_c| < 2^30; v_c is then
+// split into four balanced signed bytes
+//     v_c = 2^24 d3_c + 2^16 d2_c + 2^8 d1_c + d0_c,
+// d3_c in [-64, 64], the others in [-128, 127]. A bf16 value has 8
+// significant bits, so every element with |x_c| >= 2^-22 max_c |x_c| is
+// represented exactly (x_c 2^sigma is then an integer); a smaller element is
+// rounded, by at most 2^-sigma / 2 = 2^(E-31) <= 2^-30 of the group's largest |x|.
+// The products therefore reproduce sum_c w_c x_c exactly, up to the fp32
+// accumulation, unless a group spans more than 22 binades.
+//
+// The digits enter the products as two pairs per batch row, pair 0 = (d3, d2)
+// and pair 1 = (d1, d0); an MMA column pair is one digit pair, so a pair's
+// int32 sum is 256 C_hi + C_lo (|C| <= 2^22 per 128 columns, no overflow) and
+// weighs 2^16 2^-sigma (pair 0) or 2^-sigma (pair 1). The group keeps both
+// weights and 2^-sigma sum_c v_c (for the constant part of the
+// reconstruction). The plane and K-quant kernels build these digits in their
+// prologues, each in the shared-memory layout its tensor-core fragments read.
+//
+// split_digits: one warp, 128 columns (four per lane, f[] = this lane's
+// values). Writes the lane's four digit words (dw[k] byte i = digit 3-k of
+// element i: d3, d2, d1, d0) and the lane's pair sums (part.x = sum of
+// 256 d3 + d2, part.y = sum of 256 d1 + d0); returns sigma.
+__device__ __forceinline__ int split_digits(const float (&f)[4], uint32_t (&dw)[4], int2& part) {
+  uint32_t mb = 0;  // group max |x| (bit patterns of non-negative floats order like the values)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mb = max(mb, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+  mb = __reduce_max_sync(0xffffffffu, mb);
+  int E = 0;  // max |x| = mant * 2^E, mant in [0.5, 1)
+  if (mb >= 0x00800000u)
+    E = (int)(mb >> 23) - 126;
+  else if (mb != 0u)
+    frexpf(__uint_as_float(mb), &E);
+  const int sigma = (mb != 0u) ? (30 - E) : 0;
+  // v = rint(x 2^sigma): a power-of-two scale is exact, so one multiply when 2^sigma is normal
+  const bool direct = sigma >= -126 && sigma <= 127;
+  const float scale = __uint_as_float((uint32_t)(sigma + 127) << 23);
+  dw[0] = dw[1] = dw[2] = dw[3] = 0u;
+  part = make_int2(0, 0);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int v = __float2int_rn(direct ? f[i] * scale : ldexpf(f[i], sigma));
+    const int h1 = (v + 128) >> 8, d0 = v - 256 * h1;
+    const int h2 = (h1 + 128) >> 8, d1 = h1 - 256 * h2;
+    const int d3 = (h2 + 128) >> 8, d2 = h2 - 256 * d3;
+    dw[0] |= (static_cast<uint32_t>(d3) & 0xFFu) << (8 * i);
+    dw[1] |= (static_cast<uint32_t>(d2) & 0xFFu) << (8 * i);
+    dw[2] |= (static_cast<uint32_t>(d1) & 0xFFu) << (8 * i);
+    dw[3] |= (static_cast<uint32_t>(d0) & 0xFFu) << (8 * i);
+    part.x += h2;               // 256 d3 + d2
+    part.y += v - 65536 * h2;   // 256 d1 + d0
+  }
+  return sigma;
+}
 
 }  // namespace fl

@@ -98,8 +98,10 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
   if (lane == 0) s_cta[0] = r;
   bool ok = true;
   if (lane == 0) {
+    // bounded in time like every other wait (a deadline on the global timer)
     ok = false;
-    for (uint32_t k = 0; k < (1u << 24) && !ok; ++k) {
+    uint64_t t0 = 0;
+    for (uint32_t k = 1; !ok; ++k) {
       uint32_t done;
       asm volatile(
           "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0; selp.u32 %0, 1, 0, p; }"
@@ -107,6 +109,9 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
           : "r"(smem_u32(&s_bar))
           : "memory");
       ok = done != 0;
+      if (ok) break;
+      if (k == 1) t0 = globaltimer_ns();
+      if ((k & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
     if (!ok) atomicExch(&g_gate_error, 1);
   }

@@ -24,10 +24,12 @@
 //    from the plane words with one AND/OR per plane and one rotate per four
 //    columns (the store layout places each plane's field so that this yields
 //    u_d in byte lanes), feeds them as the u8 operand of mma.sync m16n8k32
-//    against the activations written as two signed int8 digits of a 15-bit
-//    per-group fixed point (built once per CTA for every slice it touches),
-//    and turns the int32 group sum into fp32 with the group scale and the
-//    constant part (c_b - c_a) sum_c x_c.
+//    against the activations written as four signed int8 digits of a 31-bit
+//    per-group fixed point (built once per CTA for every slice it touches;
+//    the digits go in as two pairs per batch row, each pair an MMA column
+//    pair), and turns the int32 group sums into fp32 with the group scale
+//    and the constant part (c_b - c_a) sum_c x_c; the two pairs' sums meet
+//    in one shuffle when the unit ends.
 //  * Layers with too few blocks to fill the GPU are split into column slices;
 //    a slice writes a partial to the caller's workspace and the last team to
 //    finish a block (atomic ticket) adds the slices in order. No CTA ever
@@ -51,7 +53,6 @@ constexpr int kProducerWarps = kTeams;  // producer warp t feeds team t
 constexpr int kThreads = kConsumers + 32 * kProducerWarps;
 constexpr int kTeamStages = 2;
 constexpr int kStages = kTeams * kTeamStages;
-constexpr int kStageBytes = 18432;
 constexpr int kMaxCtas = 960;   // unit ranges per launch (bounded by the kernel-parameter space)
 constexpr int kRed = 8;               // outputs per thread per pass of the slice reduction
 constexpr int kMaxSlots = 64;         // distinct (problem, slice) pairs one CTA may touch
@@ -59,10 +60,15 @@ constexpr int kLevelCache = 4096;     // most units per CTA; all their plane ran
 constexpr int kListCache = 512;       // most units per CTA of a listed pass; their block indices are cached
 constexpr int kSkipUnit = 0xFF;       // level-cache mark of a listed unit whose block index is out of range
 constexpr int kSmemLimit = 232448 - 16384;  // opt-in shared memory per block on B200, less static use
-constexpr int kDigitBudget = kSmemLimit - kStages * kStageBytes;
+// Stage size by N-tile count: 18 KB tiles while the products are light (batch <= 4); half that
+// at larger batches, whose four-digit activations need the shared memory and whose math per
+// weight byte is several times heavier, so fewer bytes in flight still keep up.
+__host__ __device__ constexpr int stage_bytes(int nt) { return nt <= 2 ? 18432 : 9216; }
+__host__ __device__ constexpr int digit_budget(int nt) { return kSmemLimit - kStages * stage_bytes(nt); }
 
-// Groups per tile for np planes: largest tg with tg * (256 + 2048 np) <= kStageBytes.
-__host__ __device__ constexpr int tile_groups(int np) { return np == 1 ? 8 : np == 2 ? 4 : 2; }
+// Groups per tile for np planes: largest tg with tg * (256 + 2048 np) <= stage_bytes(nt)
+// (8, 4, 2, 2 groups for 1-4 planes at 18 KB; 4, 2, 1, 1 at 9 KB).
+__host__ __device__ constexpr int tile_groups(int np, int nt) { return stage_bytes(nt) / (256 + 2048 * np); }
 
 struct Problem {
   const uint8_t* store;
@@ -112,8 +118,10 @@ __device__ int g_error;  // set when a bounded wait runs out (never expected)
 // One (problem, column slice) touched by a CTA: the units [u0, u1) of the CTA's range (relative
 // to its first unit) are its blocks b0, b0 + 1, ...; everything the producer and consumers need
 // is copied here once, so the hot loops never index the kernel-parameter problem table.
-// Activation digits: rows 2b / 2b+1 hold the hi / lo digits of batch row b (stride bytes per
-// row); gconst[(padded batch row) * ngroups + group] = (2^-sigma, 2^-sigma sum_c v_c).
+// Activation digits (fl_common.cuh): rows 4b .. 4b+3 hold digits d3, d2, d1, d0 of batch row b
+// (stride bytes per row), i.e. digit pair p = 2b + r (r = 0: d3 d2, r = 1: d1 d0) is rows 2p,
+// 2p+1; gconst[(padded pair row) * ngroups + group] = (pair weight, constant part): (2^(16 -
+// sigma), 2^-sigma sum_c v_c) for r = 0 and (2^-sigma, 0) for r = 1.
 struct __align__(16) Slot {
   int p, j, u0, u1, b0;
   int nblocks, G, ngroups, slices, gfirst;  // gfirst = first group of the slice in the row
@@ -192,38 +200,22 @@ __device__ __forceinline__ float cfac_of(int k0, int np) {
 __device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, int g, int lane) {
   const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
                       __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-  // group max |x| (the bit patterns of non-negative floats order like the values)
-  uint32_t mb = 0;
+  uint32_t dw[4];
+  int2 part;
+  const int sigma = split_digits(f, dw, part);
+  const uint32_t dh = sl.digits + (uint32_t)((4 * b) * sl.stride + 128 * g + 4 * lane);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) mb = max(mb, __float_as_uint(f[i]) & 0x7FFFFFFFu);
-  mb = __reduce_max_sync(0xffffffffu, mb);
-  int E = 0;  // m = mant * 2^E, mant in [0.5, 1)
-  if (mb >= 0x00800000u)
-    E = (int)(mb >> 23) - 126;
-  else if (mb != 0u)
-    frexpf(__uint_as_float(mb), &E);
-  const int sigma = (mb != 0u) ? (14 - E) : 0;
-  // v = rint(x 2^sigma): a power-of-two scale is exact, so one multiply when 2^sigma is normal
-  const bool direct = sigma >= -126 && sigma <= 127;
-  const float scale = __uint_as_float((uint32_t)(sigma + 127) << 23);
-  uint32_t hw = 0, lw = 0;
-  int part = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int vv = __float2int_rn(direct ? f[i] * scale : ldexpf(f[i], sigma));
-    const int h = (vv + 128) >> 8;
-    const int l = vv - 256 * h;
-    hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
-    lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
-    part += vv;
-  }
-  const uint32_t dh = sl.digits + (uint32_t)((2 * b) * sl.stride + 128 * g + 4 * lane);
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh), "r"(hw) : "memory");
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)sl.stride), "r"(lw) : "memory");
-  part = __reduce_add_sync(0xffffffffu, part);
+  for (int k = 0; k < 4; ++k)
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)(k * sl.stride)), "r"(dw[k]) : "memory");
+  part.x = __reduce_add_sync(0xffffffffu, part.x);
+  part.y = __reduce_add_sync(0xffffffffu, part.y);
   if (lane == 0) {
-    const uint32_t gc = sl.gconst + 8u * (uint32_t)(b * sl.ngroups + g);
-    asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(ldexpf(1.0f, -sigma)), "f"(ldexpf((float)part, -sigma))
+    const uint32_t gc = sl.gconst + 8u * (uint32_t)(2 * b * sl.ngroups + g);
+    asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc), "f"(ldexpf(1.0f, 16 - sigma)),
+                 "f"(ldexpf(fmaf(65536.f, (float)part.x, (float)part.y), -sigma))
+                 : "memory");
+    asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(gc + 8u * (uint32_t)sl.ngroups), "f"(ldexpf(1.0f, -sigma)),
+                 "f"(0.f)
                  : "memory");
   }
 }
@@ -262,11 +254,11 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
       }
     }
   }
-  // padded batch rows read zero constants
+  // padded pair rows read zero constants
   for (int i = 0; i < nsl; ++i) {
     const Slot& sl = slots[i];
-    for (int e = tid; e < (batch_pad - batch) * sl.ngroups; e += nthreads)
-      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(sl.gconst + 8u * (uint32_t)(batch * sl.ngroups + e)),
+    for (int e = tid; e < (batch_pad - 2 * batch) * sl.ngroups; e += nthreads)
+      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(sl.gconst + 8u * (uint32_t)(2 * batch * sl.ngroups + e)),
                    "f"(0.f), "f"(0.f)
                    : "memory");
   }
@@ -301,8 +293,8 @@ __device__ __forceinline__ void convert_staged(const Slot* slots, int nsl, int b
   }
   for (int i = 0; i < nsl; ++i) {
     const Slot& sl = slots[i];
-    for (int e = tid; e < (batch_pad - batch) * sl.ngroups; e += nthreads)
-      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(sl.gconst + 8u * (uint32_t)(batch * sl.ngroups + e)),
+    for (int e = tid; e < (batch_pad - 2 * batch) * sl.ngroups; e += nthreads)
+      asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(sl.gconst + 8u * (uint32_t)(2 * batch * sl.ngroups + e)),
                    "f"(0.f), "f"(0.f)
                    : "memory");
   }
@@ -358,8 +350,7 @@ __device__ __forceinline__ void group_compute(uint32_t wrow, uint32_t srow, int 
           acc[nt][0] = fmaf(v0, s0, acc[nt][0]);
           acc[nt][1] = fmaf(v1, s1, acc[nt][1]);
         }
-        return;
-      }
+      } else {
       uint4 B[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -408,6 +399,7 @@ __device__ __forceinline__ void group_compute(uint32_t wrow, uint32_t srow, int 
         acc[nt][0] = fmaf(v0, s0, acc[nt][0]);
         acc[nt][1] = fmaf(v1, s1, acc[nt][1]);
       }
+      }
 }
 
 // One tile for one warp: all tg groups of the tile. At batch <= 4 a full tile runs with a
@@ -417,7 +409,7 @@ template <int K0, int NP, int NT, bool FULL>
 __device__ __forceinline__ void tile_compute(uint32_t stage, int tg_arg, const uint32_t (&dlane)[NT],
                                              const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
                                              int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
-  constexpr int TG = tile_groups(NP);
+  constexpr int TG = tile_groups(NP, NT);
   const int tg = FULL ? TG : tg_arg;
   const uint32_t planes = stage + 256u * tg;
   const uint32_t wrow = planes + 32u * r0 + 8u * t;
@@ -439,7 +431,7 @@ __device__ __forceinline__ void dispatch_tile(int k0, int np, uint32_t stage, in
                                               const uint32_t (&dstep)[NT], uint32_t gc_lane, int gstride,
                                               int slice_goff, float cfac, int r0, int t, float (&acc)[NT][2]) {
 #define FL_TILE(K0_, NP_)                                                                            \
-  if (NT == 1 && tg == tile_groups(NP_))                                                            \
+  if (NT == 1 && tg == tile_groups(NP_, NT))                                                            \
     tile_compute<K0_, NP_, NT, true>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc); \
   else                                                                                               \
     tile_compute<K0_, NP_, NT, false>(stage, tg, dlane, dstep, gc_lane, gstride, slice_goff, cfac, r0, t, acc)
@@ -630,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   if (warp == 0) {
     // Slot table: lane i fills slot i, the i-th (problem, slice) pair from the CTA's first one
     // (a multi-problem launch has one slice per problem); digit areas laid out back to back.
-    const uint32_t base = smem_u32(smem + kStages * kStageBytes);
+    const uint32_t base = smem_u32(smem + kStages * stage_bytes(NT));
     const int s0 = a.cta_slice[blockIdx.x] >> 7, nsl_cta = a.cta_slice[blockIdx.x] & 127;
     uint32_t carry = 0;
     int items = 0, n = 0;
@@ -666,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         sl.y = P.y;
         sl.partial = P.partial;
         sl.tickets = P.tickets;
-        bytes = (uint32_t)(2 * a.batch * sl.stride + 8 * 4 * NT * sl.ngroups);
+        bytes = (uint32_t)(4 * a.batch * sl.stride + 8 * 4 * NT * sl.ngroups);
         nit = a.batch * sl.ngroups;
       }
       uint32_t incl = bytes;
@@ -682,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       }
       if (live) {
         sl.digits = base + carry + incl - bytes;
-        sl.gconst = sl.digits + (uint32_t)(2 * a.batch * sl.stride);
+        sl.gconst = sl.digits + (uint32_t)(4 * a.batch * sl.stride);
         sl.it0 = items + iincl - nit;
         slots[i] = sl;
       }
@@ -711,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   const int ditems = slots[nsl - 1].it0 + a.batch * slots[nsl - 1].ngroups;  // activation items
   const bool dmulti = ditems > 4 * kConsumerWarps;
   // staged: all activation rows fit the stage buffers, which stay idle until the digits are built
-  const bool dstaged = dmulti && ditems * 256 <= kStages * kStageBytes;
+  const bool dstaged = dmulti && ditems * 256 <= kStages * stage_bytes(NT);
   if (warp >= kConsumerWarps) {
     // ---------------------------------------------------------------- producer warps
     {
@@ -733,7 +725,11 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
     }
     named_bar(kBarProducers, 32 * kProducerWarps);
     bar_arrive(kBarLevels, kThreads);
-    if (dmulti) named_bar(kBarX, kThreads);
+    if (dmulti) {
+      named_bar(kBarX, kThreads);
+      // the staged activations never arrived: issue nothing into stages they may still reach
+      if (s_failed) return;
+    }
     if (lane != 0) return;
     const int team = warp - kConsumerWarps;
     int issued = 0, si = 0;
@@ -744,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       const int pr = (int)lvc[k];
       const int k0 = pr >> 4, np = pr & 15;
       if (np == 0 || (LISTED && pr == kSkipUnit)) continue;
-      const int tgm = tile_groups(np);
+      const int tgm = tile_groups(np, NT);
       const int ngs = sl.ngroups;
       const int G = sl.G;
       const uint8_t* blk = sl.store + (size_t)b * 8448u * G;
@@ -756,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
           atomicExch(&g_error, 1);
           return;
         }
-        uint8_t* st = smem + s * kStageBytes;
+        uint8_t* st = smem + s * stage_bytes(NT);
         const int gg = sl.gfirst + g0;
         const uint32_t bytes = 256u * tg + 2048u * tg * np;
         mbar_expect_tx(&full_bar[s], bytes);
@@ -778,13 +774,15 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   // 1. activation digits of every (problem, slice) the range touches
   if (dstaged) {
     if (threadIdx.x == 0) stage_x(slots, nsl, a.batch, smem, &x_bar, ditems);
-    if (!mbar_wait(&x_bar, 0u)) {
-      if (lane == 0) {
-        atomicExch(&g_error, 3);
-        s_failed = 1;
-      }
+    // warp-uniform outcome: a warp whose wait ran out converts nothing and flags the CTA
+    // before its arrive, so the producers (after kBarX) and every consumer (after kBarLevels)
+    // see the flag and the CTA skips its tiles
+    if (__all_sync(0xffffffffu, mbar_wait(&x_bar, 0u))) {
+      convert_staged(slots, nsl, a.batch, 4 * NT, smem, threadIdx.x, kConsumers, ditems);
+    } else if (lane == 0) {
+      atomicExch(&g_error, 3);
+      s_failed = 1;
     }
-    convert_staged(slots, nsl, a.batch, 4 * NT, smem, threadIdx.x, kConsumers, ditems);
     bar_arrive(kBarX, kThreads);  // the stage buffers are free for the weight stream
   } else {
     build_digits(slots, nsl, a.batch, 4 * NT, threadIdx.x, kConsumers, ditems, dmulti);
@@ -799,7 +797,11 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
   const uint32_t smem_base = smem_u32(smem);
   uint32_t dlane[NT], dstep[NT], gc_lane = 0;
   int cur_slot = -1, si = 0, used = 0;
-  bool failed = false;
+  // failed: a wait of this warp ran out (or the staged activations never arrived, CTA-uniform
+  // here). From then on the warp skips its waits and its math but still takes every team
+  // barrier below, so no named barrier is left short of a participant; the outputs are not
+  // valid and the error word says so.
+  bool failed = s_failed != 0;
   for (int k = team; k < nunits; k += kTeams) {
     while (si + 1 < nsl && k >= slots[si].u1) ++si;
     const Slot& sl = slots[si];
@@ -829,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int row = 8 * nt + g;
-        const bool liveb = row < 2 * a.batch;
+        const bool liveb = row < 4 * a.batch;
         dlane[nt] = liveb ? sl.digits + (uint32_t)(row * sl.stride + 32 * t) : smem_u32(zeros + 32 * t);
         dstep[nt] = liveb ? 128u : 0u;
       }
@@ -839,32 +841,39 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
     float acc[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-    const int tgm = tile_groups(np);
+    const int tgm = tile_groups(np, NT);
     for (int g0 = 0; g0 < sl.ngroups; g0 += tgm) {
       const int tg = min(tgm, sl.ngroups - g0);
       const int s = kTeamStages * team + (used % kTeamStages);
-      if (!mbar_wait(&full_bar[s], (uint32_t)((used / kTeamStages) & 1))) {
+      ++used;
+      if (failed) continue;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[s], (uint32_t)(((used - 1) / kTeamStages) & 1)))) {
         if (lane == 0) {
           atomicExch(&g_error, 2);
           s_failed = 1;
         }
         failed = true;
-        break;
+        continue;
       }
-      dispatch_tile<NT>(k0, np, smem_base + s * kStageBytes, tg, dlane, dstep, gc_lane, gstride, g0, cfac, r0, t,
+      dispatch_tile<NT>(k0, np, smem_base + s * stage_bytes(NT), tg, dlane, dstep, gc_lane, gstride, g0, cfac, r0, t,
                         acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);
-      ++used;
     }
-    if (failed) break;  // a stage never filled: stop, but still reach the CTA's last barrier
 
-    // ---- unit done: this warp's 16 rows are final (or a slice partial)
+    // ---- unit done: this warp's 16 rows are final (or a slice partial). Lane t holds digit
+    // pair t & 1 of batch row 2 nt + t / 2; the pairs' sums meet in one shuffle and the even
+    // lane writes.
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      acc[nt][0] += __shfl_xor_sync(0xffffffffu, acc[nt][0], 1);
+      acc[nt][1] += __shfl_xor_sync(0xffffffffu, acc[nt][1], 1);
+    }
     if (sl.slices == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int bb = 4 * nt + t;
-        if (bb < a.batch) {
+        const int bb = 2 * nt + (t >> 1);
+        if ((t & 1) == 0 && bb < a.batch) {
           float* y0 = y + (size_t)bb * ystride + row_base + g;
           if (a.mode == 1) {
             acc[nt][0] += y0[0];
@@ -878,8 +887,8 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
       // partial for this slice; the last team to finish the block adds the slices in order
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int bb = 4 * nt + t;
-        if (bb < a.batch) {
+        const int bb = 2 * nt + (t >> 1);
+        if ((t & 1) == 0 && bb < a.batch) {
           float* pp = sl.partial + (((size_t)sl.j * sl.nblocks + b) * a.batch + bb) * 64 + 16 * mt + g;
           pp[0] = acc[nt][0];
           pp[8] = acc[nt][1];
@@ -958,23 +967,26 @@ struct Plan {
   int slices, slice_groups;
 };
 
+// N-tiles of the products: two digit pairs per batch row, four pairs per 8-column N-tile.
+__host__ __device__ constexpr int ntiles(int batch) { return (batch + 1) / 2; }
+
 static size_t slot_bytes(int batch, int ngroups) {
-  const int nt = (batch + 3) / 4;
-  return (size_t)2 * batch * (128 * ngroups + 16) + (size_t)8 * 4 * nt * ngroups;
+  const int nt = ntiles(batch);
+  return (size_t)4 * batch * (128 * ngroups + 16) + (size_t)8 * 4 * nt * ngroups;
 }
 
 // Widest column slice (in 128-column groups) whose digits fit in one slot.
-static int max_groups_fit(int batch, long budget = kDigitBudget) {
-  const int nt = (batch + 3) / 4;
-  const long avail = budget - 32L * batch;
-  return (int)std::max(1L, avail / (256L * batch + 32L * nt));
+static int max_groups_fit(int batch, long budget) {
+  const int nt = ntiles(batch);
+  const long avail = budget - 64L * batch;
+  return (int)std::max(1L, avail / (512L * batch + 32L * nt));
 }
 
 // Column split for a single layer: enough units to fill the GPU, slices of whole
 // groups, and a slice narrow enough for the activation digits to fit in smem.
 static Plan plan_single(int nblocks, int G, int batch, int nsm) {
   Plan pl;
-  const int max_sg = max_groups_fit(batch);
+  const int max_sg = max_groups_fit(batch, digit_budget(ntiles(batch)));
   const int s_mem = (G + max_sg - 1) / max_sg;
   const int s_fill = (2 * nsm + nblocks - 1) / nblocks;
   int s = std::max(s_mem, std::min(s_fill, std::max(1, G / 4)));
@@ -992,8 +1004,10 @@ static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
 
 // Contiguous cost-balanced unit ranges, one per CTA (cost ~ columns read). A range is also
 // closed early when the digits of its distinct (problem, slice) pairs would overflow shared
-// memory, at kMaxSlots pairs, or at the level-cache size; such cuts can make more ranges than
-// SMs (a second, partial wave). The fused gate's epilogue (a reduction of the CTA's logits and
+// memory, at kMaxSlots pairs, or at the level-cache size; after every cut the cost still to
+// place is spread evenly over the ranges still to make, so an early cut does not leave a later
+// range oversized. Cuts can still make more ranges than SMs (a second, partial wave) when
+// memory forces more than that. The fused gate's epilogue (a reduction of the CTA's logits and
 // a publish, a few us) is charged to the gate problem's units, so the CTAs holding them get
 // fewer weight bytes.
 constexpr double kGateUnitWeight = 1.08;
@@ -1006,7 +1020,7 @@ static double unit_weight(const Args<MAXP>& a, int i) {
 }
 
 template <int MAXP>
-static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
+static bool partition(Args<MAXP>& a, int nsm, size_t budget) {
   double total = 0;
   int pairs = 0;
   for (int i = 0; i < a.nproblems; ++i) {
@@ -1017,7 +1031,8 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
   const int units = L.unit_begin + L.nblocks * L.slices;
   const int target = std::max(1, std::min(nsm, units));
   total += kSlotCost * (pairs + target - 1);  // about one slot per pair plus one per cut
-  const double per_cta = total / target;
+  double per_cta = total / target;
+  double start = 0;  // cumulative cost where the current range began
   int n = 0;
   a.cta_begin[0] = 0;
   a.cta_slice[0] = 0;
@@ -1034,7 +1049,7 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
         const int u = P.unit_begin + j * P.nblocks + b;
         bool cut = false;
         if (count > 0) {
-          if (n + 1 < target && acc + 0.5 * cost > per_cta * (n + 1)) cut = true;
+          if (n + 1 < target && acc + 0.5 * cost - start > per_cta) cut = true;
           if (b == 0 && (dig + sb > budget || nslots == kMaxSlots)) cut = true;
           if (count == (a.listed ? kListCache : kLevelCache)) cut = true;
         }
@@ -1046,6 +1061,8 @@ static bool partition(Args<MAXP>& a, int nsm, size_t budget = kDigitBudget) {
           dig = 0;
           nslots = 0;
           count = 0;
+          start = acc;
+          per_cta = (total - acc) / std::max(1, target - n);
         }
         if (b == 0 || count == 0) {
           dig += sb;
@@ -1073,31 +1090,30 @@ static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
   return FL_OK;
 }
 
-static fl_status launch_nt_gate(const Args<FL_MAX_PROBLEMS>& a, cudaStream_t st) {
-  switch ((a.batch + 3) / 4) {
-    case 1: return launch<FL_MAX_PROBLEMS, 1, true>(a, st);
-    case 2: return launch<FL_MAX_PROBLEMS, 2, true>(a, st);
-    case 3: return launch<FL_MAX_PROBLEMS, 3, true>(a, st);
-    default: return launch<FL_MAX_PROBLEMS, 4, true>(a, st);
+template <int MAXP, bool GATE, bool LISTED>
+static fl_status launch_by_batch(const Args<MAXP>& a, cudaStream_t st) {
+  switch (ntiles(a.batch)) {
+    case 1: return launch<MAXP, 1, GATE, LISTED>(a, st);
+    case 2: return launch<MAXP, 2, GATE, LISTED>(a, st);
+    case 3: return launch<MAXP, 3, GATE, LISTED>(a, st);
+    case 4: return launch<MAXP, 4, GATE, LISTED>(a, st);
+    case 5: return launch<MAXP, 5, GATE, LISTED>(a, st);
+    case 6: return launch<MAXP, 6, GATE, LISTED>(a, st);
+    case 7: return launch<MAXP, 7, GATE, LISTED>(a, st);
+    default: return launch<MAXP, 8, GATE, LISTED>(a, st);
   }
+}
+
+static fl_status launch_nt_gate(const Args<FL_MAX_PROBLEMS>& a, cudaStream_t st) {
+  return launch_by_batch<FL_MAX_PROBLEMS, true, false>(a, st);
 }
 
 template <int MAXP>
 static fl_status launch_nt(const Args<MAXP>& a, cudaStream_t st) {
   if constexpr (MAXP > 1) {
-    if (a.listed) switch ((a.batch + 3) / 4) {
-        case 1: return launch<MAXP, 1, false, true>(a, st);
-        case 2: return launch<MAXP, 2, false, true>(a, st);
-        case 3: return launch<MAXP, 3, false, true>(a, st);
-        default: return launch<MAXP, 4, false, true>(a, st);
-      }
+    if (a.listed) return launch_by_batch<MAXP, false, true>(a, st);
   }
-  switch ((a.batch + 3) / 4) {
-    case 1: return launch<MAXP, 1, false>(a, st);
-    case 2: return launch<MAXP, 2, false>(a, st);
-    case 3: return launch<MAXP, 3, false>(a, st);
-    default: return launch<MAXP, 4, false>(a, st);
-  }
+  return launch_by_batch<MAXP, false, false>(a, st);
 }
 
 static fl_status check_weight(const fl_plane_weight* w, const char* what) {
@@ -1109,9 +1125,11 @@ static fl_status check_weight(const fl_plane_weight* w, const char* what) {
   return FL_OK;
 }
 
-static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const uint8_t* lv_to, const uint16_t* x,
-                        int batch, float* y, void* ws, size_t ws_bytes, void* stream, int mode,
-                        const char* what) {
+// Every host-side check of a single-layer call, then its launch parameters in `a`; nothing is
+// enqueued.
+static fl_status prepare_single(Args<1>& a, const fl_plane_weight* w, const uint8_t* lv_from, const uint8_t* lv_to,
+                                const uint16_t* x, int batch, float* y, void* ws, size_t ws_bytes, int mode,
+                                const char* what) {
   fl_status st = check_weight(w, what);
   if (st != FL_OK) return st;
   if (!lv_from || !x || !y || (mode == 1 && !lv_to)) return fail(FL_ERR_ARG, "%s: NULL pointer argument", what);
@@ -1126,7 +1144,6 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
   if (need > 0 && (!ws || ws_bytes < need))
     return fail(FL_ERR_WORKSPACE, "%s: workspace %zu bytes, need %zu", what, ws ? ws_bytes : (size_t)0, need);
   if (need > 0 && !aligned16(ws)) return fail(FL_ERR_ALIGN, "%s: workspace not 16-byte aligned", what);
-  static thread_local Args<1> a;
   a.nproblems = 1;
   a.batch = batch;
   a.mode = mode;
@@ -1155,7 +1172,17 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
     P.tickets = nullptr;
     P.partial = nullptr;
   }
-  if (!partition(a, nsm)) return fail(FL_ERR_SHAPE, "%s: layer too large for one launch", what);
+  if (!partition(a, nsm, (size_t)digit_budget(ntiles(batch))))
+    return fail(FL_ERR_SHAPE, "%s: layer too large for one launch", what);
+  return FL_OK;
+}
+
+static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const uint8_t* lv_to, const uint16_t* x,
+                        int batch, float* y, void* ws, size_t ws_bytes, void* stream, int mode,
+                        const char* what) {
+  static thread_local Args<1> a;
+  const fl_status st = prepare_single(a, w, lv_from, lv_to, x, batch, y, ws, ws_bytes, mode, what);
+  if (st != FL_OK) return st;
   return launch_nt(a, static_cast<cudaStream_t>(stream));
 }
 
@@ -1208,7 +1235,7 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
   if (reinterpret_cast<uintptr_t>(runs) & 3u) return fail(FL_ERR_ALIGN, "%s: runs not 4-byte aligned", what);
   if (lists != nullptr && (counts == nullptr || gate != nullptr))
     return fail(FL_ERR_ARG, "%s: a listed pass needs counts and has no gate", what);
-  size_t budget = kDigitBudget;
+  size_t budget = (size_t)digit_budget(ntiles(batch));
   if (gate) {
     if (gate->problem < 0 || gate->problem >= n)
       return fail(FL_ERR_ARG, "%s: gate problem %d not in 0..%d", what, gate->problem, n - 1);
@@ -1337,19 +1364,21 @@ int take_device_error() {
   return v;
 }
 
-// One thread waits (100 polls) on a barrier that expects an arrival nobody makes.
-__global__ void selftest_timeout_kernel() {
+// One thread waits on a barrier that expects an arrival nobody makes, with the given deadline
+// (the same bounded wait as the kernels' stage barriers, shorter).
+__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   mbar_init(&bar, 1);
   fence_mbar_init();
-  if (!mbar_wait(&bar, 0u, 100u)) atomicExch(&g_error, 4);
+  if (!mbar_wait(&bar, 0u, limit_ns)) atomicExch(&g_error, 4);
 }
 
 }  // namespace gemv
 }  // namespace fl
 
 extern "C" fl_status fl_selftest_wait_timeout(void* stream) {
-  FL_CHECK_CUDA(launch_pdl(gemv::selftest_timeout_kernel, dim3(1), dim3(1), 0, static_cast<cudaStream_t>(stream), 1),
+  FL_CHECK_CUDA(launch_pdl(gemv::selftest_timeout_kernel, dim3(1), dim3(1), 0, static_cast<cudaStream_t>(stream), 1,
+                           (uint64_t)1000000u),
                 "launch selftest_timeout");
   return FL_OK;
 }
@@ -1405,11 +1434,16 @@ extern "C" fl_status fl_gemv_depth_static(const fl_plane_weight* w, const uint8_
   if (need > 0) {
     st = gemv::static_scratch(&scratch, what);
     if (st != FL_OK) return st;
+  }
+  static thread_local gemv::Args<1> a;
+  st = gemv::prepare_single(a, w, levels, nullptr, x, batch, y, scratch,
+                            need > 0 ? (size_t)FL_GEMV_STATIC_SCRATCH_BYTES : 0, 0, what);
+  if (st != FL_OK) return st;  // rejected before anything is enqueued: the shared array is untouched
+  if (need > 0) {
     // the split's tickets start at zero; the partials are written before they are read
     const size_t tickets = ((size_t)nblocks * 4 + 255) / 256 * 256;
     FL_CHECK_CUDA(cudaMemsetAsync(scratch, 0, tickets, static_cast<cudaStream_t>(stream)),
                   "cudaMemsetAsync(static scratch tickets)");
   }
-  return gemv::single(w, levels, nullptr, x, batch, y, scratch, need > 0 ? (size_t)FL_GEMV_STATIC_SCRATCH_BYTES : 0,
-                      stream, 0, what);
+  return gemv::launch_nt(a, static_cast<cudaStream_t>(stream));
 }

@@ -14,9 +14,11 @@
 // 64 rows x 1 Q6_K super-block = 13440 B) is one contiguous 1-D bulk copy. Codes become u8
 // tensor-core operands with one or two mask/shift operations per four weights (the record
 // layouts are built for it); each sub-block is one mma.sync (m16n8k32 for Q4_K's 32-weight
-// sub-blocks, m16n8k16 for Q6_K's 16-weight ones) against the activations' int8 digits; the
-// sub-block scale is applied to the int32 result with an integer multiply-add, and each
-// 128-column half of a super-block is converted to fp32 once.
+// sub-blocks, m16n8k16 for Q6_K's 16-weight ones) against the activations' four int8 digits
+// (fl_common.cuh; two digit pairs per batch row, one MMA column pair each); the sub-block
+// scale is applied to the int32 result with an integer multiply-add, each 128-column half of a
+// super-block is converted to fp32 once per pair, and a batch row's two pairs meet in one
+// shuffle when the unit ends.
 #include <algorithm>
 
 #include "fl_common.cuh"
@@ -70,9 +72,11 @@ struct Args {
 __device__ int g_error;  // set when a bounded wait runs out (never expected)
 
 // One (problem, column slice) touched by a CTA; see the plane-store GEMV for the scheme.
-// Activation digits: rows 2b / 2b+1 hold the hi / lo digits of batch row b (stride bytes per
-// row, Q4_K slots in the permuted order its MMA fragments read); per (padded batch row,
-// 128-column group): iscale = 2^-sigma and gsum = 8 sums of 16 columns.
+// Activation digits: rows 4b .. 4b+3 hold digits d3, d2, d1, d0 of batch row b (stride bytes
+// per row, Q4_K slots in the permuted order its MMA fragments read), i.e. digit pair p = 2b + r
+// is rows 2p, 2p+1; per (padded pair row, 128-column group): iscale = the pair's weight
+// (2^(16 - sigma) for r = 0, 2^-sigma for r = 1) and gsum = 8 sums of 16 columns of the pair's
+// value (256 d3 + d2, or 256 d1 + d0).
 struct __align__(16) Slot {
   int p, j, u0, u1, b0;
   int nblocks, nsb, nsbs, slices, sbfirst;  // nsbs = super-blocks of the slice
@@ -155,9 +159,9 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
   return old;
 }
 
-// A slot's digit area, batch rows padded to 4 NT. The padded strides spread the rows that
+// A slot's digit area, pair rows padded to 4 NT. The padded strides spread the rows that
 // one warp reads together over distinct shared-memory banks.
-//   digits: 2 batch rows of digit_stride bytes (hi, lo)
+//   digits: 4 rows of digit_stride bytes per batch row (d3, d2, d1, d0)
 //   iscale: [4 NT][ngroups + 1] floats, area rounded up to 16 bytes
 //   gsum:   [4 NT][gsum_row bytes]: per 128-column group 8 int32 sums of 16 columns
 __host__ __device__ constexpr int digit_stride(int ngroups) { return 128 * ngroups + 32; }
@@ -165,7 +169,7 @@ __host__ __device__ constexpr int iscale_row(int ngroups) { return ngroups + 1; 
 __host__ __device__ constexpr int gsum_row(int ngroups) { return 32 * ngroups + 16; }
 __host__ __device__ constexpr int iscale_area(int nt, int ngroups) { return (16 * nt * iscale_row(ngroups) + 15) & ~15; }
 __host__ __device__ constexpr int slot_area(int batch, int nt, int ngroups) {
-  return 2 * batch * digit_stride(ngroups) + iscale_area(nt, ngroups) + 4 * nt * gsum_row(ngroups);
+  return 4 * batch * digit_stride(ngroups) + iscale_area(nt, ngroups) + 4 * nt * gsum_row(ngroups);
 }
 
 // Rows of the 64-row block held by lane row g of warp mt: Q4_K records (144 B) are
@@ -201,44 +205,31 @@ __device__ __forceinline__ uint32_t lds_u32_if(uint32_t a, bool p) {
 __device__ __forceinline__ void convert_item(uint2 raw, const Slot& sl, int b, int g, int lane) {
   const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
                       __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
-  uint32_t mb = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) mb = max(mb, __float_as_uint(f[i]) & 0x7FFFFFFFu);
-  mb = __reduce_max_sync(0xffffffffu, mb);
-  int E = 0;  // max |x| = mant * 2^E, mant in [0.5, 1)
-  if (mb >= 0x00800000u)
-    E = (int)(mb >> 23) - 126;
-  else if (mb != 0u)
-    frexpf(__uint_as_float(mb), &E);
-  const int sigma = (mb != 0u) ? (14 - E) : 0;
-  const bool direct = sigma >= -126 && sigma <= 127;
-  const float scale = __uint_as_float((uint32_t)(sigma + 127) << 23);
-  uint32_t hw = 0, lw = 0;
-  int part = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int vv = __float2int_rn(direct ? f[i] * scale : ldexpf(f[i], sigma));
-    const int h = (vv + 128) >> 8;
-    const int l = vv - 256 * h;
-    hw |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * i);
-    lw |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * i);
-    part += vv;
-  }
+  uint32_t dw[4];
+  int2 part;
+  const int sigma = split_digits(f, dw, part);
   const int wpos = (sl.type == FL_GGML_Q4_K) ? (8 * (lane >> 3) + 2 * (lane & 3) + ((lane >> 2) & 1)) : lane;
-  const uint32_t dh = sl.digits + (uint32_t)((2 * b) * sl.stride + 128 * g + 4 * wpos);
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh), "r"(hw) : "memory");
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)sl.stride), "r"(lw) : "memory");
-  // sums of 16 columns (4 lanes each)
-  part += __shfl_xor_sync(0xffffffffu, part, 1);
-  part += __shfl_xor_sync(0xffffffffu, part, 2);
-  if ((lane & 3) == 0)
-    asm volatile("st.shared.s32 [%0], %1;" ::"r"(sl.gsum + (uint32_t)(b * gsum_row(sl.ngroups) + 32 * g + (lane & ~3))),
-                 "r"(part)
-                 : "memory");
-  if (lane == 0)
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)(b * iscale_row(sl.ngroups) + g)),
+  const uint32_t dh = sl.digits + (uint32_t)((4 * b) * sl.stride + 128 * g + 4 * wpos);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(dh + (uint32_t)(k * sl.stride)), "r"(dw[k]) : "memory");
+  // sums of 16 columns (4 lanes each), per digit pair
+  part.x += __shfl_xor_sync(0xffffffffu, part.x, 1);
+  part.x += __shfl_xor_sync(0xffffffffu, part.x, 2);
+  part.y += __shfl_xor_sync(0xffffffffu, part.y, 1);
+  part.y += __shfl_xor_sync(0xffffffffu, part.y, 2);
+  const uint32_t gs0 = sl.gsum + (uint32_t)(2 * b * gsum_row(sl.ngroups) + 32 * g + (lane & ~3));
+  if ((lane & 3) == 0) {
+    asm volatile("st.shared.s32 [%0], %1;" ::"r"(gs0), "r"(part.x) : "memory");
+    asm volatile("st.shared.s32 [%0], %1;" ::"r"(gs0 + (uint32_t)gsum_row(sl.ngroups)), "r"(part.y) : "memory");
+  }
+  if (lane == 0) {
+    const uint32_t is0 = sl.iscale + 4u * (uint32_t)(2 * b * iscale_row(sl.ngroups) + g);
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(is0), "f"(ldexpf(1.0f, 16 - sigma)) : "memory");
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(is0 + 4u * (uint32_t)iscale_row(sl.ngroups)),
                  "f"(ldexpf(1.0f, -sigma))
                  : "memory");
+  }
 }
 
 // All consumer threads; every thread arrives once on kBarX after its last round of loads is
@@ -275,12 +266,12 @@ __device__ __forceinline__ void build_digits(const Slot* slots, int nsl, int bat
       }
     }
   }
-  // padded batch rows read zero scales and sums
+  // padded pair rows read zero scales and sums
   for (int i = 0; i < nsl; ++i) {
     const Slot& sl = slots[i];
-    const int n = (batch_pad - batch) * sl.ngroups;
+    const int n = (batch_pad - 2 * batch) * sl.ngroups;
     for (int e = tid; e < 9 * n; e += nthreads) {
-      const int b = batch + (e % n) / sl.ngroups, g = (e % n) % sl.ngroups;
+      const int b = 2 * batch + (e % n) / sl.ngroups, g = (e % n) % sl.ngroups;
       if (e < n)
         asm volatile("st.shared.f32 [%0], %1;" ::"r"(sl.iscale + 4u * (uint32_t)(b * iscale_row(sl.ngroups) + g)),
                      "f"(0.f)
@@ -341,10 +332,10 @@ __device__ __forceinline__ void q4k_half(uint32_t rec0, uint32_t rec1, int half,
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int bb = 4 * nt + t;
-    const float isc = lds_f32(iscale + 4u * (uint32_t)(bb * iscale_row(gstride) + gi));
+    const int pr = 4 * nt + t;  // the lane's digit-pair row
+    const float isc = lds_f32(iscale + 4u * (uint32_t)(pr * iscale_row(gstride) + gi));
     // sums over the 32-column sub-blocks from the 16-column sums
-    const uint32_t ga = gsum + (uint32_t)(bb * gsum_row(gstride) + 32 * gi);
+    const uint32_t ga = gsum + (uint32_t)(pr * gsum_row(gstride) + 32 * gi);
     const int4 Xa = lds_s4(ga);
     const int4 Xb = lds_s4(ga + 16u);
     const int32_t X0 = Xa.x + Xa.y, X1 = Xa.z + Xa.w, X2 = Xb.x + Xb.y, X3 = Xb.z + Xb.w;
@@ -523,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       }
       if (live) {
         sl.digits = base + carry + incl - bytes;
-        sl.iscale = sl.digits + (uint32_t)(2 * a.batch * sl.stride);
+        sl.iscale = sl.digits + (uint32_t)(4 * a.batch * sl.stride);
         sl.gsum = sl.iscale + (uint32_t)iscale_area(NT, sl.ngroups);
         sl.it0 = items + iincl - nit;
         slots[i] = sl;
@@ -586,6 +577,10 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
   bool live[NT];
   int row0 = 0, row1 = 0;
   int cur_slot = -1, si = 0, used = 0;
+  // failed: a wait of this warp ran out. From then on the warp skips its waits and its math but
+  // still takes every team barrier below, so no named barrier is left short of a participant;
+  // the outputs are not valid and the error word says so.
+  bool failed = false;
   for (int k = team; k < nunits; k += kTeams) {
     while (si + 1 < nsl && k >= slots[si].u1) ++si;
     const Slot& sl = slots[si];
@@ -595,9 +590,9 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       cur_slot = si;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int row = 8 * nt + g;  // digit row (2 per batch row) this lane's B fragment reads
-        live[nt] = row < 2 * a.batch;
-        dl[nt] = sl.digits + (uint32_t)(min(row, 2 * a.batch - 1) * sl.stride) + (q4 ? 8u * t : 4u * t);
+        const int row = 8 * nt + g;  // digit row (4 per batch row) this lane's B fragment reads
+        live[nt] = row < 4 * a.batch;
+        dl[nt] = sl.digits + (uint32_t)(min(row, 4 * a.batch - 1) * sl.stride) + (q4 ? 8u * t : 4u * t);
       }
       row0 = q4 ? 16 * mt + g : q6_row(mt, 0, g);
       row1 = q4 ? 16 * mt + g + 8 : q6_row(mt, 1, g);
@@ -610,9 +605,12 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
     const int tsbm = q4 ? 2 : 1;
     for (int s0 = 0; s0 < sl.nsbs; s0 += tsbm) {
       const int s = kTeamStages * team + (used % kTeamStages);
-      if (!mbar_wait(&full_bar[s], (uint32_t)((used / kTeamStages) & 1))) {
+      ++used;
+      if (failed) continue;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full_bar[s], (uint32_t)(((used - 1) / kTeamStages) & 1)))) {
         if (lane == 0) atomicExch(&g_error, 2);
-        return;
+        failed = true;
+        continue;
       }
       const uint32_t stage = smem_base + s * kStageBytes;
       if (!q4)
@@ -623,16 +621,22 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
         tile_q4<NT, 1>(stage, dl, live, iscale, gsum, gstride, s0, row0, row1, t, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);
-      ++used;
     }
 
-    // ---- unit done: this warp's 16 rows are final (or a slice partial)
+    // ---- unit done: this warp's 16 rows are final (or a slice partial). Lane t holds digit
+    // pair t & 1 of batch row 2 nt + t / 2; the pairs' sums meet in one shuffle and the even
+    // lane writes.
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      acc[nt][0] += __shfl_xor_sync(0xffffffffu, acc[nt][0], 1);
+      acc[nt][1] += __shfl_xor_sync(0xffffffffu, acc[nt][1], 1);
+    }
     const size_t ystride = (size_t)64 * sl.nblocks;
     if (sl.slices == 1) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int bb = 4 * nt + t;
-        if (bb < a.batch) {
+        const int bb = 2 * nt + (t >> 1);
+        if ((t & 1) == 0 && bb < a.batch) {
           float* yb = sl.y + (size_t)bb * ystride + 64 * b;
           yb[row0] = acc[nt][0];
           yb[row1] = acc[nt][1];
@@ -642,8 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1) kquant_gemv_kernel(const __grid_c
       // partial for this slice; the last team to finish the block adds the slices in order
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int bb = 4 * nt + t;
-        if (bb < a.batch) {
+        const int bb = 2 * nt + (t >> 1);
+        if ((t & 1) == 0 && bb < a.batch) {
           float* pp = sl.partial + (((size_t)sl.j * sl.nblocks + b) * a.batch + bb) * 64;
           pp[row0] = acc[nt][0];
           pp[row1] = acc[nt][1];
@@ -702,7 +706,10 @@ struct Plan {
 };
 
 // Shared memory of one slot's activation digits, scales and 16-column sums.
-static size_t slot_bytes(int batch, int nsbs) { return (size_t)slot_area(batch, (batch + 3) / 4, 2 * nsbs); }
+// N-tiles of the products: two digit pairs per batch row, four pairs per 8-column N-tile.
+__host__ __device__ constexpr int ntiles(int batch) { return (batch + 1) / 2; }
+
+static size_t slot_bytes(int batch, int nsbs) { return (size_t)slot_area(batch, ntiles(batch), 2 * nsbs); }
 
 // Widest column slice (in super-blocks) whose digits fit in one slot.
 static int max_sb_fit(int batch) {
@@ -733,7 +740,9 @@ static size_t workspace_for(const Plan& pl, int nblocks, int batch) {
 
 // Contiguous byte-balanced unit ranges, one per CTA. A range is also closed early when the
 // digits of its distinct (problem, slice) pairs would overflow shared memory or at kMaxSlots
-// pairs; such cuts can make more ranges than SMs (a second, partial wave).
+// pairs; after every cut the cost still to place is spread evenly over the ranges still to
+// make, so an early cut does not leave a later range oversized. Cuts can still make more
+// ranges than SMs (a second, partial wave) when memory forces more than that.
 template <int MAXP>
 static bool partition(Args<MAXP>& a, int nsm) {
   double total = 0;
@@ -741,7 +750,8 @@ static bool partition(Args<MAXP>& a, int nsm) {
   const Problem& L = a.p[a.nproblems - 1];
   const int units = L.unit_begin + L.nblocks * L.slices;
   const int target = std::max(1, std::min(nsm, units));
-  const double per_cta = total / target;
+  double per_cta = total / target;
+  double start = 0;  // cumulative cost where the current range began
   int n = 0;
   a.cta_begin[0] = 0;
   a.cta_slice[0] = 0;
@@ -758,7 +768,7 @@ static bool partition(Args<MAXP>& a, int nsm) {
         const int u = P.unit_begin + j * P.nblocks + b;
         bool cut = false;
         if (count > 0) {
-          if (n + 1 < target && acc + 0.5 * cost > per_cta * (n + 1)) cut = true;
+          if (n + 1 < target && acc + 0.5 * cost - start > per_cta) cut = true;
           if (b == 0 && (dig + sb > (size_t)kDigitBudget || nslots == kMaxSlots)) cut = true;
         }
         if (cut) {
@@ -769,6 +779,8 @@ static bool partition(Args<MAXP>& a, int nsm) {
           dig = 0;
           nslots = 0;
           count = 0;
+          start = acc;
+          per_cta = (total - acc) / std::max(1, target - n);
         }
         if (b == 0 || count == 0) {
           dig += sb;
@@ -797,11 +809,15 @@ static fl_status launch(const Args<MAXP>& a, cudaStream_t st) {
 
 template <int MAXP>
 static fl_status launch_nt(const Args<MAXP>& a, cudaStream_t st) {
-  switch ((a.batch + 3) / 4) {
+  switch (ntiles(a.batch)) {
     case 1: return launch<MAXP, 1>(a, st);
     case 2: return launch<MAXP, 2>(a, st);
     case 3: return launch<MAXP, 3>(a, st);
-    default: return launch<MAXP, 4>(a, st);
+    case 4: return launch<MAXP, 4>(a, st);
+    case 5: return launch<MAXP, 5>(a, st);
+    case 6: return launch<MAXP, 6>(a, st);
+    case 7: return launch<MAXP, 7>(a, st);
+    default: return launch<MAXP, 8>(a, st);
   }
 }
 

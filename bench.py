@@ -50,10 +50,14 @@ def parse():
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["fl", "reference"], default="fl")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config kernel measurements")
-    ap.add_argument("--profile", choices=["none", "step", "kquant", "kernels"], default="none",
+    ap.add_argument("--profile", choices=["none", "step", "kquant", "kernels", "layer"], default="none",
                     help="short run for an ncu capture: 'step' = the decode step only, 'kquant' = the K-quant "
-                         "step only, 'kernels' = one pass of every per-config kernel measurement; no JSON "
+                         "step only, 'kernels' = one pass of every per-config kernel measurement, 'layer' = "
+                         "three fl_gemv_depth calls on one layer (--shape, --batch, --level); no JSON "
                          "timing claims")
+    ap.add_argument("--shape", default="4096,4096", help="--profile layer: out,in")
+    ap.add_argument("--batch", type=int, default=1, help="--profile layer: tokens per call")
+    ap.add_argument("--level", type=int, default=3, help="--profile layer: depth level of every block (3 = D6)")
     return ap.parse_args()
 
 
@@ -69,7 +73,9 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi SM clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi SM clock / throttle-reason samples, every 10 ms, from before the warm-up to the
+    end of the timing (a device-timed region of a few ms would otherwise fall between samples),
+    plus NVML readings taken right before and right after the timed region itself."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -79,11 +85,12 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.marks = {}
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "10"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -103,6 +110,20 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
+    def mark(self, key):
+        """NVML reading of the SM clock and the active throttle reasons, stored under key."""
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            names = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+                     0x4: "sw_power_cap"}
+            self.marks[key] = {"sm_mhz": mhz, "reasons": sorted(n for b, n in names.items() if bits & b)}
+        except Exception as e:
+            self.marks[key] = {"error": str(e)[:120]}
+
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -118,10 +139,13 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+        window = "10 ms nvidia-smi samples from before the warm-up to the end of the kernel timing"
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": window,
+                    **self.marks}
         sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "window": window, **self.marks}
 
 
 def src_sha(*names):
@@ -142,6 +166,16 @@ def traffic_record(kernel_key):
         return rec
     except Exception:
         return None
+
+
+def device_ok(fl, what):
+    """The kernels' error words after a timed region: a bounded wait that ran out (or a bad list
+    entry) makes that region's outputs invalid, so its number is not printed."""
+    try:
+        fl.fl_device_status()
+    except fl.FlError as e:
+        raise SystemExit(json.dumps({"error": f"device status after {what}: {e}", "value": None}))
+    return "ok"
 
 
 def max_over_ranks(t, world, device="cuda"):
@@ -173,11 +207,27 @@ def gpu_int8_layer(torch, out, inn, gen):
     return q, s.contiguous()
 
 
-def plane_layer(torch, fl, out, inn, gen):
+def plane_layer(torch, fl, out, inn, gen, keep_block0=False):
     q, s = gpu_int8_layer(torch, out, inn, gen)
     store = torch.empty(fl.fl_plane_store_bytes(out, inn), dtype=torch.uint8, device="cuda")
     fl.fl_pack_planes(q, s, out, inn, store)
+    if keep_block0:  # the first 64-row block's codes and scales, for the in-run output check
+        return store, (q[:64].cpu().numpy(), s[:64].cpu().numpy())
     return store
+
+
+def block_reference(q, s, level, x_bits):
+    """Plain float64 outputs of one 64-row block read at `level` (the depth rule written out:
+    w_d = s (u_d - 128 + c_d), u = q + 128 with its low 8 - d bits cleared, c_d = (2^(8-d) - 1) / 2)
+    and the bar's mass sum_c |w_d| |x_c|."""
+    import numpy as np
+    d = 2 * level
+    u = q.astype(np.int64) + 128
+    ud = u & ~((1 << (8 - d)) - 1)
+    cd = ((1 << (8 - d)) - 1) / 2.0
+    w = np.repeat(s.astype(np.float64), 128, axis=1) * (ud - 128 + cd)
+    x = (x_bits.astype(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return w @ x, np.abs(w) @ np.abs(x)
 
 
 def plane_bytes(inn, level):
@@ -215,8 +265,15 @@ class DecodeStep:
         oi = oo = 0
         self.bytes_d4 = self.bytes_res = 0
         self.levels = []
-        for name, o, i in self.shapes:
-            st = plane_layer(torch, fl, o, i, gen)
+        # problems whose first 64-row block the run checks: the first layer, the first down
+        # projection (in 3072) and the head
+        self.sample_idx = (0, 6, len(self.shapes) - 1)
+        self.samples = {}
+        for pi, (name, o, i) in enumerate(self.shapes):
+            st = plane_layer(torch, fl, o, i, gen, keep_block0=pi in self.sample_idx)
+            if pi in self.sample_idx:
+                st, qs = st
+                self.samples[pi] = (qs, oi, oo, i)
             self.stores.append(st)
             d4 = torch.full((o // 64,), 2, dtype=torch.uint8, device="cuda")
             d8 = torch.full((o // 64,), 4, dtype=torch.uint8, device="cuda")
@@ -267,7 +324,24 @@ class DecodeStep:
         M = self.gates[:, 1].view(torch.float32).cpu().numpy().astype(np.float64)
         h = np.sort(H)[::-1]
         self.calib = {"entropy_sorted": h.tolist(), "margin_min": float(M.min())}
-        return float(0.5 * (h[self.NESC - 1] + h[self.NESC])), float(0.5 * M.min())
+        tau_h, tau_m = float(0.5 * (h[self.NESC - 1] + h[self.NESC])), float(0.5 * M.min())
+        self.esc_sets = [bool(H[j] > tau_h or M[j] < tau_m) for j in range(self.NSETS)]
+        return tau_h, tau_m
+
+    def check_outputs(self, j):
+        """The sampled blocks of the step last run (input set j) against block_reference at the
+        level the device ran (D8 for an escalating set, else D4): the largest error as a fraction
+        of the path's bar 2e-3 sum |w||x| + 1e-5."""
+        import numpy as np
+        lv = 4 if self.esc_sets[j] else 2
+        y = self.y.cpu().numpy()
+        worst = 0.0
+        for pi, ((q, s), oi, oo, i) in self.samples.items():
+            yref, mass = block_reference(q, s, lv, self.hx[j][oi:oi + i])
+            err = np.abs(y[oo:oo + 64].astype(np.float64) - yref)
+            worst = max(worst, float((err / (2e-3 * mass + 1e-5)).max()))
+        return {"input_set": j, "level": f"D{2 * lv}", "blocks": len(self.samples), "max_err_ratio": worst,
+                "ok": worst <= 1.0}
 
     def step_graph_body(self, j, buf=0):
         fl = self.fl
@@ -301,6 +375,17 @@ class DecodeStep:
         with torch.cuda.graph(self.gK):
             self.gemv_only()
         torch.cuda.synchronize()
+
+    def capture_first(self, k):
+        """One graph of the first k sets' steps in order (a run whose step count is not a whole
+        number of rounds replays it once, so every timed step overlaps its neighbours)."""
+        self.gFirst = None
+        if k > 0:
+            self.gFirst = self.torch.cuda.CUDAGraph()
+            with self.torch.cuda.graph(self.gFirst):
+                for j in range(k):
+                    self.step_graph_body(j)
+            self.torch.cuda.synchronize()
 
 
 def time_loop(torch, body, steps):
@@ -738,6 +823,22 @@ def run_fl(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     peak, peak_kind = load_peaks()
+    if args.profile == "layer":
+        from variable_precision_weight_b200 import synth
+        o, i = (int(v) for v in args.shape.split(","))
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(300 + o)
+        w = fl.plane_weight(plane_layer(torch, fl, o, i, gen), o, i)
+        lv = torch.full((o // 64,), args.level, dtype=torch.uint8, device="cuda")
+        x = torch.from_numpy(synth.bf16_normal((args.batch, i), 3, args.batch).view("int16")).cuda()
+        y = torch.empty((args.batch, o), device="cuda")
+        wsb = fl.fl_gemv_workspace_bytes(o, i, args.batch)
+        ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        for k in range(3):
+            fl.fl_gemv_depth(w, lv, x, args.batch, y, ws, wsb)
+        torch.cuda.synchronize()
+        fl.fl_device_status()
+        return 0
     if args.profile == "kquant":
         items, keep, _ = kquant_step(torch, fl)
         arr = fl.kquant_problems(items)
@@ -757,25 +858,35 @@ def run_fl(args, rank, world, local_rank):
             extra_measurements(torch, fl, peak)
         return 0
 
-    # the timed steps: whole rounds of the NS sets as one graph each, the rest one step at a time
+    # the timed steps: whole rounds of the NS sets as one graph each, then one graph holding the
+    # remaining sets' steps in order: every launch overlaps its neighbours for any step count
+    rem = args.steps % NS
+    step.capture_first(rem)
+
     def body(r):
         if r < args.steps // NS:
             step.gAll.replay()
         else:
-            for k in range(args.steps - (args.steps // NS) * NS):
-                step.g[k].replay()
+            step.gFirst.replay()
 
+    clk = ClockSampler(local_rank)
+    clk.__enter__()
     for k in range(args.warmup):
         step.g[k % NS].replay()
     step.gAll.replay()
+    if step.gFirst is not None:
+        step.gFirst.replay()
     step.runs.zero_()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    n_calls = args.steps // NS + (1 if args.steps % NS else 0)
-    with ClockSampler(local_rank) as clk:
-        t = time_loop(torch, body, n_calls)
+    n_calls = args.steps // NS + (1 if rem else 0)
+    clk.mark("nvml_before_timed_region")
+    t = time_loop(torch, body, n_calls)
+    clk.mark("nvml_after_timed_region")
     t = max_over_ranks(t, world)
+    status = device_ok(fl, "the timed steps")
+    parity = step.check_outputs((args.steps - 1) % NS)
     n_esc = int(step.runs.item())                 # residual passes the device decided to run
     value = job_rate(args.steps * step.bytes_d4 + n_esc * step.bytes_res, world, t) / 1e9
     tok_s = job_rate(args.steps, world, t)
@@ -783,6 +894,8 @@ def run_fl(args, rank, world, local_rank):
     # dominant kernel alone: the step's D4 pass (gate fused), graph-replayed back to back
     reps = max(200, args.steps // 10)
     tk = time_loop(torch, lambda k: step.gK.replay(), reps) / reps
+    clk.__exit__(None, None, None)
+    device_ok(fl, "the roofline launch timing")
     achieved = step.bytes_d4 / tk / 1e9
     spread = {}
     try:  # the launch's own spread: 100 replays, each bracketed by events
@@ -794,7 +907,8 @@ def run_fl(args, rank, world, local_rank):
         torch.cuda.synchronize()
         us = np.array([e0.elapsed_time(e1) * 1e3 for e0, e1 in evs])
         spread = {"us_p10": float(np.percentile(us, 10)), "us_p50": float(np.percentile(us, 50)),
-                  "us_p90": float(np.percentile(us, 90))}
+                  "us_p90": float(np.percentile(us, 90)),
+                  "frac_p50": step.bytes_d4 / (float(np.percentile(us, 50)) * 1e-6) / 1e9 / peak}
     except Exception as e:
         spread = {"spread_error": str(e)[:200]}
 
@@ -847,6 +961,7 @@ def run_fl(args, rank, world, local_rank):
     te = time_loop(torch, lambda k: g_e2e[k % 2].replay(), e2e_rounds)
     te = max_over_ranks(te, world)
     n_esc_e = int(step.runs.item())
+    device_ok(fl, "the end-to-end steps")
     assert np.array_equal(hres.numpy(), step.gates.cpu().numpy()), "read-back differs from the device rows"
     e2e_val = job_rate(e2e_steps * step.bytes_d4 + n_esc_e * step.bytes_res, world, te) / 1e9
 
@@ -855,6 +970,7 @@ def run_fl(args, rank, world, local_rank):
         extra = {"cfg1_in_pass_share_decision": in_pass_measurement(torch, fl, step, peak),
                  "cfg1_verified_speculation_k4": spec_measurement(torch, fl, step, peak)}
         extra.update(extra_measurements(torch, fl, peak))
+        device_ok(fl, "the per-configuration measurements")
 
     if rank != 0:
         return 0
@@ -864,7 +980,7 @@ def run_fl(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u8 codes x s8 activation digits -> s32 (15-bit per-group fixed-point x), fp32 scales/accumulate",
+        "dtype": "u8 codes x s8 activation digits -> s32 (31-bit per-group fixed-point x), fp32 scales/accumulate",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": 1, "weight_bytes_per_step_d4": step.bytes_d4,
                    "weight_bytes_per_escalation": step.bytes_res, "escalated_steps": n_esc,
@@ -878,6 +994,10 @@ def run_fl(args, rank, world, local_rank):
                      "traffic": tr["bytes_per_launch"] if tr else None,
                      "kernel": "plane_gemv_kernel (fl_gemv_batched_gate, 197 problems, D4, logit gate fused)",
                      "us_per_launch": tk * 1e6, "bytes_per_launch": step.bytes_d4, **spread,
+                     "frac_statistic": "achieved and frac use us_per_launch, the mean over back-to-back "
+                                       "graph replays of the launch; frac_p50 uses the median of 100 "
+                                       "replays each bracketed by its own events (graph-launch overhead "
+                                       "included)",
                      "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,
                      # plane GEMV launches per step (the D4 pass plus the escalated steps' residual
                      # pass, both full reads of the store) x time per launch / step time
@@ -887,6 +1007,9 @@ def run_fl(args, rank, world, local_rank):
                 "d2h_bytes_per_step": 32, "steps": e2e_steps,
                 "tokens_per_s": job_rate(e2e_steps, world, te)},
         "gpu_launches": 2 * args.steps,  # D4 pass + conditional residual pass (returns at once when not needed)
+        "device_status": status,
+        "parity_sample": parity,
+        "timed_graphs": f"{args.steps // NS} x {NS}-step graph + 1 x {rem}-step graph",
         "clocks": clk.summary(),
         "kernels": extra,
     }

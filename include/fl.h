@@ -34,7 +34,8 @@
  *   - fl_last_error() returns a message describing the most recent failure
  *     on the calling thread.
  *   - bf16 activations are passed as their 16-bit patterns (uint16_t).
- *   - Batch (tokens per call) is 1..16; activations are row-major
+ *   - Batch (tokens per call) is 1..16 (1..32 for fl_gemv_depth and
+ *     fl_gemv_residual); activations are row-major
  *     [batch][in], outputs row-major [batch][out] fp32.
  */
 #ifndef FL_H_
@@ -65,6 +66,9 @@ typedef enum {
 } fl_status;
 
 #define FL_MAX_BATCH 16
+/* Single-layer depth / residual calls (fl_gemv_depth, fl_gemv_residual) take batches up to
+ * this; from batch 9 they run on the fifth-generation tensor cores (tcgen05, TMEM). */
+#define FL_MAX_GEMV_BATCH 32
 #define FL_MAX_STOPS 16
 #define FL_MAX_PROBLEMS 256
 
@@ -177,7 +181,9 @@ FL_API fl_status fl_level_map(const float* xy, int nblocks, const float* centers
 /*                                                                           */
 /* levels   device, uint8 [out / 64], values 0..4 (0 ZERO .. 4 D8); values   */
 /*          above 4 are read as 4.                                           */
-/* x        device, bf16 [batch][in], 16-byte aligned; batch 1..16           */
+/* x        device, bf16 [batch][in], 16-byte aligned; batch 1..32 (batch 9  */
+/*          and up run on the tcgen05 tensor cores: u8 codes in TMEM, digits  */
+/*          in shared memory, int32 accumulators in TMEM)                     */
 /* y        device, fp32 [batch][out], 4-byte aligned; overwritten           */
 /* workspace device scratch for splitting a layer's columns across CTAs:     */
 /*          at least fl_gemv_workspace_bytes(out, in, batch) bytes, 16-byte  */
@@ -198,10 +204,13 @@ FL_API fl_status fl_gemv_depth(const fl_plane_weight* w, const uint8_t* levels, 
  * decode loop). The column-split scratch lives in a fixed array of
  * FL_GEMV_STATIC_SCRATCH_BYTES inside the library's device image, so this
  * call allocates nothing.
- *   - Same arguments and arithmetic as fl_gemv_depth, minus the workspace.
- *   - Shapes whose split needs more scratch than the array holds
- *     (fl_gemv_workspace_bytes(out, in, batch) > FL_GEMV_STATIC_SCRATCH_BYTES)
- *     return FL_ERR_WORKSPACE; use fl_gemv_depth for them.
+ *   - Same arguments and arithmetic as fl_gemv_depth, minus the workspace;
+ *     batch 1..16, always on the int8 mma.sync kernel (fl_gemv_depth moves
+ *     batches 9 and up to the tcgen05 kernel, whose split is sized apart).
+ *   - Shapes whose split needs more scratch than the array holds return
+ *     FL_ERR_WORKSPACE (for batch 1..8 that is when
+ *     fl_gemv_workspace_bytes(out, in, batch) > FL_GEMV_STATIC_SCRATCH_BYTES);
+ *     use fl_gemv_depth for them.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *     The address is kept for the life of the process, per device ordinal: it

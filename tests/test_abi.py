@@ -68,7 +68,8 @@ def test_host_side_rejections(fl):
     assert _status(fl, fl.fl_gemv_depth, w, 16, 16, 1, 16, None, 0, s0) == ERR_ARG
     w = fl.plane_weight(16, 64, 128)
     assert _status(fl, fl.fl_gemv_depth, w, 16, 16, 0, 16, None, 0, s0) == ERR_SHAPE       # batch 0
-    assert _status(fl, fl.fl_gemv_depth, w, 16, 16, 17, 16, None, 0, s0) == ERR_SHAPE      # batch 17
+    assert _status(fl, fl.fl_gemv_depth, w, 16, 16, 33, 16, None, 0, s0) == ERR_SHAPE      # batch 33
+    assert _status(fl, fl.fl_gemv_depth_static, w, 16, 16, 17, 16, s0) == ERR_SHAPE       # batch 17 (no tcgen05)
     assert _status(fl, fl.fl_gemv_residual, w, 16, None, 16, 1, 16, None, 0, s0) == ERR_ARG
     assert _status(fl, fl.fl_gemv_kquant, 16, 13, 64, 256, 16, 1, 16, None, 0, s0) == ERR_UNSUP   # Q5_K
     assert _status(fl, fl.fl_gemv_kquant, 16, 10, 64, 256, 16, 1, 16, None, 0, s0) == ERR_UNSUP   # Q2_K
@@ -85,6 +86,7 @@ def test_host_side_rejections(fl):
     probs = fl.gemv_problems([(16, 64, 128, 16, None, 16, 16)])
     assert _status(fl, fl.fl_gemv_batched, probs, 0, 1, 0, s0) == ERR_ARG
     assert _status(fl, fl.fl_gemv_batched, probs, 1, 1, 2, s0) == ERR_ARG                  # mode
+    assert _status(fl, fl.fl_gemv_batched, probs, 1, 17, 0, s0) == ERR_SHAPE               # batch 17
     gsz = fl.fl_gemv_gate_workspace_bytes(1)
     assert gsz > 0 and fl.fl_gemv_gate_workspace_bytes(0) == 0
     spec = fl.gate_spec(1, 0.0, 0.0, 16, 16, 16, 16, 16, gsz)                  # problem 1 of 1

@@ -99,7 +99,7 @@ def test_decode_step_batched_pass_full_size(env, orc):
         assert int(es.item()) == 1
 
 
-@pytest.mark.parametrize("batch", [1, 16])
+@pytest.mark.parametrize("batch", [1, 8, 16, 32])
 def test_large_single_layers_full_size(env, orc, batch):
     """The large-shape sweep at full size (uniform D6), single-layer calls with column splits."""
     torch, fl = env

@@ -95,6 +95,14 @@ CASES = [
     (256, 14336, 16, "uniform"),
     (2048, 1024, 1, "d4"),
     (640, 3072, 2, "zero_heavy"),
+    # batch 9 and up: the tcgen05 tensor-core path (block pairs, digits in shared memory)
+    (448, 1664, 9, "uniform"),        # 7 blocks: the last pair holds one block
+    (448, 1664, 17, "uniform"),
+    (320, 2048, 24, "uniform"),
+    (2048, 1024, 32, "d4"),
+    (640, 3072, 20, "zero_heavy"),
+    (64, 4096, 32, "uniform"),        # one block, column slices
+    (256, 14336, 32, "uniform"),      # few blocks, wide rows: many column slices + tickets
 ]
 
 
@@ -175,7 +183,7 @@ def outlier_x(batch, inn, k, *key, big=256.0):
 # weight that reconstructs to exactly 0 (a D8 code 0), so it adds nothing to sum |w||x| and
 # the bar is set by the small elements alone, 2^k below it.
 @pytest.mark.parametrize("k", [10, 14, 20])
-@pytest.mark.parametrize("batch", [1, 3, 8])
+@pytest.mark.parametrize("batch", [1, 3, 8, 16, 32])
 def test_gemv_outlier_on_a_zero_weight(env, orc, k, batch):
     torch, fl = env
     out, inn = 192, 1664
@@ -269,6 +277,56 @@ def test_residual_vs_oracle_and_identity(env, orc):
     y48, _ = gemv_gpu(torch, fl, store, out, inn, d4, x, mode=1, to_levels=d8, y0=y4)
     y8ref, mass8 = orc.gemv_depth(q, s, d8, x, with_mass=True)
     check_close(y48, y8ref, mass8, "D4+res")
+
+
+@pytest.mark.parametrize("batch", [9, 16, 32])
+def test_residual_tensor_core_path(env, orc, batch):
+    """Residual from every level pair on the tcgen05 path, column slices included, and
+    D4 + residual(D4 -> D8) = D8 there."""
+    torch, fl = env
+    out, inn = 448, 4096
+    q, s = synth.int8_layer(out, inn, 38, batch)
+    a = synth.seeded_levels(out // 64, 39, batch)
+    b = np.maximum(a, synth.seeded_levels(out // 64, 40, batch))
+    b[0], a[0] = 2, 3                                  # a non-raising block adds nothing
+    x = synth.bf16_normal((batch, inn), 41, batch)
+    store = pack_gpu(torch, fl, q, s)
+    y0 = synth.rng(42, batch).standard_normal((batch, out)).astype(np.float32)
+    y, _ = gemv_gpu(torch, fl, store, out, inn, a, x, mode=1, to_levels=b, y0=y0)
+    dref, mass = orc.gemv_residual(q, s, a, b, x, with_mass=True)
+    check_close(y, y0.astype(np.float64) + dref, mass, f"tc residual b{batch}")
+    assert np.array_equal(y[:, :64], y0[:, :64])
+    d4 = np.full(out // 64, 2, np.uint8)
+    d8 = np.full(out // 64, 4, np.uint8)
+    y4, _ = gemv_gpu(torch, fl, store, out, inn, d4, x)
+    y48, _ = gemv_gpu(torch, fl, store, out, inn, d4, x, mode=1, to_levels=d8, y0=y4)
+    y8ref, mass8 = orc.gemv_depth(q, s, d8, x, with_mass=True)
+    check_close(y48, y8ref, mass8, f"tc D4+res b{batch}")
+
+
+def test_tensor_core_path_repeated_calls_leave_workspace_zero(env, orc):
+    torch, fl = env
+    out, inn, batch = 192, 14336, 24
+    q, s = synth.int8_layer(out, inn, 43)
+    lv = synth.seeded_levels(out // 64, 44)
+    x = synth.bf16_normal((batch, inn), 45)
+    store = pack_gpu(torch, fl, q, s)
+    wsb = fl.fl_gemv_workspace_bytes(out, inn, batch)
+    assert wsb > 0
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    y = torch.empty((batch, out), dtype=torch.float32, device="cuda")
+    w = fl.plane_weight(store, out, inn)
+    yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+    for _ in range(3):
+        fl.fl_gemv_depth(w, dev(torch, lv), dev(torch, x), batch, y, ws, wsb)
+        torch.cuda.synchronize()
+        check_close(y.cpu().numpy(), yref, mass, "tc repeat")
+    npair = (out // 64 + 1) // 2
+    assert int(ws[:4 * npair].count_nonzero().item()) == 0
+    fl.fl_device_status()
+    with pytest.raises(fl.FlError) as e:
+        fl.fl_gemv_depth(w, dev(torch, lv), dev(torch, x), batch, y, ws, wsb - 16)
+    assert e.value.status == -6
 
 
 def test_residual_split_columns(env, orc):

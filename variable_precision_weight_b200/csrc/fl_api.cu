@@ -72,6 +72,9 @@ int take_device_error();
 namespace kq {
 int take_device_error();
 }
+namespace tc {
+int take_device_error();
+}
 int take_gate_error();
 }  // namespace fl
 
@@ -79,8 +82,9 @@ extern "C" fl_status fl_device_status(void) {
   using namespace fl;
   FL_CHECK_CUDA(cudaDeviceSynchronize(), "fl_device_status: cudaDeviceSynchronize");
   const int g = gemv::take_device_error(), k = kq::take_device_error(), t = take_gate_error();
-  if (g < 0 || k < 0 || t < 0) return fail(FL_ERR_CUDA, "fl_device_status: reading the error words failed");
-  if (g == 0 && k == 0 && t == 0) return FL_OK;
+  const int c = tc::take_device_error();
+  if (g < 0 || k < 0 || t < 0 || c < 0) return fail(FL_ERR_CUDA, "fl_device_status: reading the error words failed");
+  if (g == 0 && k == 0 && t == 0 && c == 0) return FL_OK;
   auto what = [](int c) {
     return c == 1 ? "a producer's wait for a free stage" : c == 2 ? "a consumer's wait for a full stage"
          : c == 3 ? "the wait for staged activations" : c == 4 ? "the self-test wait" : "a wait";
@@ -89,5 +93,10 @@ extern "C" fl_status fl_device_status(void) {
     return fail(FL_ERR_ARG, "plane GEMV: a listed block index was out of range; that unit was skipped");
   if (g) return fail(FL_ERR_TIMEOUT, "plane GEMV: %s ran out (code %d); its outputs are not valid", what(g), g);
   if (k) return fail(FL_ERR_TIMEOUT, "K-quant GEMV: %s ran out (code %d); its outputs are not valid", what(k), k);
+  if (c) {
+    const char* cw = c == 1 ? "the producer's wait for a free stage" : c == 2 ? "the MMA issuer's wait for codes or a free accumulator"
+                   : c == 3 ? "a converter's wait for a full stage or a free code buffer" : "an epilogue wait for the MMAs";
+    return fail(FL_ERR_TIMEOUT, "tensor-core GEMV: %s ran out (code %d); its outputs are not valid", cw, c);
+  }
   return fail(FL_ERR_TIMEOUT, "logit gate: the wait for the cluster's partials ran out; its outputs are NaN");
 }

@@ -97,23 +97,41 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // room for the context being time-sliced with another process's work.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
-// Wait on an mbarrier phase, bounded in time: each try_wait may suspend the thread for a
-// hardware-chosen interval, so the bound is a deadline on the global timer (read every 64
-// failed polls, counted from the first), not a poll count. Returns false (the caller records
-// the failure) if the phase has not completed by then.
+// One poll of an mbarrier phase. With a suspend-time hint the thread sleeps until the phase
+// completes or the hint elapses, instead of returning at once: a waiting warp then takes no
+// issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok)
+               : "r"(a), "r"(parity)
+               : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t a, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(a), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendNs = 20000;  // longest single sleep of a waiting thread
+
+// Wait on an mbarrier phase, bounded in time. One plain poll first (the common case in a
+// running pipeline); then the thread sleeps in suspend-hinted polls, each ending when the phase
+// completes, and the deadline on the global timer is checked between them. Returns false (the
+// caller records the failure) if the phase has not completed by then.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
-  uint64_t t0 = 0;
-  for (uint32_t k = 1;; ++k) {
-    uint32_t ok;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if (k == 1) t0 = globaltimer_ns();
-    if ((k & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
+  if (mbar_try(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_sleep(a, parity, kSuspendNs)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

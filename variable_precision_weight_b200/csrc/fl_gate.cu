@@ -110,8 +110,13 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
           : "memory");
       ok = done != 0;
       if (ok) break;
-      if (k == 1) t0 = globaltimer_ns();
-      if ((k & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if ((k & 1023u) == 0u) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0)
+          t0 = now;
+        else if (now - t0 > kWaitLimitNs)
+          break;
+      }
     }
     if (!ok) atomicExch(&g_gate_error, 1);
   }

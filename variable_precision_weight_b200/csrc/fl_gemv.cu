@@ -42,6 +42,14 @@
 #include "fl_gate_merge.cuh"
 
 namespace fl {
+
+// The tensor-core (tcgen05) path of fl_gemv_tc.cu: single-layer calls at batches from 9 up to
+// FL_MAX_GEMV_BATCH.
+bool tc_takes(int batch);
+size_t tc_workspace_bytes(int out, int in, int batch);
+fl_status tc_single(const fl_plane_weight* w, const uint8_t* lv_from, const uint8_t* lv_to, const uint16_t* x,
+                    int batch, float* y, void* ws, size_t ws_bytes, void* stream, int mode, const char* what);
+
 namespace gemv {
 
 constexpr int kTeams = 4;
@@ -1134,7 +1142,9 @@ static fl_status prepare_single(Args<1>& a, const fl_plane_weight* w, const uint
   if (st != FL_OK) return st;
   if (!lv_from || !x || !y || (mode == 1 && !lv_to)) return fail(FL_ERR_ARG, "%s: NULL pointer argument", what);
   if (reinterpret_cast<uintptr_t>(y) & 3u) return fail(FL_ERR_ALIGN, "%s: y not 4-byte aligned", what);
-  if (batch < 1 || batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..16)", what, batch);
+  if (batch < 1 || batch > FL_MAX_GEMV_BATCH)
+    return fail(FL_ERR_SHAPE, "%s: batch=%d (1..%d)", what, batch, FL_MAX_GEMV_BATCH);
+  if (batch > FL_MAX_BATCH) return fail(FL_ERR_SHAPE, "%s: batch=%d (1..%d on this path)", what, batch, FL_MAX_BATCH);
   if (!aligned16(x)) return fail(FL_ERR_ALIGN, "%s: x not 16-byte aligned", what);
   const int nsm = device_sm_count();
   if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
@@ -1180,6 +1190,14 @@ static fl_status prepare_single(Args<1>& a, const fl_plane_weight* w, const uint
 static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const uint8_t* lv_to, const uint16_t* x,
                         int batch, float* y, void* ws, size_t ws_bytes, void* stream, int mode,
                         const char* what) {
+  if (batch >= 1 && batch <= FL_MAX_GEMV_BATCH && tc_takes(batch)) {
+    fl_status st = check_weight(w, what);
+    if (st != FL_OK) return st;
+    if (!lv_from || !x || !y || (mode == 1 && !lv_to)) return fail(FL_ERR_ARG, "%s: NULL pointer argument", what);
+    if (reinterpret_cast<uintptr_t>(y) & 3u) return fail(FL_ERR_ALIGN, "%s: y not 4-byte aligned", what);
+    if (!aligned16(x)) return fail(FL_ERR_ALIGN, "%s: x not 16-byte aligned", what);
+    return tc_single(w, lv_from, lv_to, x, batch, y, ws, ws_bytes, stream, mode, what);
+  }
   static thread_local Args<1> a;
   const fl_status st = prepare_single(a, w, lv_from, lv_to, x, batch, y, ws, ws_bytes, mode, what);
   if (st != FL_OK) return st;
@@ -1192,7 +1210,8 @@ static fl_status single(const fl_plane_weight* w, const uint8_t* lv_from, const 
 using namespace fl;
 
 extern "C" size_t fl_gemv_workspace_bytes(int out, int in, int batch) {
-  if (out <= 0 || in <= 0 || out % 64 || in % 128 || batch < 1 || batch > FL_MAX_BATCH) return 0;
+  if (out <= 0 || in <= 0 || out % 64 || in % 128 || batch < 1 || batch > FL_MAX_GEMV_BATCH) return 0;
+  if (tc_takes(batch)) return tc_workspace_bytes(out, in, batch);
   const int nsm = device_sm_count();
   if (nsm <= 0) return 0;
   gemv::Plan pl = gemv::plan_single(out / 64, in / 128, batch, nsm);

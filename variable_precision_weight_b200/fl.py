@@ -21,6 +21,7 @@ _lib = C.CDLL(LIB_PATH)
 
 FL_OK = 0
 FL_MAX_BATCH = 16
+FL_MAX_GEMV_BATCH = 32
 FL_MAX_STOPS = 16
 FL_MAX_PROBLEMS = 256
 FL_GGML_Q4_K = 12

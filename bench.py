@@ -678,7 +678,7 @@ def extra_measurements(torch, fl, peak):
         gen.manual_seed(300 + o)
         stores = [plane_layer(torch, fl, o, i, gen) for _ in range(ncp)]
         lv6 = torch.full((o // 64,), 3, dtype=torch.uint8, device="cuda")
-        for batch in (1, 4, 8, 16):
+        for batch in (1, 4, 8, 16, 32):
             x = torch.from_numpy(synth.bf16_normal((batch, i), 3, batch).view("int16")).cuda()
             y = torch.empty((batch, o), device="cuda")
             wsb = fl.fl_gemv_workspace_bytes(o, i, batch)

@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", choices=["fl", "reference"], default="fl")
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config kernel measurements")
+    ap.add_argument("--shard", action="store_true",
+                    help="split every layer's blocks over the ranks (strong scaling) instead of one replica per GPU")
     ap.add_argument("--profile", choices=["none", "step", "kquant", "kernels", "layer"], default="none",
                     help="short run for an ncu capture: 'step' = the decode step only, 'kquant' = the K-quant "
                          "step only, 'kernels' = one pass of every per-config kernel measurement, 'layer' = "
@@ -1017,6 +1019,150 @@ def run_fl(args, rank, world, local_rank):
     return 0
 
 
+def run_shard(args, rank, world, local_rank):
+    """The decode step with the read split over the ranks (strong scaling: the step's total work is
+    fixed; each rank reads its byte-balanced share of every layer's blocks, x replicated). Per step:
+    one batched D4 pass over the rank's block ranges; the gate partial of the rank's share of the
+    head's logits (the vocabulary is split with the head's blocks); one all-gather of the partials
+    and the merge on the device, identical on every rank; the D4->D8 residual pass over the rank's
+    ranges, run or skipped on the device by the merged escalate flag; the gate gathered and merged
+    again; one all-gather of the output rows. Device time with CUDA events, max over ranks."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from variable_precision_weight_b200 import fl, shard, synth
+
+    torch.cuda.set_device(local_rank)
+    if not dist.is_initialized():   # one rank launched without torchrun
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29531")
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=120))
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(2000)                       # every rank builds the same model
+    shapes = synth.qwen3_step_shapes()
+    layers, lv_host, to8 = [], [], []
+    for _, o, i in shapes:
+        layers.append((plane_layer(torch, fl, o, i, gen), o, i,
+                       torch.full((o // 64,), 2, dtype=torch.uint8, device="cuda")))
+        lv_host.append(np.full(o // 64, 2, np.uint8))
+        to8.append(torch.full((o // 64,), 4, dtype=torch.uint8, device="cuda"))
+    plans = shard.plan(lv_host, [i for _, _, i in shapes], world)
+    rows, total = shard.rank_rows(plans, rank)
+    counts = [shard.rank_rows(plans, r)[1] for r in range(world)]
+    NS, NESC = 8, 2
+    tot_in = sum(i for _, _, i in shapes)
+    xs = torch.empty((NS, tot_in), dtype=torch.int16, device="cuda")
+    for j in range(NS):
+        xs[j].copy_(torch.from_numpy(synth.bf16_normal((tot_in,), 3000, j).view("int16")))
+    # as wide as the largest rank's rows, so the row exchange sends it with no copy
+    y_local = torch.zeros(max(counts), dtype=torch.float32, device="cuda")
+    y_all = torch.zeros(world * max(counts), dtype=torch.float32, device="cuda")
+    p_all = torch.zeros(world * fl.GATE_PARTIAL_BYTES, dtype=torch.uint8, device="cuda")
+    prob_d4, prob_r = [], []
+    for j in range(NS):
+        lay, oi = [], 0
+        for st, o, i, lv in layers:
+            lay.append((st, o, i, lv, xs[j, oi:oi + i]))
+            oi += i
+        it4, placed = shard.local_items(lay, plans, rank, y_local)
+        itr, _ = shard.local_items(lay, plans, rank, y_local, 1, to8)
+        prob_d4.append(fl.gemv_problems(it4))
+        prob_r.append(fl.gemv_problems(itr))
+    n_items = len(placed)
+    head = len(shapes) - 1
+    h_idx, h_off, h_rows = next(((k, off, n) for k, (li, off, n) in enumerate(placed) if li == head), (0, 0, 0))
+    h_first = 64 * plans[head][rank]
+    assert h_rows > 0 and n_items == len(shapes), "every rank holds blocks of every layer at these shapes"
+    part = torch.zeros(fl.GATE_PARTIAL_BYTES, dtype=torch.uint8, device="cuda")
+    gates = torch.zeros(8, dtype=torch.int32, device="cuda")
+    esc = gates[4:5].view(torch.uint8)[0:1]
+    runs = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # the conditional residual launch carries a fused gate over the rank's own head rows; its
+    # outputs go to scratch (the step's gate is the merged one)
+    gsz = fl.fl_gemv_gate_workspace_bytes(1)
+    gws = torch.zeros(gsz, dtype=torch.uint8, device="cuda")
+    scratch = torch.zeros(8, dtype=torch.int32, device="cuda")
+    spec_local = fl.gate_spec(h_idx, 1e30, -1.0, scratch[0:1].view(torch.float32), scratch[1:2].view(torch.float32),
+                              scratch[2:4], scratch[4:5].view(torch.uint8)[0:1], gws, gsz)
+    tau = [1e30, -1.0]
+
+    def gate():
+        fl.fl_logit_gate_partial(y_local[h_off:h_off + h_rows], h_rows, 1, h_first, part)
+        allp = shard.gather_partials(part, world, out=p_all)
+        fl.fl_logit_gate_merge(allp, world, 1, tau[0], tau[1], gates[0:1].view(torch.float32),
+                               gates[1:2].view(torch.float32), gates[2:4], esc)
+
+    def d4(j):
+        fl.fl_gemv_batched(prob_d4[j], n_items, 1, 0)
+        gate()
+
+    def step(j):
+        d4(j)
+        fl.fl_gemv_batched_gate_if(prob_r[j], n_items, 1, 1, spec_local, esc, runs)
+        gate()
+        shard.gather_rows(y_local, counts, out=y_all)
+
+    # entropy threshold from the merged D4 gate so NESC of the NS input sets escalate
+    H = []
+    for j in range(NS):
+        d4(j)
+        H.append(float(gates[0:1].view(torch.float32).item()))
+    h = sorted(H, reverse=True)
+    tau[0] = 0.5 * (h[NESC - 1] + h[NESC])
+    # one CUDA graph per input set (NCCL's collectives captured with the kernels), after one
+    # eager pass of each so every communicator is set up before capture
+    for j in range(NS):
+        step(j)
+    torch.cuda.synchronize()
+    graphs = []
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        for j in range(NS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                step(j)
+            graphs.append(g)
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    clk = ClockSampler(local_rank)
+    try:
+        with clk:
+            for k in range(args.warmup):
+                graphs[k % NS].replay()
+            runs.zero_()
+            dist.barrier()
+            torch.cuda.synchronize()
+            clk.mark("before_timed")
+            t = time_loop(torch, lambda k: graphs[k % NS].replay(), args.steps)
+            clk.mark("after_timed")
+        t = max_over_ranks(t, world)
+    finally:
+        torch.cuda.synchronize()
+        del graphs      # graphs holding NCCL calls go before the process group does
+    device_ok(fl, "the sharded steps")
+    n_esc = int(runs.item())
+    bytes_d4 = sum((o // 64) * plane_bytes(i, 2) for _, o, i in shapes)
+    bytes_res = sum((o // 64) * (256 * (i // 128) + 2048 * (i // 128) * 2) for _, o, i in shapes)
+    if rank != 0:
+        return 0
+    # every rank takes the same gate decision, so rank 0's count of residual passes is the job's
+    value = (args.steps * bytes_d4 + n_esc * bytes_res) / t / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": "u8 codes x s8 activation digits -> s32 (31-bit per-group fixed-point x), fp32 scales/accumulate",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch": 1,
+                       "parallelism": f"every layer's 64-row blocks split over {world} ranks by the bytes read",
+                       "rows_per_rank": counts, "escalated_steps": n_esc, "input_sets": NS,
+                       "l2": "weights (0.33 GB at D4) larger than L2; input sets rotate"},
+            "tokens_per_s": args.steps / t, "clocks": clk.summary(),
+            "gpu_launches": 6 * args.steps}   # D4 pass, residual pass, 2 x (partial + merge); NCCL's not counted
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -1030,10 +1176,12 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
+        if args.shard:
+            return run_shard(args, rank, world, local_rank)
         return run_fl(args, rank, world, local_rank)
     finally:
-        if world > 1:
-            import torch.distributed as dist
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
             dist.destroy_process_group()
 
 

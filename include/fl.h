@@ -373,6 +373,53 @@ FL_API fl_status fl_logit_gate(const float* logits, int vocab, int batch, float 
                         float* margin, int32_t* top2, uint8_t* escalate, void* stream);
 
 /* ========================================================================= */
+/* The read split over devices. Blocks are independent, so ranks can each    */
+/* read a contiguous range of every layer's 64-row blocks (the same          */
+/* fl_gemv_* calls on the range: plane store + first * 8448 * (in / 128),    */
+/* out = 64 * count, levels + first) and exchange their outputs; the gate    */
+/* then needs the whole row of logits, which the ranks hold in pieces, so   */
+/* each rank reduces its piece to a partial and every rank merges all the   */
+/* partials the same way ([PoD] abstract: the gate reads the low-precision  */
+/* output distribution; [FoQLens] progress table: each block read to its    */
+/* own depth).                                                               */
+/* ========================================================================= */
+
+/* Contiguous block ranges for nranks ranks, balanced by the bytes each block's depth reads
+ * (256 G + 2048 G d / 2 at depth d, G = in / 128; ZERO blocks read nothing): rank r reads
+ * blocks [first_block[r], first_block[r + 1]), first_block[0] = 0, first_block[nranks] =
+ * nblocks; a block goes to the range that holds the midpoint of its bytes, so ranges differ
+ * by at most one block's bytes. Ranges may be empty (nranks > nblocks). A layer that reads
+ * nothing is split by block count. Host only: levels is a HOST array of nblocks level bytes
+ * (values above 4 read as 4), first_block a HOST array of nranks + 1 ints. */
+FL_API fl_status fl_shard_blocks(const uint8_t* levels, int nblocks, int in, int nranks, int* first_block);
+
+/* A rank's partial of the gate over its piece of the logits: per row, m = max z,
+ * s = sum e^(z - m), t = sum (z - m) e^(z - m), the largest and second largest value (v2)
+ * with their GLOBAL indices i1, i2 (piece index + index_base; ties to the lower index).
+ * 32 bytes, the same record the fused gate merges. */
+typedef struct {
+  float m, s, t, v2;
+  int32_t i1, i2, pad0, pad1;
+} fl_gate_partial;
+
+/* logits  device fp32 [batch][vocab] (this rank's piece of each row), 16-byte aligned,
+ *         vocab % 4 == 0; index_base + vocab <= 2^24
+ * partial device fl_gate_partial [batch], 16-byte aligned, written. One launch: a cluster of
+ *         8 or 16 CTAs per row, the reduction fl_logit_gate runs. If the cluster's wait for its
+ *         CTAs' partials runs out (1 s) the record's s is NaN, so the merged entropy and margin
+ *         are NaN, and fl_device_status reports the wait. */
+FL_API fl_status fl_logit_gate_partial(const float* logits, int vocab, int batch, int index_base,
+                                       fl_gate_partial* partial, void* stream);
+
+/* Merge nparts partials per row, partials laid out [nparts][batch] (the gathered pieces in
+ * rank order), in that order, and write entropy / margin / top2 / escalate exactly as
+ * fl_logit_gate defines them for the whole row (equal up to fp32 summation order). Every rank
+ * that merges the same partials computes the same outputs. Output pointers as fl_logit_gate;
+ * partials device, 16-byte aligned; 1 <= nparts <= 4096. One launch. */
+FL_API fl_status fl_logit_gate_merge(const fl_gate_partial* partials, int nparts, int batch, float tau_h, float tau_m,
+                                     float* entropy, float* margin, int32_t* top2, uint8_t* escalate, void* stream);
+
+/* ========================================================================= */
 /* Verified speculation ([PoD] abstract: a low-precision draft verified at   */
 /* 8 bits gives the 8-bit model's output at a comparable weight-byte cost).  */
 /* Greedy, over a window of k steps (1 <= k <= FL_MAX_BATCH):                */

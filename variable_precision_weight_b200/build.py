@@ -24,7 +24,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libfl.so")
 SOURCES = ["fl_api.cu", "fl_pack.cu", "fl_lens.cu", "fl_gemv.cu", "fl_gemv_tc.cu", "fl_gate.cu", "fl_kquant.cu",
-           "fl_decide.cu", "fl_spec.cu"]
+           "fl_decide.cu", "fl_spec.cu", "fl_shard.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

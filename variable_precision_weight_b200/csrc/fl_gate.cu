@@ -16,6 +16,10 @@
 // across the cluster: every CTA stores its partial into CTA rank 0's shared memory and
 // arrives on an mbarrier there, and rank 0 merges and writes the row's outputs. Merge orders
 // are fixed (deterministic); one launch, no global scratch.
+//
+// The same kernel gives the partial of a row piece when the vocabulary is split over devices:
+// indices are offset by the piece's first global index and rank 0 stores the merged record
+// (max, S, T, top-2) instead of the row's outputs.
 #include "fl_gate_merge.cuh"
 
 namespace fl {
@@ -28,11 +32,12 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-template <int C, int T, int CACHE>
+template <int C, int T, int CACHE, bool PARTIAL>
 __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__ logits, int vocab, float tau_h,
                                                        float tau_m, float* __restrict__ entropy,
                                                        float* __restrict__ margin, int32_t* __restrict__ top2,
-                                                       uint8_t* __restrict__ escalate) {
+                                                       uint8_t* __restrict__ escalate, int index_base,
+                                                       GateRec* __restrict__ partial) {
   __shared__ GateRec s_warp[T / 32];
   __shared__ GateRec s_cta[C];          // used in rank 0: one slot per CTA of the cluster
   __shared__ __align__(8) uint64_t s_bar;  // rank 0: the other CTAs' partials have arrived
@@ -62,7 +67,7 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
 #pragma unroll
     for (int k = 0; k < CACHE; ++k) {
       const int q = base + (int)threadIdx.x + k * T;
-      idx[k] = 4 * q;
+      idx[k] = index_base + 4 * q;
       if (q < q1) {
         v[k] = __ldg(z4 + q);
         nv = k + 1;
@@ -123,8 +128,13 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
   __syncwarp();
   r = warp_merge(lane < C ? s_cta[lane] : empty_rec());
   if (lane == 0) {
-    gate_outputs(r, tau_h, tau_m, entropy + row, margin + row, top2 + 2 * row, escalate + row);
-    if (!ok) entropy[row] = margin[row] = NAN;
+    if constexpr (PARTIAL) {
+      if (!ok) r.S = NAN;  // the merged gate's entropy and margin come out NaN
+      partial[row] = r;
+    } else {
+      gate_outputs(r, tau_h, tau_m, entropy + row, margin + row, top2 + 2 * row, escalate + row);
+      if (!ok) entropy[row] = margin[row] = NAN;
+    }
   }
 }
 
@@ -132,18 +142,19 @@ __global__ void __launch_bounds__(T) logit_gate_kernel(const float* __restrict__
 
 namespace fl {
 
-template <int C, int T, int CACHE>
+template <int C, int T, int CACHE, bool PARTIAL>
 static cudaError_t gate_launch_c(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,
-                                 float* margin, int32_t* top2, uint8_t* escalate, cudaStream_t st) {
-  return launch_pdl(logit_gate_kernel<C, T, CACHE>, dim3((unsigned)(batch * C)), dim3(T), 0, st, C, logits, vocab,
-                    tau_h, tau_m, entropy, margin, top2, escalate);
+                                 float* margin, int32_t* top2, uint8_t* escalate, int index_base, GateRec* partial,
+                                 cudaStream_t st) {
+  return launch_pdl(logit_gate_kernel<C, T, CACHE, PARTIAL>, dim3((unsigned)(batch * C)), dim3(T), 0, st, C, logits,
+                    vocab, tau_h, tau_m, entropy, margin, top2, escalate, index_base, partial);
 }
 
 // 16-CTA clusters where the device can place one (decided once per process), else 8.
 static bool gate_wide_clusters() {
   static int wide = -1;
   if (wide < 0) {
-    auto kern = logit_gate_kernel<16, 256, 10>;
+    auto kern = logit_gate_kernel<16, 256, 10, false>;
     int n = 0;
     bool ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
     if (ok) {
@@ -168,8 +179,26 @@ static bool gate_wide_clusters() {
 static cudaError_t gate_launch(const float* logits, int vocab, int batch, float tau_h, float tau_m, float* entropy,
                                float* margin, int32_t* top2, uint8_t* escalate, cudaStream_t st) {
   if (gate_wide_clusters())
-    return gate_launch_c<16, 256, 10>(logits, vocab, batch, tau_h, tau_m, entropy, margin, top2, escalate, st);
-  return gate_launch_c<8, 512, 10>(logits, vocab, batch, tau_h, tau_m, entropy, margin, top2, escalate, st);
+    return gate_launch_c<16, 256, 10, false>(logits, vocab, batch, tau_h, tau_m, entropy, margin, top2, escalate, 0,
+                                             nullptr, st);
+  return gate_launch_c<8, 512, 10, false>(logits, vocab, batch, tau_h, tau_m, entropy, margin, top2, escalate, 0,
+                                          nullptr, st);
+}
+
+// The partial records of the rows' pieces (indices offset by index_base), one cluster per row.
+cudaError_t gate_partial_launch(const float* logits, int vocab, int batch, int index_base, GateRec* partial,
+                                cudaStream_t st) {
+  if (gate_wide_clusters()) {
+    static bool attr = false;
+    if (!attr) {
+      cudaFuncSetAttribute(logit_gate_kernel<16, 256, 10, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      attr = true;
+    }
+    return gate_launch_c<16, 256, 10, true>(logits, vocab, batch, 0.f, 0.f, nullptr, nullptr, nullptr, nullptr,
+                                            index_base, partial, st);
+  }
+  return gate_launch_c<8, 512, 10, true>(logits, vocab, batch, 0.f, 0.f, nullptr, nullptr, nullptr, nullptr,
+                                         index_base, partial, st);
 }
 
 }  // namespace fl

@@ -101,6 +101,9 @@ _sigs = {
     "fl_gemv_kquant_batched": (_I, [C.POINTER(fl_kquant_problem), _I, _I, _P]),
     "fl_level_decide": (_I, [C.POINTER(fl_decide_problem), _I, _I, C.POINTER(fl_decide_params), _P]),
     "fl_spec_accept": (_I, [_P, _P, _I, _P, _P, _P]),
+    "fl_shard_blocks": (_I, [_P, _I, _I, _I, _P]),
+    "fl_logit_gate_partial": (_I, [_P, _I, _I, _I, _P, _P]),
+    "fl_logit_gate_merge": (_I, [_P, _I, _I, _F, _F, _P, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _fn = getattr(_lib, _name)
@@ -304,3 +307,29 @@ def fl_level_decide(problems, n: int, batch: int, params: fl_decide_params, stre
 def fl_spec_accept(draft_top2, verified_top2, k: int, result, totals=None, stream=None) -> None:
     _check(_lib.fl_spec_accept(_ptr(draft_top2), _ptr(verified_top2), k, _ptr(result), _ptr(totals),
                                _stream(stream)))
+
+
+# ----------------------------------------------------------------------------- the read split over ranks
+
+GATE_PARTIAL_BYTES = 32  # one fl_gate_partial
+
+
+def fl_shard_blocks(levels, inn: int, nranks: int) -> list:
+    """Host levels (uint8 numpy array) -> [nranks + 1] first-block indices of each rank's range."""
+    import numpy as np
+    lv = np.ascontiguousarray(levels, dtype=np.uint8)
+    first = (C.c_int * (nranks + 1))()
+    _check(_lib.fl_shard_blocks(lv.ctypes.data if lv.size else None, int(lv.size), inn, nranks, first))
+    return [int(v) for v in first]
+
+
+def fl_logit_gate_partial(logits, vocab: int, batch: int, index_base: int, partial, stream=None) -> None:
+    """partial: a device buffer of batch * 32 bytes (fl_gate_partial records)."""
+    _check(_lib.fl_logit_gate_partial(_ptr(logits), vocab, batch, index_base, _ptr(partial), _stream(stream)))
+
+
+def fl_logit_gate_merge(partials, nparts: int, batch: int, tau_h: float, tau_m: float, entropy, margin, top2,
+                        escalate, stream=None) -> None:
+    """partials: device [nparts][batch] fl_gate_partial records (nparts * batch * 32 bytes)."""
+    _check(_lib.fl_logit_gate_merge(_ptr(partials), nparts, batch, float(tau_h), float(tau_m), _ptr(entropy),
+                                    _ptr(margin), _ptr(top2), _ptr(escalate), _stream(stream)))

@@ -145,6 +145,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// y += v as a reduction performed in L2 (no value returned, so nothing waits for it); the add
+// rounds to nearest like a plain fp32 add.
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t rotr32(uint32_t v, uint32_t n) {
   return __funnelshift_r(v, v, n);
 }

@@ -517,6 +517,20 @@ __device__ __forceinline__ void gate_publish(const Args<MAXP>& a, const GateRec&
   if (lane == 0) *a.gate_ticket = 0u;
 }
 
+// The consumer warps' partials gws [kConsumerWarps][batch] are in shared memory: warp 0 merges
+// them (one lane per warp) and publishes.
+template <int MAXP>
+__device__ __forceinline__ void gate_cta_finish(const Args<MAXP>& a, const GateRec* gws, int warp, int lane) {
+  named_bar(kBarGate, kConsumers);
+  if (warp != 0) return;
+  GateRec mine = empty_rec();
+  for (int bb = 0; bb < a.batch; ++bb) {
+    const GateRec r = warp_merge(lane < kConsumerWarps ? gws[lane * a.batch + bb] : empty_rec());
+    if (lane == bb) mine = r;
+  }
+  gate_publish(a, mine, lane);
+}
+
 // All consumer threads of a CTA that holds gate-problem units, after the CTA's outputs are
 // written: the CTA's rows of that problem are one contiguous range [r0, r1) (still in L2).
 // Every thread loads its strided share (up to kGateLoads values per batch row at once), takes
@@ -574,14 +588,7 @@ __device__ __forceinline__ void gate_cta_reduce(const Args<MAXP>& a, const float
     r = warp_merge(r);
     if (lane == 0) gws[warp * a.batch + bb] = r;
   }
-  named_bar(kBarGate, kConsumers);
-  if (warp != 0) return;
-  GateRec mine = empty_rec();
-  for (int bb = 0; bb < a.batch; ++bb) {
-    const GateRec r = warp_merge(lane < kConsumerWarps ? gws[lane * a.batch + bb] : empty_rec());
-    if (lane == bb) mine = r;
-  }
-  gate_publish(a, mine, lane);
+  gate_cta_finish(a, gws, warp, lane);
 }
 
 // Plane range [k0, k0 + np) read for block b, packed as k0 << 4 | np.
@@ -884,11 +891,14 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
         if ((t & 1) == 0 && bb < a.batch) {
           float* y0 = y + (size_t)bb * ystride + row_base + g;
           if (a.mode == 1) {
-            acc[nt][0] += y0[0];
-            acc[nt][1] += y0[8];
+            // the residual adds to y where y lives (a reduction in L2, no load on the team's
+            // path); each output is added to once per pass
+            red_add_f32(y0, acc[nt][0]);
+            red_add_f32(y0 + 8, acc[nt][1]);
+          } else {
+            y0[0] = acc[nt][0];
+            y0[8] = acc[nt][1];
           }
-          y0[0] = acc[nt][0];
-          y0[8] = acc[nt][1];
         }
       }
     } else {
@@ -919,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
             if (a.mode == 0)
               *yy = sum;
             else
-              *yy += sum;
+              red_add_f32(yy, sum);
           }
         } else
         // each thread's outputs (up to kRed) and slices: every load is issued before the sums
@@ -947,7 +957,7 @@ __global__ void __launch_bounds__(kThreads, 1) plane_gemv_kernel(const __grid_co
               if (a.mode == 0)
                 *yy = sum[q];
               else
-                *yy += sum[q];
+                red_add_f32(yy, sum[q]);
             }
           }
         }

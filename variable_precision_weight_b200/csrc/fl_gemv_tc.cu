@@ -546,7 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemv_kernel(const __grid_const
               const int bb = 8 * ch0 + i;
               if (bb < a.batch) {
                 float* yy = a.y + (size_t)bb * ystride + 64 * b + rb;
-                *yy = (a.mode == 0) ? acc[i] : *yy + acc[i];
+                if (a.mode == 0)
+                  *yy = acc[i];
+                else
+                  red_add_f32(yy, acc[i]);  // added where y lives: no load on the epilogue's path
               }
             }
           }
@@ -604,15 +607,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemv_kernel(const __grid_const
       if (b < a.nblk) {  // y is only 4-byte aligned: four scalar stores
         float* yy = a.y + (size_t)bb * 64 * a.nblk + 64 * b + rb;
         if (a.mode == 1) {
-          sum.x += yy[0];
-          sum.y += yy[1];
-          sum.z += yy[2];
-          sum.w += yy[3];
+          red_add_f32(yy, sum.x);
+          red_add_f32(yy + 1, sum.y);
+          red_add_f32(yy + 2, sum.z);
+          red_add_f32(yy + 3, sum.w);
+        } else {
+          yy[0] = sum.x;
+          yy[1] = sum.y;
+          yy[2] = sum.z;
+          yy[3] = sum.w;
         }
-        yy[0] = sum.x;
-        yy[1] = sum.y;
-        yy[2] = sum.z;
-        yy[3] = sum.w;
       }
     }
     __syncthreads();

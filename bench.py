@@ -52,8 +52,9 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config kernel measurements")
     ap.add_argument("--shard", action="store_true",
                     help="split every layer's blocks over the ranks (strong scaling) instead of one replica per GPU")
-    ap.add_argument("--profile", choices=["none", "step", "kquant", "kernels", "layer"], default="none",
-                    help="short run for an ncu capture: 'step' = the decode step only, 'kquant' = the K-quant "
+    ap.add_argument("--profile", choices=["none", "step", "residual", "kquant", "kernels", "layer"], default="none",
+                    help="short run for an ncu capture: 'step' = the decode step only, 'residual' = the decode "
+                         "step's D4 -> D8 residual pass (gate fused) three times, 'kquant' = the K-quant "
                          "step only, 'kernels' = one pass of every per-config kernel measurement, 'layer' = "
                          "three fl_gemv_depth calls on one layer (--shape, --batch, --level); no JSON "
                          "timing claims")
@@ -849,6 +850,14 @@ def run_fl(args, rank, world, local_rank):
         torch.cuda.synchronize()
         return 0
     step = DecodeStep(torch, fl, seed=1000 + rank)
+    if args.profile == "residual":
+        # after the 25 calibration launches: the D4 -> D8 residual pass (gate fused) of input
+        # set 0, three times, as the step runs it when the gate escalates
+        for k in range(3):
+            fl.fl_gemv_batched_gate(step.prob_res[0], step.n, 1, 1, step.specs[0])
+        torch.cuda.synchronize()
+        fl.fl_device_status()
+        return 0
     step.capture()
     NS = step.NSETS
 

@@ -57,6 +57,10 @@ constexpr int kEpiWarps = 8;                 // warps 8-15
 
 __host__ __device__ constexpr int n_cols(int batch) { return (4 * batch + 15) / 16 * 16; }
 
+// Column slice j of `slices` over G groups: groups [slice_first(j), slice_first(j + 1)), the
+// slices as equal as whole groups allow (widths differ by one at most).
+__host__ __device__ constexpr int slice_first(int j, int G, int slices) { return (int)((long long)j * G / slices); }
+
 struct Args {
   const uint8_t* store;
   const uint8_t* lv_from;
@@ -302,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemv_kernel(const __grid_const
       sl.u0 = u - u_begin;
       sl.u1 = ue - u_begin;
       sl.p0 = u - j * a.npair;
-      sl.gfirst = j * a.slice_groups;
-      sl.ng = min(a.slice_groups, a.G - sl.gfirst);
+      sl.gfirst = slice_first(j, a.G, a.slices);
+      sl.ng = slice_first(j + 1, a.G, a.slices) - sl.gfirst;
       sl.dig = base + off;
       off += (uint32_t)(a.N * 128 * sl.ng);
       sl.gc = base + off;
@@ -636,7 +640,10 @@ static int groups_fit(int batch) {
 }
 
 // Column slices: as wide as the digits allow, and narrow enough that the units (slice x block
-// pair) number about four per SM, so contiguous ranges balance.
+// pair) number about four per SM, so contiguous ranges balance. The slices are equal to a group
+// (slice_first): a short last slice made a CTA of many small units, each paying the unit's fixed
+// cost, the launch's slowest (4096 -> 14336 at batch 16: 52.6 us with a two-group last slice,
+// 34.0 us with equal ones).
 static Plan plan(int nblk, int G, int batch, int nsm) {
   Plan pl;
   pl.npair = (nblk + 1) / 2;
@@ -668,25 +675,29 @@ static WsLayout ws_layout(const Plan& pl, int G, int batch) {
   return w;
 }
 
-// Contiguous ranges of units (slice-major), balanced by groups read; a range is also cut when
+// A unit's fixed cost (its end: partial stores, the epilogue's barrier and ticket), in groups.
+constexpr double kUnitCost = 1.0;
+
+// Contiguous ranges of units (slice-major), balanced by groups read plus each unit's fixed cost; a range is also cut when
 // the digits of the slices it touches would overflow shared memory, at kMaxSlots slices, or at
 // the level-cache size; after every cut the rest is spread evenly over the ranges still to make.
 static bool partition(Args& a, const Plan& pl, int nsm, size_t* max_dig) {
   const int units = pl.slices * pl.npair;
   const int target = std::max(1, std::min(nsm, units));
   double total = 0;
-  for (int j = 0; j < pl.slices; ++j) total += (double)pl.npair * std::min(pl.slice_groups, a.G - j * pl.slice_groups);
+  for (int j = 0; j < pl.slices; ++j)
+    total += (double)pl.npair * (slice_first(j + 1, a.G, pl.slices) - slice_first(j, a.G, pl.slices) + kUnitCost);
   double per = total / target, acc = 0, start = 0;
   int n = 0, nslots = 0, count = 0;
   size_t dig = 0;
   a.cta_begin[0] = 0;
   for (int u = 0; u < units; ++u) {
     const int j = u / pl.npair, p = u % pl.npair;
-    const int ng = std::min(pl.slice_groups, a.G - j * pl.slice_groups);
+    const int ng = slice_first(j + 1, a.G, pl.slices) - slice_first(j, a.G, pl.slices);
     const size_t sb = (((size_t)pl.N * 128 * ng + 16 * a.batch * ng) + 1023) / 1024 * 1024;
     bool cut = false;
     if (count > 0) {
-      if (n + 1 < target && acc + 0.5 * ng - start > per) cut = true;
+      if (n + 1 < target && acc + 0.5 * (ng + kUnitCost) - start > per) cut = true;
       if ((p == 0 || count == 0) && (dig + sb > (size_t)kDigitBudget || nslots == kMaxSlots)) cut = true;
       if (count == kLevelCache) cut = true;
     }
@@ -704,7 +715,7 @@ static bool partition(Args& a, const Plan& pl, int nsm, size_t* max_dig) {
       dig += sb;
       ++nslots;
     }
-    acc += ng;
+    acc += ng + kUnitCost;
     ++count;
   }
   a.cta_begin[++n] = units;

@@ -103,6 +103,7 @@ CASES = [
     (640, 3072, 20, "zero_heavy"),
     (64, 4096, 32, "uniform"),        # one block, column slices
     (256, 14336, 32, "uniform"),      # few blocks, wide rows: many column slices + tickets
+    (7680, 1664, 16, "uniform"),      # 60 pairs: 13 groups over 10 slices of one or two groups
 ]
 
 

@@ -412,9 +412,10 @@ FL_API fl_status fl_logit_gate_partial(const float* logits, int vocab, int batch
                                        fl_gate_partial* partial, void* stream);
 
 /* Merge nparts partials per row, partials laid out [nparts][batch] (the gathered pieces in
- * rank order), in that order, and write entropy / margin / top2 / escalate exactly as
- * fl_logit_gate defines them for the whole row (equal up to fp32 summation order). Every rank
- * that merges the same partials computes the same outputs. Output pointers as fl_logit_gate;
+ * rank order), in one fixed order (lane l of a warp takes parts l, l + 32, ..., then the lanes
+ * merge in a fixed tree), and write entropy / margin / top2 / escalate exactly as fl_logit_gate
+ * defines them for the whole row (equal up to fp32 summation order; top2 ties go to the lower
+ * global index). Every rank that merges the same partials computes the same outputs. Output pointers as fl_logit_gate;
  * partials device, 16-byte aligned; 1 <= nparts <= 4096. One launch. */
 FL_API fl_status fl_logit_gate_merge(const fl_gate_partial* partials, int nparts, int batch, float tau_h, float tau_m,
                                      float* entropy, float* margin, int32_t* top2, uint8_t* escalate, void* stream);

@@ -332,7 +332,8 @@ FL_API fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, int n,
 /*           floor(f * out / 64) entries receive the lifted blocks' indices   */
 /*           in ascending order (the block list of fl_gemv_batched_listed)    */
 /* params: 1 <= gamma <= kappa <= 4; ladder: lambda finite, >= 0; share:     */
-/* 0 <= f <= 1. One launch (ladder) or two (share), asynchronous on stream.   */
+/* 0 <= f <= 1. One launch (ladder, or share with counters) or two (share),   */
+/* asynchronous on stream.                                                    */
 /* ========================================================================= */
 #define FL_DECIDE_LADDER 0
 #define FL_DECIDE_SHARE 1
@@ -345,12 +346,18 @@ typedef struct {
   int32_t* lifted;
 } fl_decide_problem;
 
+/* counters (share rule; may be NULL): device int32 [n], 4-byte aligned, ZERO-FILLED before
+ * first use and left zero by every completed call. With counters the share rule takes one
+ * launch: each CTA adds the blocks it scored to its layers' counters, and the CTA whose addition
+ * completes a layer selects that layer's share at once. Without them (and for the ladder) the
+ * selection is a second launch. Calls sharing counters must not overlap. */
 typedef struct {
   int rule;
   int gamma;
   int kappa;
   float lambda;
   float f;
+  int32_t* counters;
 } fl_decide_params;
 
 FL_API fl_status fl_level_decide(const fl_decide_problem* problems, int n, int batch, const fl_decide_params* params,

@@ -120,16 +120,23 @@ def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
     up_out = [torch.full((o // 64,), -1, dtype=torch.int32, device="cuda") for o, _ in shapes]
     probs = fl.decide_problems([(it[0], it[1], it[2], it[6], lv, sc, up)
                                 for it, lv, sc, up in zip(items, lv_out, sc_out, up_out)])
-    for rule, lam_, f in ((fl.FL_DECIDE_LADDER, lam, 0.0), (fl.FL_DECIDE_LADDER, 0.0, 0.0),
-                          (fl.FL_DECIDE_LADDER, 1e30, 0.0), (fl.FL_DECIDE_SHARE, 0.0, 0.0),
-                          (fl.FL_DECIDE_SHARE, 0.0, 0.16), (fl.FL_DECIDE_SHARE, 0.0, 0.5),
-                          (fl.FL_DECIDE_SHARE, 0.0, 1.0)):
-        fl.fl_level_decide(probs, len(shapes), batch, fl.decide_params(rule, gamma, kappa, lam_, f))
+    counters = torch.zeros(len(shapes), dtype=torch.int32, device="cuda")
+    for rule, lam_, f, one in ((fl.FL_DECIDE_LADDER, lam, 0.0, False), (fl.FL_DECIDE_LADDER, 0.0, 0.0, False),
+                               (fl.FL_DECIDE_LADDER, 1e30, 0.0, False), (fl.FL_DECIDE_SHARE, 0.0, 0.0, False),
+                               (fl.FL_DECIDE_SHARE, 0.0, 0.16, False), (fl.FL_DECIDE_SHARE, 0.0, 0.5, False),
+                               (fl.FL_DECIDE_SHARE, 0.0, 1.0, False), (fl.FL_DECIDE_SHARE, 0.0, 0.0, True),
+                               (fl.FL_DECIDE_SHARE, 0.0, 0.16, True), (fl.FL_DECIDE_SHARE, 0.0, 0.5, True),
+                               (fl.FL_DECIDE_SHARE, 0.0, 1.0, True)):
+        for t in up_out:
+            t.fill_(-1)
+        fl.fl_level_decide(probs, len(shapes), batch,
+                           fl.decide_params(rule, gamma, kappa, lam_, f, counters if one else None))
         torch.cuda.synchronize()
+        assert int(counters.abs().sum().item()) == 0          # the one-launch counters are left zero
         for i, (y, (q, s, x)) in enumerate(zip(ys, host)):
             lev, sc = lv_out[i].cpu().numpy(), sc_out[i].cpu().numpy()
             ref_lev, ref_red = orc.level_decide(y, s, gamma, kappa, rule, lam=lam_, f=np.float32(f))
-            what = f"rule {rule} lam {lam_} f {f} problem {i}"
+            what = f"rule {rule} lam {lam_} f {f} one launch {one} problem {i}"
             if rule == fl.FL_DECIDE_LADDER:
                 check_ladder(lev, sc, ref_lev, ref_red, gamma, kappa, lam_, what)
             else:
@@ -149,8 +156,9 @@ def test_ladder_and_share_vs_oracle(env, orc, gamma, batch):
         check_ladder(lev, sc, ref_lev, ref_red, gamma, kappa, lam, f"no-score ladder problem {i}")
 
 
+@pytest.mark.parametrize("one", [False, True])
 @pytest.mark.parametrize("nb", [10, 400])
-def test_share_ties_go_to_lower_index(env, orc, nb):
+def test_share_ties_go_to_lower_index(env, orc, nb, one):
     """Identical blocks give bit-identical scores; the share lifts the lowest indices (10
     blocks: the one-warp ranking; 400: the radix select, the cut inside the tied group)."""
     torch, fl = env
@@ -165,8 +173,9 @@ def test_share_ties_go_to_lower_index(env, orc, nb):
     lv = torch.empty(nb, dtype=torch.uint8, device="cuda")
     sc = torch.empty(nb, dtype=torch.float32, device="cuda")
     f = 0.35
+    counters = torch.zeros(1, dtype=torch.int32, device="cuda") if one else None
     fl.fl_level_decide(fl.decide_problems([(st, o, n, yd, lv, sc)]), 1, 2,
-                       fl.decide_params(fl.FL_DECIDE_SHARE, 2, 3, f=f))
+                       fl.decide_params(fl.FL_DECIDE_SHARE, 2, 3, f=f, counters=counters))
     torch.cuda.synchronize()
     n_up = int(np.floor(np.float64(np.float32(f)) * nb))
     scores = sc.cpu().numpy()
@@ -176,8 +185,8 @@ def test_share_ties_go_to_lower_index(env, orc, nb):
     assert np.array_equal(orc.level_decide(y, s, 2, 3, 1, f=np.float32(f))[0], lv.cpu().numpy())
 
 
-@pytest.mark.parametrize("rule", [0, 1])
-def test_in_pass_pipeline(env, orc, rule):
+@pytest.mark.parametrize("rule,one", [(0, False), (1, False), (1, True)])
+def test_in_pass_pipeline(env, orc, rule, one):
     """Base pass at D4 -> decision -> residual pass from D4 to the decided levels, all layers
     in one launch each: y equals the oracle's depth GEMV at the decided levels."""
     torch, fl = env
@@ -192,7 +201,8 @@ def test_in_pass_pipeline(env, orc, rule):
     sc = [torch.empty(o // 64, dtype=torch.float32, device="cuda") for o, _ in shapes]
     up = [torch.empty(o // 64, dtype=torch.int32, device="cuda") for o, _ in shapes]
     probs = fl.decide_problems([(it[0], it[1], it[2], it[6], t, c, u) for it, t, c, u in zip(items, to, sc, up)])
-    params = fl.decide_params(rule, gamma, kappa, lam, 0.16)
+    counters = torch.zeros(len(shapes), dtype=torch.int32, device="cuda") if one else None
+    params = fl.decide_params(rule, gamma, kappa, lam, 0.16, counters)
     fl.fl_level_decide(probs, len(shapes), batch, params)
     res = [(it[0], it[1], it[2], it[3], t, it[5], it[6]) for it, t in zip(items, to)]
     if rule == fl.FL_DECIDE_SHARE:          # residual over the lifted blocks only
@@ -216,7 +226,8 @@ def test_in_pass_pipeline(env, orc, rule):
     assert lifted > 0
 
 
-def test_share_rule_on_a_layer_too_large_for_shared_memory(env, orc):
+@pytest.mark.parametrize("one", [False, True])
+def test_share_rule_on_a_layer_too_large_for_shared_memory(env, orc, one):
     """A layer of 12,000 blocks: the selection reads the scores from global memory."""
     torch, fl = env
     o, n = 64 * 12000, 128
@@ -234,8 +245,9 @@ def test_share_rule_on_a_layer_too_large_for_shared_memory(env, orc):
     ref_red = orc.level_decide(y.cpu().numpy(), s.cpu().numpy(), 2, 4, 0, lam=1.0)[1]
     rank0 = int((ref_red > ref_red[0]).sum())             # blocks scoring above the tied group
     for f in (0.25, (rank0 + 20) / 12000, 0.999):          # the second cuts the tied group
+        counters = torch.zeros(1, dtype=torch.int32, device="cuda") if one else None
         fl.fl_level_decide(fl.decide_problems([(st, o, n, y, lv, sc)]), 1, 1,
-                           fl.decide_params(fl.FL_DECIDE_SHARE, 2, 4, f=f))
+                           fl.decide_params(fl.FL_DECIDE_SHARE, 2, 4, f=f, counters=counters))
         torch.cuda.synchronize()
         ref_lev, ref_red = orc.level_decide(y.cpu().numpy(), s.cpu().numpy(), 2, 4, 1, f=np.float32(f))
         check_share(lv.cpu().numpy(), sc.cpu().numpy(), ref_lev, ref_red, 2, 4, f, f"large layer f {f}")

@@ -23,6 +23,11 @@
 // over the 64-bit keys with per-warp shared-memory histograms, its scores staged in shared
 // memory up to 7,680 blocks. It then writes every block's level and, when asked, the lifted
 // blocks' indices in ascending order (a block-wide scan per 512 blocks).
+// score_select_kernel (share rule with caller counters, one launch): CTAs score contiguous
+// chunks of blocks and count them per layer; the CTA that completes a layer's count runs the
+// same selection with its 256 threads. On the 197-layer decode step it measured slower than
+// the two launches (16.4 against 11.4 us): the head layer's selection then starts only after
+// the last chunk is scored and runs on half the threads.
 #include <math.h>
 
 #include "fl_common.cuh"
@@ -56,6 +61,8 @@ struct Args {
   int kappa;
   float lambda;
   float step2;                     // (2^(8 - 2 gamma))^2
+  int32_t* counters;               // share rule in one launch: blocks scored per problem (or NULL)
+  int chunk;                       // blocks per CTA of the one-launch variant
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -64,12 +71,167 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+constexpr int kWarpRank = 256;     // layers up to this many blocks: one warp ranks the keys
+constexpr int kSmemScores = 7680;   // a layer's scores staged in shared memory up to this many blocks (30 KB)
+
+// key of block i: larger score first, then the lower index (scores are >= 0, so their bit
+// patterns order like their values). Scores may have been written by other CTAs of the same
+// launch: they are read at L2 (`ld.global.cg`), never from a CTA's own L1.
+__device__ __forceinline__ uint64_t share_key(const float* score, int i) {
+  return ((uint64_t)__float_as_uint(__ldcg(score + i)) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
+}
+__device__ __forceinline__ uint64_t share_key_smem(const float* score, int i) {
+  return ((uint64_t)__float_as_uint(score[i]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
+}
+
+template <int T>
+struct ShareSmem {
+  uint32_t hist[T / 32][256];  // one histogram per warp: positive scores share their top bits,
+                               // so one shared bin would serialise
+  uint64_t prefix;
+  uint32_t left, tied;
+  int warp_up[T / 32];
+};
+
+// The share rule for problem P by all T threads of a CTA: the floor(f n) largest keys rise to
+// kappa. s_score: dynamic shared memory for up to kSmemScores staged scores.
+template <int T>
+__device__ void select_share(const Problem& P, int gamma, int kappa, float* s_score, ShareSmem<T>& sm, int tid) {
+  constexpr int W = T / 32;
+  const int nb = P.out / 64;
+  const float* score = P.score;
+  if (nb <= kWarpRank) {
+    // small layer: one warp ranks every key against all others (keys are distinct, so a key
+    // rises iff fewer than n_up keys exceed it); no block-wide barrier
+    if (tid >= 32) return;
+    uint64_t key[kWarpRank / 32];
+#pragma unroll
+    for (int m = 0; m < kWarpRank / 32; ++m) {
+      const int i = 32 * m + tid;
+      key[m] = i < nb ? share_key(score, i) : 0ull;
+    }
+    int above[kWarpRank / 32] = {};
+#pragma unroll
+    for (int m2 = 0; m2 < kWarpRank / 32; ++m2) {
+      if (32 * m2 >= nb) break;
+      for (int src = 0; src < 32; ++src) {
+        const uint64_t kj = __shfl_sync(0xffffffffu, key[m2], src);
+        if (32 * m2 + src < nb) {
+#pragma unroll
+          for (int m = 0; m < kWarpRank / 32; ++m) above[m] += kj > key[m];
+        }
+      }
+    }
+    int base = 0;
+#pragma unroll
+    for (int m = 0; m < kWarpRank / 32; ++m) {
+      const int i = 32 * m + tid;
+      const bool up = i < nb && above[m] < P.n_up;
+      if (i < nb) P.levels[i] = (uint8_t)(up ? kappa : gamma);
+      const unsigned bal = __ballot_sync(0xffffffffu, up);
+      if (up && P.lifted) P.lifted[base + __popc(bal & ((1u << tid) - 1u))] = i;
+      base += __popc(bal);
+    }
+    return;
+  }
+  const bool staged = nb <= kSmemScores;
+  if (staged) {
+    for (int i = tid; i < nb; i += T) s_score[i] = __ldcg(score + i);
+    __syncthreads();
+  }
+  auto key_of = [&](int i) { return staged ? share_key_smem(s_score, i) : share_key(score, i); };
+  uint64_t kth = 0;                         // with 0 < n_up < nb: the keys >= kth rise
+  if (P.n_up > 0 && P.n_up < nb) {
+    if (tid == 0) {
+      sm.prefix = 0;
+      sm.left = (uint32_t)P.n_up;
+    }
+    // radix select of the n_up-th largest key, 8 bits a pass from the top; the four passes
+    // over the score bits settle it unless the cut falls inside a group of equal scores,
+    // which the four passes over the index bits then split lower index first
+    for (int pass = 0; pass < 8; ++pass) {
+      const int shift = 56 - 8 * pass;
+      for (int d = tid; d < W * 256; d += T) (&sm.hist[0][0])[d] = 0;
+      __syncthreads();
+      const uint64_t prefix = sm.prefix;
+      const uint64_t mask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+      uint32_t* const my = sm.hist[tid >> 5];
+      for (int i = tid; i < nb; i += T) {
+        const uint64_t k = key_of(i);
+        if ((k & mask) == prefix) atomicAdd(&my[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      for (int d = tid; d < 256; d += T) {
+        uint32_t sum = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) sum += sm.hist[w][d];
+        sm.hist[0][d] = sum;
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // lane l owns digits 255 - 8 l down to 248 - 8 l; find the digit where the count of
+        // larger keys first reaches left
+        uint32_t cnt[8], tot = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          cnt[k] = sm.hist[0][255 - 8 * tid - k];
+          tot += cnt[k];
+        }
+        uint32_t before = tot;              // inclusive scan over lanes, then exclusive
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, before, o);
+          if (tid >= o) before += v;
+        }
+        before -= tot;
+        const uint32_t left = sm.left;
+        const bool mine = before < left && left <= before + tot;
+        if (mine) {
+          uint32_t acc = before;
+          int k = 0;
+          while (acc + cnt[k] < left) acc += cnt[k++];
+          const uint32_t digit = 255u - 8u * tid - (uint32_t)k;
+          sm.prefix = prefix | ((uint64_t)digit << shift);
+          sm.left = left - acc;
+          sm.tied = cnt[k];
+        }
+      }
+      __syncthreads();
+      if (pass == 3 && sm.left == sm.tied) break;   // every key with the cut's score rises
+    }
+    kth = sm.prefix;
+  }
+  // levels, and the lifted indices in ascending order (a block-wide scan per T blocks)
+  int base = 0;
+  for (int i0 = 0; i0 < nb; i0 += T) {
+    const int i = i0 + tid;
+    const bool up = i < nb && (P.n_up >= nb || (P.n_up > 0 && key_of(i) >= kth));
+    if (i < nb) P.levels[i] = (uint8_t)(up ? kappa : gamma);
+    if (P.lifted == nullptr) continue;
+    const unsigned bal = __ballot_sync(0xffffffffu, up);
+    if ((tid & 31) == 0) sm.warp_up[tid >> 5] = __popc(bal);
+    __syncthreads();
+    int before = base, total = 0;
+    for (int w = 0; w < W; ++w) {
+      const int c = sm.warp_up[w];
+      if (w < (tid >> 5)) before += c;
+      total += c;
+    }
+    if (up) P.lifted[before + __popc(bal & ((1u << (tid & 31)) - 1u))] = i;
+    base += total;
+    __syncthreads();
+  }
+}
+
+// The score of every block (one warp per block) and, for the ladder, its level. The fused
+// variant (share rule, one launch): each CTA scores a contiguous chunk of a.chunk blocks, adds
+// them to the counters of the layers they belong to, and the CTA whose addition completes a
+// layer selects that layer's share at once (select_share with the CTA's 256 threads), then
+// clears the counter.
+constexpr int kMaxChunk = 64;   // blocks per CTA of the fused variant
+
 template <int MAXP>
-__global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constant__ Args<MAXP> a) {
-  pdl_release();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gb = blockIdx.x * kWarps + warp;
-  if (gb >= a.nblocks) return;
+__device__ __forceinline__ void score_block(const Args<MAXP>& a, int gb, int lane) {
   // the problem holding global block gb: the last one whose block_begin <= gb
   int lo = 0, hi = a.nproblems - 1;
   while (lo < hi) {
@@ -79,8 +241,6 @@ __global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constan
   }
   const Problem& P = a.p[lo];
   const int c = gb - P.block_begin;
-  pdl_wait();
-
   // squared outputs of the block's 64 rows, every batch row, and squared scales of the
   // block ([G][64] fp32 at the head of its 8448 G bytes); loads issued four at a time
   float yy = 0.f, ss = 0.f;
@@ -88,9 +248,8 @@ __global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constan
     float2 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      v[u] = t0 + u < a.batch
-                 ? *reinterpret_cast<const float2*>(P.y + (size_t)(t0 + u) * P.out + 64 * c + 2 * lane)
-                 : make_float2(0.f, 0.f);
+      v[u] = t0 + u < a.batch ? *reinterpret_cast<const float2*>(P.y + (size_t)(t0 + u) * P.out + 64 * c + 2 * lane)
+                              : make_float2(0.f, 0.f);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       yy = fmaf(v[u].x, v[u].x, yy);
@@ -129,151 +288,64 @@ __global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constan
     }
     P.levels[c] = (uint8_t)lev;
   }
+  if (a.counters) __threadfence();  // the score, device-wide, before the CTA's count
 }
 
-constexpr int kWarpRank = 256;     // layers up to this many blocks: one warp ranks the keys
-constexpr int kSmemScores = 7680;   // a layer's scores staged in shared memory up to this many blocks (30 KB)
-constexpr int kShareWarps = kShareThreads / 32;
+template <int MAXP>
+__global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constant__ Args<MAXP> a) {
+  pdl_release();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gb = blockIdx.x * kWarps + warp;
+  pdl_wait();
+  if (gb < a.nblocks) score_block(a, gb, lane);
+}
 
-// key of block i: larger score first, then the lower index (scores are >= 0, so their bit
-// patterns order like their values)
-__device__ __forceinline__ uint64_t share_key(const float* score, int i) {
-  return ((uint64_t)__float_as_uint(score[i]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
+template <int MAXP>
+__global__ void __launch_bounds__(32 * kWarps) score_select_kernel(const __grid_constant__ Args<MAXP> a) {
+  extern __shared__ float s_score[];             // the selected layer's staged scores
+  __shared__ ShareSmem<32 * kWarps> sm;
+  __shared__ int s_last[kMaxChunk];              // layers whose counts this CTA completed
+  __shared__ int s_nlast;
+  pdl_release();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = blockIdx.x * a.chunk, c1 = min(c0 + a.chunk, a.nblocks);
+  pdl_wait();
+  for (int gb = c0 + warp; gb < c1; gb += kWarps) score_block(a, gb, lane);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // the layers overlapping [c0, c1): the first is the last whose block_begin <= c0
+    int lo = 0, hi = a.nproblems - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.p[mid].block_begin <= c0) lo = mid;
+      else hi = mid - 1;
+    }
+    int n = 0;
+    for (int p = lo; p < a.nproblems && a.p[p].block_begin < c1; ++p) {
+      const int pb = a.p[p].block_begin, nb = a.p[p].out / 64;
+      const int cnt = min(c1, pb + nb) - max(c0, pb);
+      if (cnt > 0 && atomicAdd(&a.counters[p], cnt) + cnt == nb) s_last[n++] = p;
+    }
+    if (n) __threadfence();  // the other CTAs' scores are read after their counts
+    s_nlast = n;
+  }
+  __syncthreads();
+  for (int k = 0; k < s_nlast; ++k) {
+    const int p = s_last[k];
+    select_share<32 * kWarps>(a.p[p], a.gamma, a.kappa, s_score, sm, threadIdx.x);
+    __syncthreads();
+    if (threadIdx.x == 0) a.counters[p] = 0;
+  }
 }
 
 template <int MAXP>
 __global__ void __launch_bounds__(kShareThreads) share_kernel(const __grid_constant__ Args<MAXP> a) {
   extern __shared__ float s_score[];
-  __shared__ uint32_t hist[kShareWarps][256];  // one histogram per warp: positive scores share
-                                               // their top bits, so one shared bin would serialise
-  __shared__ uint64_t s_prefix;
-  __shared__ uint32_t s_left, s_tied;
+  __shared__ ShareSmem<kShareThreads> sm;
   pdl_release();
   const Problem& P = a.p[blockIdx.x];
-  const int nb = P.out / 64;
-  const int tid = threadIdx.x;
   pdl_wait();
-  const float* score = P.score;
-  if (nb <= kWarpRank) {
-    // small layer: one warp ranks every key against all others (keys are distinct, so a key
-    // rises iff fewer than n_up keys exceed it); no block-wide barrier
-    if (tid >= 32) return;
-    uint64_t key[kWarpRank / 32];
-#pragma unroll
-    for (int m = 0; m < kWarpRank / 32; ++m) {
-      const int i = 32 * m + tid;
-      key[m] = i < nb ? share_key(score, i) : 0ull;
-    }
-    int above[kWarpRank / 32] = {};
-#pragma unroll
-    for (int m2 = 0; m2 < kWarpRank / 32; ++m2) {
-      if (32 * m2 >= nb) break;
-      for (int src = 0; src < 32; ++src) {
-        const uint64_t kj = __shfl_sync(0xffffffffu, key[m2], src);
-        if (32 * m2 + src < nb) {
-#pragma unroll
-          for (int m = 0; m < kWarpRank / 32; ++m) above[m] += kj > key[m];
-        }
-      }
-    }
-    int base = 0;
-#pragma unroll
-    for (int m = 0; m < kWarpRank / 32; ++m) {
-      const int i = 32 * m + tid;
-      const bool up = i < nb && above[m] < P.n_up;
-      if (i < nb) P.levels[i] = (uint8_t)(up ? a.kappa : a.gamma);
-      const unsigned bal = __ballot_sync(0xffffffffu, up);
-      if (up && P.lifted) P.lifted[base + __popc(bal & ((1u << tid) - 1u))] = i;
-      base += __popc(bal);
-    }
-    return;
-  }
-  uint64_t kth = 0;                         // with 0 < n_up < nb: the keys >= kth rise
-  if (P.n_up > 0 && P.n_up < nb) {
-    if (nb <= kSmemScores) {
-      for (int i = tid; i < nb; i += kShareThreads) s_score[i] = score[i];
-      score = s_score;
-    }
-    if (tid == 0) {
-      s_prefix = 0;
-      s_left = (uint32_t)P.n_up;
-    }
-    // radix select of the n_up-th largest key, 8 bits a pass from the top; the four passes
-    // over the score bits settle it unless the cut falls inside a group of equal scores,
-    // which the four passes over the index bits then split lower index first
-    for (int pass = 0; pass < 8; ++pass) {
-      const int shift = 56 - 8 * pass;
-      for (int d = tid; d < kShareWarps * 256; d += kShareThreads) (&hist[0][0])[d] = 0;
-      __syncthreads();
-      const uint64_t prefix = s_prefix;
-      const uint64_t mask = pass == 0 ? 0ull : (~0ull << (shift + 8));
-      uint32_t* const my = hist[tid >> 5];
-      for (int i = tid; i < nb; i += kShareThreads) {
-        const uint64_t k = share_key(score, i);
-        if ((k & mask) == prefix) atomicAdd(&my[(k >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (tid < 256) {
-        uint32_t sum = 0;
-#pragma unroll
-        for (int w = 0; w < kShareWarps; ++w) sum += hist[w][tid];
-        hist[0][tid] = sum;
-      }
-      __syncthreads();
-      if (tid < 32) {
-        // lane l owns digits 255 - 8 l down to 248 - 8 l; find the digit where the count of
-        // larger keys first reaches s_left
-        uint32_t cnt[8], tot = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          cnt[k] = hist[0][255 - 8 * tid - k];
-          tot += cnt[k];
-        }
-        uint32_t before = tot;              // inclusive scan over lanes, then exclusive
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t v = __shfl_up_sync(0xffffffffu, before, o);
-          if (tid >= o) before += v;
-        }
-        before -= tot;
-        const uint32_t left = s_left;
-        const bool mine = before < left && left <= before + tot;
-        if (mine) {
-          uint32_t acc = before;
-          int k = 0;
-          while (acc + cnt[k] < left) acc += cnt[k++];
-          const uint32_t digit = 255u - 8u * tid - (uint32_t)k;
-          s_prefix = prefix | ((uint64_t)digit << shift);
-          s_left = left - acc;
-          s_tied = cnt[k];
-        }
-      }
-      __syncthreads();
-      if (pass == 3 && s_left == s_tied) break;   // every key with the cut's score rises
-    }
-    kth = s_prefix;
-  }
-  // levels, and the lifted indices in ascending order (a block-wide scan per 512 blocks)
-  __shared__ int s_warp_up[kShareWarps];
-  int base = 0;
-  for (int i0 = 0; i0 < nb; i0 += kShareThreads) {
-    const int i = i0 + tid;
-    const bool up = i < nb && (P.n_up >= nb || (P.n_up > 0 && share_key(score, i) >= kth));
-    if (i < nb) P.levels[i] = (uint8_t)(up ? a.kappa : a.gamma);
-    if (P.lifted == nullptr) continue;
-    const unsigned bal = __ballot_sync(0xffffffffu, up);
-    if ((tid & 31) == 0) s_warp_up[tid >> 5] = __popc(bal);
-    __syncthreads();
-    int before = base, total = 0;
-    for (int w = 0; w < kShareWarps; ++w) {
-      const int c = s_warp_up[w];
-      if (w < (tid >> 5)) before += c;
-      total += c;
-    }
-    if (up) P.lifted[before + __popc(bal & ((1u << (tid & 31)) - 1u))] = i;
-    base += total;
-    __syncthreads();
-  }
+  select_share<kShareThreads>(P, a.gamma, a.kappa, s_score, sm, threadIdx.x);
 }
 
 }  // namespace decide
@@ -303,6 +375,8 @@ extern "C" fl_status fl_level_decide(const fl_decide_problem* problems, int n, i
   a.gamma = q.gamma;
   a.kappa = q.kappa;
   a.lambda = q.lambda;
+  a.counters = q.rule == FL_DECIDE_SHARE ? q.counters : nullptr;
+  if (reinterpret_cast<uintptr_t>(q.counters) & 3u) return fail(FL_ERR_ALIGN, "%s: counters not 4-byte aligned", what);
   const float step = (float)(1 << (8 - 2 * q.gamma));
   a.step2 = step * step;
   long blocks = 0;
@@ -339,14 +413,25 @@ extern "C" fl_status fl_level_decide(const fl_decide_problem* problems, int n, i
   a.nblocks = (int)blocks;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)((blocks + kWarps - 1) / kWarps);
+  int max_nb = 0;
+  for (int i = 0; i < n; ++i) max_nb = max_nb > problems[i].w.out / 64 ? max_nb : problems[i].w.out / 64;
+  const size_t stage = sizeof(float) * (size_t)(max_nb < kSmemScores ? max_nb : kSmemScores);
+  if (a.counters) {  // share rule, one launch: the last CTA to score a layer selects it
+    // chunks of whole warps' blocks, about four CTAs per SM (one wave at this kernel's registers)
+    const int nsm = device_sm_count();
+    if (nsm <= 0) return fail(FL_ERR_CUDA, "%s: no CUDA device", what);
+    long per = (blocks + 4L * nsm - 1) / (4L * nsm);
+    per = (per + kWarps - 1) / kWarps * kWarps;
+    a.chunk = (int)(per < kWarps ? kWarps : per > kMaxChunk ? kMaxChunk : per);
+    const unsigned fgrid = (unsigned)((blocks + a.chunk - 1) / a.chunk);
+    FL_CHECK_CUDA(launch_pdl(score_select_kernel<FL_MAX_PROBLEMS>, dim3(fgrid), dim3(32 * kWarps), stage, st, 1, a),
+                  "launch level_decide score+select");
+    return FL_OK;
+  }
   FL_CHECK_CUDA(launch_pdl(score_kernel<FL_MAX_PROBLEMS>, dim3(grid), dim3(32 * kWarps), 0, st, 1, a),
                 "launch level_decide score");
-  if (q.rule == FL_DECIDE_SHARE) {
-    int max_nb = 0;
-    for (int i = 0; i < n; ++i) max_nb = max_nb > problems[i].w.out / 64 ? max_nb : problems[i].w.out / 64;
-    const size_t smem = sizeof(float) * (size_t)(max_nb < kSmemScores ? max_nb : kSmemScores);
-    FL_CHECK_CUDA(launch_pdl(share_kernel<FL_MAX_PROBLEMS>, dim3((unsigned)n), dim3(kShareThreads), smem, st, 1, a),
+  if (q.rule == FL_DECIDE_SHARE)
+    FL_CHECK_CUDA(launch_pdl(share_kernel<FL_MAX_PROBLEMS>, dim3((unsigned)n), dim3(kShareThreads), stage, st, 1, a),
                   "launch level_decide share");
-  }
   return FL_OK;
 }

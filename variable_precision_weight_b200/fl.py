@@ -68,7 +68,8 @@ class fl_decide_problem(C.Structure):
 
 
 class fl_decide_params(C.Structure):
-    _fields_ = [("rule", C.c_int), ("gamma", C.c_int), ("kappa", C.c_int), ("lambda_", C.c_float), ("f", C.c_float)]
+    _fields_ = [("rule", C.c_int), ("gamma", C.c_int), ("kappa", C.c_int), ("lambda_", C.c_float), ("f", C.c_float),
+                ("counters", C.c_void_p)]
 
 
 FL_DECIDE_LADDER = 0
@@ -296,8 +297,11 @@ def decide_problems(items) -> "C.Array":
     return arr
 
 
-def decide_params(rule: int, gamma: int, kappa: int, lam: float = 0.0, f: float = 0.0) -> fl_decide_params:
-    return fl_decide_params(rule, gamma, kappa, float(lam), float(f))
+def decide_params(rule: int, gamma: int, kappa: int, lam: float = 0.0, f: float = 0.0,
+                  counters=None) -> fl_decide_params:
+    """counters: a zero-filled device int32 tensor of one entry per problem makes the share rule
+    one launch (the last CTA to score a layer selects it)."""
+    return fl_decide_params(rule, gamma, kappa, float(lam), float(f), _ptr(counters))
 
 
 def fl_level_decide(problems, n: int, batch: int, params: fl_decide_params, stream=None) -> None:

@@ -230,15 +230,20 @@ __device__ void select_share(const Problem& P, int gamma, int kappa, float* s_sc
 // clears the counter.
 constexpr int kMaxChunk = 64;   // blocks per CTA of the fused variant
 
+// The problem holding global block gb: the last one whose block_begin <= gb.
 template <int MAXP>
-__device__ __forceinline__ void score_block(const Args<MAXP>& a, int gb, int lane) {
-  // the problem holding global block gb: the last one whose block_begin <= gb
+__device__ __forceinline__ int problem_of(const Args<MAXP>& a, int gb) {
   int lo = 0, hi = a.nproblems - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (a.p[mid].block_begin <= gb) lo = mid;
     else hi = mid - 1;
   }
+  return lo;
+}
+
+template <int MAXP>
+__device__ __forceinline__ void score_block(const Args<MAXP>& a, int gb, int lo, int lane) {
   const Problem& P = a.p[lo];
   const int c = gb - P.block_begin;
   // squared outputs of the block's 64 rows, every batch row, and squared scales of the
@@ -296,8 +301,10 @@ __global__ void __launch_bounds__(32 * kWarps) score_kernel(const __grid_constan
   pdl_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gb = blockIdx.x * kWarps + warp;
+  if (gb >= a.nblocks) return;
+  const int lo = problem_of(a, gb);  // parameters only: before the wait
   pdl_wait();
-  if (gb < a.nblocks) score_block(a, gb, lane);
+  score_block(a, gb, lo, lane);
 }
 
 template <int MAXP>
@@ -310,16 +317,11 @@ __global__ void __launch_bounds__(32 * kWarps) score_select_kernel(const __grid_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c0 = blockIdx.x * a.chunk, c1 = min(c0 + a.chunk, a.nblocks);
   pdl_wait();
-  for (int gb = c0 + warp; gb < c1; gb += kWarps) score_block(a, gb, lane);
+  for (int gb = c0 + warp; gb < c1; gb += kWarps) score_block(a, gb, problem_of(a, gb), lane);
   __syncthreads();
   if (threadIdx.x == 0) {
-    // the layers overlapping [c0, c1): the first is the last whose block_begin <= c0
-    int lo = 0, hi = a.nproblems - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (a.p[mid].block_begin <= c0) lo = mid;
-      else hi = mid - 1;
-    }
+    // the layers overlapping [c0, c1), from the one holding block c0
+    const int lo = problem_of(a, c0);
     int n = 0;
     for (int p = lo; p < a.nproblems && a.p[p].block_begin < c1; ++p) {
       const int pb = a.p[p].block_begin, nb = a.p[p].out / 64;

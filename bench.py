@@ -1033,11 +1033,12 @@ def run_fl(args, rank, world, local_rank):
 def run_shard(args, rank, world, local_rank):
     """The decode step with the read split over the ranks (strong scaling: the step's total work is
     fixed; each rank reads its byte-balanced share of every layer's blocks, x replicated). Per step:
-    one batched D4 pass over the rank's block ranges; the gate partial of the rank's share of the
-    head's logits (the vocabulary is split with the head's blocks); one all-gather of the partials
-    and the merge on the device, identical on every rank; the D4->D8 residual pass over the rank's
-    ranges, run or skipped on the device by the merged escalate flag; the gate gathered and merged
-    again; one all-gather of the output rows. Device time with CUDA events, max over ranks."""
+    one batched D4 pass over the rank's block ranges that also reduces the rank's share of the
+    head's logits to the gate's partial (the vocabulary is split with the head's blocks); one
+    all-gather of the partials and the merge on the device, identical on every rank; the D4->D8
+    residual pass over the rank's ranges (partial fused too), run or skipped on the device by the
+    merged escalate flag; its partials gathered and merged again; one all-gather of the output
+    rows. Device time with CUDA events, max over ranks."""
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -1088,29 +1089,26 @@ def run_shard(args, rank, world, local_rank):
     gates = torch.zeros(8, dtype=torch.int32, device="cuda")
     esc = gates[4:5].view(torch.uint8)[0:1]
     runs = torch.zeros(1, dtype=torch.int32, device="cuda")
-    # the conditional residual launch carries a fused gate over the rank's own head rows; its
-    # outputs go to scratch (the step's gate is the merged one)
+    # each pass reduces the rank's head rows to the gate's partial in its own launch (the fused
+    # gate in partial mode); the partials are gathered and merged into the step's gate
     gsz = fl.fl_gemv_gate_workspace_bytes(1)
     gws = torch.zeros(gsz, dtype=torch.uint8, device="cuda")
-    scratch = torch.zeros(8, dtype=torch.int32, device="cuda")
-    spec_local = fl.gate_spec(h_idx, 1e30, -1.0, scratch[0:1].view(torch.float32), scratch[1:2].view(torch.float32),
-                              scratch[2:4], scratch[4:5].view(torch.uint8)[0:1], gws, gsz)
+    spec_p = fl.gate_spec(h_idx, 0.0, 0.0, None, None, None, None, gws, gsz)
     tau = [1e30, -1.0]
 
-    def gate():
-        fl.fl_logit_gate_partial(y_local[h_off:h_off + h_rows], h_rows, 1, h_first, part)
+    def merge():
         allp = shard.gather_partials(part, world, out=p_all)
         fl.fl_logit_gate_merge(allp, world, 1, tau[0], tau[1], gates[0:1].view(torch.float32),
                                gates[1:2].view(torch.float32), gates[2:4], esc)
 
     def d4(j):
-        fl.fl_gemv_batched(prob_d4[j], n_items, 1, 0)
-        gate()
+        fl.fl_gemv_batched_gate_partial(prob_d4[j], n_items, 1, 0, spec_p, None, None, h_first, part)
+        merge()
 
     def step(j):
         d4(j)
-        fl.fl_gemv_batched_gate_if(prob_r[j], n_items, 1, 1, spec_local, esc, runs)
-        gate()
+        fl.fl_gemv_batched_gate_partial(prob_r[j], n_items, 1, 1, spec_p, esc, runs, h_first, part)
+        merge()
         shard.gather_rows(y_local, counts, out=y_all)
 
     # entropy threshold from the merged D4 gate so NESC of the NS input sets escalate
@@ -1169,7 +1167,7 @@ def run_shard(args, rank, world, local_rank):
                        "rows_per_rank": counts, "escalated_steps": n_esc, "input_sets": NS,
                        "l2": "weights (0.33 GB at D4) larger than L2; input sets rotate"},
             "tokens_per_s": args.steps / t, "clocks": clk.summary(),
-            "gpu_launches": 6 * args.steps}   # D4 pass, residual pass, 2 x (partial + merge); NCCL's not counted
+            "gpu_launches": 4 * args.steps}   # D4 pass, residual pass (partials fused), 2 merges; NCCL's not counted
     print(json.dumps(line), flush=True)
     return 0
 

@@ -418,6 +418,17 @@ typedef struct {
 FL_API fl_status fl_logit_gate_partial(const float* logits, int vocab, int batch, int index_base,
                                        fl_gate_partial* partial, void* stream);
 
+/* The batched pass with the gate fused (fl_gemv_batched_gate, and fl_gemv_batched_gate_if when
+ * run_if is not NULL) that writes, instead of the gate's outputs, the merged partial of the
+ * gate problem's logits per batch row to partial [batch] (device, 16-byte aligned), indices
+ * offset by index_base (index_base + out <= 2^24): a rank's piece of a vocabulary split over
+ * devices, reduced in the launch that computes it. The gate spec's thresholds and output
+ * pointers are not used (they may be NULL); its problem and workspace are. runs as
+ * fl_gemv_batched_gate_if. */
+FL_API fl_status fl_gemv_batched_gate_partial(const fl_gemv_problem* problems, int n, int batch, int mode,
+                                              const fl_gate_spec* gate, const uint8_t* run_if, uint32_t* runs,
+                                              int index_base, fl_gate_partial* partial, void* stream);
+
 /* Merge nparts partials per row, partials laid out [nparts][batch] (the gathered pieces in
  * rank order), in one fixed order (lane l of a warp takes parts l, l + 32, ..., then the lanes
  * merge in a fixed tree), and write entropy / margin / top2 / escalate exactly as fl_logit_gate

@@ -116,3 +116,45 @@ def test_sharded_read_assembles_to_the_whole_layers(env, orc, nranks, mode):
         err = np.abs(y_full[li].astype(np.float64) - yref)
         assert np.all(err <= REL * mass + ABS), (li, float((err / (REL * mass + ABS)).max()))
     fl.fl_device_status()
+
+
+@pytest.mark.parametrize("nparts", [1, 3])
+def test_fused_gate_partials_merge_to_the_whole_row(env, orc, nparts):
+    """The head's logits split into row pieces, each piece its own batched pass with the gate
+    fused in partial mode (the rank's share of the vocabulary reduced in the launch that
+    computes it); the merged partials equal the oracle's gate of the whole row, and the pieces'
+    outputs the oracle's product."""
+    torch, fl, shard = env
+    out, inn = 64 * 47, 512
+    q, s = synth.int8_layer(out, inn, 80)
+    lv = np.full(out // 64, 2, np.uint8)
+    x = synth.bf16_normal((1, inn), 81)
+    store = torch.empty(fl.fl_plane_store_bytes(out, inn), dtype=torch.uint8, device="cuda")
+    fl.fl_pack_planes(dev(torch, q), dev(torch, s), out, inn, store)
+    lvd, xd = dev(torch, lv), dev(torch, x)
+    first = fl.fl_shard_blocks(lv, inn, nparts)
+    y = torch.zeros((1, out), dtype=torch.float32, device="cuda")
+    parts = torch.zeros((nparts, fl.GATE_PARTIAL_BYTES), dtype=torch.uint8, device="cuda")
+    wsb = fl.fl_gemv_gate_workspace_bytes(1)
+    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    spec = fl.gate_spec(0, 0.0, 0.0, None, None, None, None, ws, wsb)
+    for r in range(nparts):
+        b0, b1 = first[r], first[r + 1]
+        if b1 == b0:
+            continue
+        item = (store[b0 * 8448 * (inn // 128):], 64 * (b1 - b0), inn, lvd[b0:], None, xd, y[0, 64 * b0:64 * b1])
+        fl.fl_gemv_batched_gate_partial(fl.gemv_problems([item]), 1, 1, 0, spec, None, None, 64 * b0, parts[r])
+    yref, mass = orc.gemv_depth(q, s, lv, x, with_mass=True)
+    H0, M0, _, _ = orc.logit_gate(yref.astype(np.float32), 1e30, -1.0)
+    tau_h, tau_m = float(H0[0]), float(M0[0]) / 2
+    ent, mar = torch.empty(1, device="cuda"), torch.empty(1, device="cuda")
+    top2, esc = torch.empty((1, 2), dtype=torch.int32, device="cuda"), torch.empty(1, dtype=torch.uint8, device="cuda")
+    fl.fl_logit_gate_merge(parts, nparts, 1, tau_h, tau_m, ent, mar, top2, esc)
+    torch.cuda.synchronize()
+    yg = y.cpu().numpy()
+    assert np.all(np.abs(yg.astype(np.float64) - yref) <= REL * mass + ABS)
+    H, M, t2, _ = orc.logit_gate(yg, tau_h, tau_m)       # the gate of the outputs the passes wrote
+    assert np.array_equal(top2.cpu().numpy(), t2)
+    assert np.allclose(ent.cpu().numpy(), H, rtol=1e-5, atol=0)
+    assert np.allclose(mar.cpu().numpy(), M, rtol=1e-5, atol=1e-7)
+    fl.fl_device_status()

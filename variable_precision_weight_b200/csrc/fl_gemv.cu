@@ -117,6 +117,10 @@ struct Args {
   // (optional) counts the passes that ran
   const uint8_t* run_if;
   uint32_t* runs;
+  // the fused gate's merged record per batch row is written here instead of the gate's outputs
+  // (a rank's piece of a vocabulary split over devices), indices offset by gate_index_base
+  GateRec* gate_partial;
+  int gate_index_base;
   int listed;          // some problem has a block list (units per CTA <= kListCache)
   Problem p[MAXP];
 };
@@ -511,8 +515,15 @@ __device__ __forceinline__ void gate_publish(const Args<MAXP>& a, const GateRec&
     GateRec r = empty_rec();
     for (int c = lane; c < a.gate_ncta; c += 32) r = merge2(r, ldcg_rec(&a.gate_part[(size_t)c * FL_MAX_BATCH + bb]));
     r = warp_merge(r);
-    if (lane == 0)
-      gate_outputs(r, a.tau_h, a.tau_m, a.entropy + bb, a.margin + bb, a.top2 + 2 * bb, a.escalate + bb);
+    if (lane == 0) {
+      if (a.gate_partial) {
+        if (r.i1 != 0x7fffffff) r.i1 += a.gate_index_base;  // no index (an empty piece) stays so
+        if (r.i2 != 0x7fffffff) r.i2 += a.gate_index_base;
+        a.gate_partial[bb] = r;
+      } else {
+        gate_outputs(r, a.tau_h, a.tau_m, a.entropy + bb, a.margin + bb, a.top2 + 2 * bb, a.escalate + bb);
+      }
+    }
   }
   if (lane == 0) *a.gate_ticket = 0u;
 }
@@ -1172,6 +1183,8 @@ static fl_status prepare_single(Args<1>& a, const fl_plane_weight* w, const uint
   a.gate_p = -1;
   a.run_if = nullptr;
   a.runs = nullptr;
+  a.gate_partial = nullptr;
+  a.gate_index_base = 0;
   a.listed = 0;
   Problem& P = a.p[0];
   P.store = w->store;
@@ -1250,7 +1263,8 @@ constexpr size_t kGateWorkspaceBytes = kGateTicketBytes + (size_t)kMaxCtas * FL_
 
 static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int mode, const fl_gate_spec* gate,
                          const uint8_t* run_if, uint32_t* runs, void* stream, const char* what,
-                         const int32_t* const* lists = nullptr, const int* counts = nullptr) {
+                         const int32_t* const* lists = nullptr, const int* counts = nullptr,
+                         fl_gate_partial* partial = nullptr, int index_base = 0) {
   if (!problems) return fail(FL_ERR_ARG, "%s: problems is NULL", what);
   if (n < 1 || n > FL_MAX_PROBLEMS) return fail(FL_ERR_ARG, "%s: n=%d (1..%d)", what, n, FL_MAX_PROBLEMS);
   if (mode != 0 && mode != 1) return fail(FL_ERR_ARG, "%s: mode=%d (0 depth, 1 residual)", what, mode);
@@ -1262,6 +1276,8 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
   a.gate_p = -1;
   a.run_if = run_if;
   a.runs = runs;
+  a.gate_partial = reinterpret_cast<GateRec*>(partial);
+  a.gate_index_base = index_base;
   a.listed = lists != nullptr ? 1 : 0;
   if (reinterpret_cast<uintptr_t>(runs) & 3u) return fail(FL_ERR_ALIGN, "%s: runs not 4-byte aligned", what);
   if (lists != nullptr && (counts == nullptr || gate != nullptr))
@@ -1270,14 +1286,17 @@ static fl_status batched(const fl_gemv_problem* problems, int n, int batch, int 
   if (gate) {
     if (gate->problem < 0 || gate->problem >= n)
       return fail(FL_ERR_ARG, "%s: gate problem %d not in 0..%d", what, gate->problem, n - 1);
-    if (!gate->entropy || !gate->margin || !gate->top2 || !gate->escalate || !gate->workspace)
+    if ((!partial && (!gate->entropy || !gate->margin || !gate->top2 || !gate->escalate)) || !gate->workspace)
       return fail(FL_ERR_ARG, "%s: gate output or workspace pointer is NULL", what);
+    if (partial && (!aligned16(partial) || index_base < 0 ||
+                    (long long)index_base + problems[gate->problem].w.out > (1LL << 24)))
+      return fail(FL_ERR_ARG, "%s: partial must be 16-byte aligned, index_base + out below 2^24", what);
     if (gate->workspace_bytes < kGateWorkspaceBytes)
       return fail(FL_ERR_WORKSPACE, "%s: gate workspace %zu bytes, need %zu", what, gate->workspace_bytes,
                   kGateWorkspaceBytes);
     if (!aligned16(gate->workspace)) return fail(FL_ERR_ALIGN, "%s: gate workspace not 16-byte aligned", what);
-    if ((reinterpret_cast<uintptr_t>(gate->entropy) | reinterpret_cast<uintptr_t>(gate->margin) |
-         reinterpret_cast<uintptr_t>(gate->top2)) & 3u)
+    if (!partial && ((reinterpret_cast<uintptr_t>(gate->entropy) | reinterpret_cast<uintptr_t>(gate->margin) |
+                      reinterpret_cast<uintptr_t>(gate->top2)) & 3u))
       return fail(FL_ERR_ALIGN, "%s: gate entropy, margin and top2 must be 4-byte aligned", what);
     a.gate_p = gate->problem;
     a.tau_h = gate->tau_h;
@@ -1381,6 +1400,18 @@ extern "C" fl_status fl_gemv_batched_gate_if(const fl_gemv_problem* problems, in
   if (!gate) return fail(FL_ERR_ARG, "%s: gate spec is NULL", what);
   if (!run_if) return fail(FL_ERR_ARG, "%s: run_if is NULL", what);
   return gemv::batched(problems, n, batch, mode, gate, run_if, runs, stream, what);
+}
+
+extern "C" fl_status fl_gemv_batched_gate_partial(const fl_gemv_problem* problems, int n, int batch, int mode,
+                                                  const fl_gate_spec* gate, const uint8_t* run_if, uint32_t* runs,
+                                                  int index_base, fl_gate_partial* partial, void* stream) {
+  const char* what = "fl_gemv_batched_gate_partial";
+  if (!gate) return fail(FL_ERR_ARG, "%s: gate spec is NULL", what);
+  if (!partial) return fail(FL_ERR_ARG, "%s: partial is NULL", what);
+  if (gate->problem < 0 || gate->problem >= n || !problems)
+    return fail(FL_ERR_ARG, "%s: gate problem %d not in 0..%d", what, gate->problem, n - 1);
+  return gemv::batched(problems, n, batch, mode, gate, run_if, runs, stream, what, nullptr, nullptr, partial,
+                       index_base);
 }
 
 // ---------------------------------------------------------------- failure detection

@@ -95,6 +95,8 @@ _sigs = {
     "fl_gemv_gate_workspace_bytes": (_S, [_I]),
     "fl_gemv_batched_gate": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, C.POINTER(fl_gate_spec), _P]),
     "fl_gemv_batched_gate_if": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, C.POINTER(fl_gate_spec), _P, _P, _P]),
+    "fl_gemv_batched_gate_partial": (_I, [C.POINTER(fl_gemv_problem), _I, _I, _I, C.POINTER(fl_gate_spec), _P, _P, _I,
+                                          _P, _P]),
     "fl_logit_gate": (_I, [_P, _I, _I, _F, _F, _P, _P, _P, _P, _P]),
     "fl_kquant_bytes": (_S, [_I, _I, _I]),
     "fl_kquant_workspace_bytes": (_S, [_I, _I, _I, _I]),
@@ -249,6 +251,12 @@ def fl_gemv_batched_gate_if(problems, n: int, batch: int, mode: int, gate: fl_ga
                             stream=None) -> None:
     _check(_lib.fl_gemv_batched_gate_if(problems, n, batch, mode, C.byref(gate), _ptr(run_if), _ptr(runs),
                                         _stream(stream)))
+
+
+def fl_gemv_batched_gate_partial(problems, n: int, batch: int, mode: int, gate: fl_gate_spec, run_if, runs,
+                                 index_base: int, partial, stream=None) -> None:
+    _check(_lib.fl_gemv_batched_gate_partial(problems, n, batch, mode, C.byref(gate), _ptr(run_if), _ptr(runs),
+                                             index_base, _ptr(partial), _stream(stream)))
 
 
 def fl_logit_gate(logits, vocab: int, batch: int, tau_h: float, tau_m: float, entropy, margin, top2, escalate,
